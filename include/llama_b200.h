@@ -1,0 +1,235 @@
+/*
+ * llama_b200.h -- C ABI of the B200 (sm_100a) LLaMA-style decoder-block library.
+ *
+ * The library computes the forward pass of a pre-norm decoder block, in
+ * prefill (a whole prompt chunk at once) and KV-cached decode (one new token
+ * per sequence), and optionally of a whole model (embedding, N blocks, final
+ * norm, lm_head, greedy argmax).  Pages cited below by title:
+ *
+ *   [MLX-13B]  "iOS设备上运行LLaMA2-13B：基于苹果MLX框架的完整技术指南"
+ *   [DeepDive] "LLaMA架构深度解析：从开源大模型设计到高效推理的工程实现全流程",
+ *              section 二 "LLaMA架构组件"
+ *   [Decoder]  "老码农和你一起学AI系列：关于LLaMA解码器"
+ *   [HandsOn]  "《Hands-On Large Language Models》阅读笔记(二)"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  The caller owns ALL memory.  Every pointer named "device" is CUDA
+ *   device memory on the current device; the library never allocates device
+ *   memory and never frees what it is given.  Every device pointer must be
+ *   16-byte aligned (LLAMA_ERR_ALIGNMENT otherwise).
+ * Layout.  Row-major everywhere.  A Linear weight is [out_features, in_features]
+ *   and computes y = x W^T with no bias ([DeepDive] nn.Linear(..., bias=False);
+ *   [MLX-13B] module tree).  The residual stream x is float32 [tokens, dim],
+ *   token t of sequence b at row b*seq_len + t.  Norm weights are float32 [dim].
+ *   Projection weights, the embedding and lm_head are `dims.dtype`.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  All work is enqueued on it; no call synchronises, except
+ *   llama_device_status.
+ * Errors.  Calls return a llama_status and never throw.  Argument checks run
+ *   before anything is enqueued; on failure nothing is enqueued and the cache
+ *   length is unchanged.  Device-side failures (a bounded wait that ran out)
+ *   are recorded in a status word at the start of the workspace and read with
+ *   llama_device_status after the caller synchronises the stream.
+ * Concurrency.  Two calls that share a workspace or a cache must not overlap
+ *   on the GPU (enqueue them on one stream).
+ */
+#ifndef LLAMA_B200_H
+#define LLAMA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LLAMA_B200_ABI_VERSION 1
+
+typedef enum llama_status {
+  LLAMA_OK = 0,
+  LLAMA_ERR_INVALID_ARG = 1,         /* null pointer, bad size, bad enum, aliasing */
+  LLAMA_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. head_dim 48) */
+  LLAMA_ERR_CACHE_FULL = 3,          /* length + new tokens > capacity */
+  LLAMA_ERR_ALIGNMENT = 4,           /* a device pointer is not 16-byte aligned */
+  LLAMA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < the *_workspace_size query */
+  LLAMA_ERR_CUDA = 6,                /* a CUDA runtime/driver call failed */
+  LLAMA_ERR_DEVICE_TIMEOUT = 7       /* a bounded device wait ran out (read via llama_device_status) */
+} llama_status;
+
+/* RoPE variant.  HALF: rotate-half, x*cos(emb) + cat(-x2, x1)*sin(emb) with
+ * emb = cat(freqs, freqs) ([DeepDive] class LLaMARoPE).  INTERLEAVED: the
+ * "traditional" variant named in [MLX-13B] "LLaMA 2 的结构分析"
+ * (RoPE(128, traditional=True)); read as adjacent pairs (x[2i], x[2i+1])
+ * rotated by p * theta^(-2i/head_dim). */
+typedef enum llama_rope_style { LLAMA_ROPE_HALF = 0, LLAMA_ROPE_INTERLEAVED = 1 } llama_rope_style;
+
+/* Storage / operand type of weights, projections and the KV cache.
+ * LLAMA_F32: every operand fp32, CUDA-core arithmetic (no TF32).
+ * LLAMA_BF16: bf16 operands on the tensor cores with fp32 accumulation.
+ * The residual stream is fp32 in both. */
+typedef enum llama_dtype { LLAMA_F32 = 0, LLAMA_BF16 = 1 } llama_dtype;
+
+/* Block hyper-parameters ([MLX-13B] 模型配置 config.json; [DeepDive] LLaMAConfig).
+ * Supported: head_dim in {64, 96, 128} (and 32 for LLAMA_F32);
+ * n_heads % n_kv_heads == 0 (GQA group n_heads/n_kv_heads, query head h
+ * reads KV head h / group, [DeepDive] LLaMAAttention); dim, ffn_dim and
+ * n_heads*head_dim multiples of 8; eps > 0; rope_theta > 1. */
+typedef struct llama_dims {
+  int32_t dim;
+  int32_t n_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t ffn_dim;
+  float eps;
+  float rope_theta;
+  int32_t rope_style; /* llama_rope_style */
+  int32_t dtype;      /* llama_dtype */
+} llama_dims;
+
+/* One block's weights (device pointers, caller-owned).
+ *   attn_norm, ffn_norm : float32 [dim]
+ *   wq [n_heads*head_dim, dim], wk/wv [n_kv_heads*head_dim, dim]   (dtype)
+ *   wo [dim, n_heads*head_dim]                                     (dtype)
+ *   w1 (gate) / w3 (up) [ffn_dim, dim], w2 (down) [dim, ffn_dim]   (dtype)
+ * A fused qkv weight ([HandsOn] Phi-3 qkv_proj [9216, 3072]) is passed as
+ * wq = base, wk = base + nh*hd rows, wv = wk + nkv*hd rows (q, then k, then
+ * v); a fused gate_up weight ([HandsOn] gate_up_proj) as w1 = base,
+ * w3 = base + ffn_dim rows (gate first).  When wq, wk, wv are contiguous in
+ * that order the QKV projection runs as one GEMM. */
+typedef struct llama_layer_weights {
+  const float* attn_norm;
+  const void* wq;
+  const void* wk;
+  const void* wv;
+  const void* wo;
+  const float* ffn_norm;
+  const void* w1;
+  const void* w3;
+  const void* w2;
+} llama_layer_weights;
+
+/* ------------------------------------------------------------------ KV cache */
+
+/* Opaque host object describing one layer's KV cache ([MLX-13B] KV 缓存实现
+ * 片段: new, already-rotated keys and values are appended after the cached
+ * ones along the sequence axis; the next tokens' RoPE positions start at the
+ * current length).  It holds pointers, capacity and length only.  */
+typedef struct llama_kv_cache llama_kv_cache;
+
+/* k_buf, v_buf: caller-owned device buffers, each [batch][n_kv_heads][capacity][head_dim]
+ * of dims->dtype.  The new cache has length 0.
+ * Errors: INVALID_ARG (null, batch/capacity <= 0, bad dims), ALIGNMENT. */
+llama_status llama_kv_cache_create(const llama_dims* dims, int32_t batch, int32_t capacity, void* k_buf,
+                                   void* v_buf, llama_kv_cache** out);
+/* Declare that positions [0, len) of every sequence already hold valid
+ * (rotated) keys and values -- e.g. a synthetic pre-filled cache.
+ * Errors: INVALID_ARG (len < 0), CACHE_FULL (len > capacity). */
+llama_status llama_kv_cache_set_length(llama_kv_cache* cache, int32_t len);
+/* Current length (positions filled), or -1 for a null handle. */
+int32_t llama_kv_cache_length(const llama_kv_cache* cache);
+int32_t llama_kv_cache_capacity(const llama_kv_cache* cache);
+void llama_kv_cache_destroy(llama_kv_cache* cache);
+
+/* ------------------------------------------------------------------ workspace */
+
+/* Bytes of device workspace a layer call with `batch` sequences of up to
+ * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
+ * The workspace is caller-owned scratch; its first 256 bytes hold the
+ * device status word and must be zeroed once before first use. */
+size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_len);
+
+/* Byte offsets, inside the workspace of a layer call with (batch, seq_len),
+ * of the intermediate tensors the call leaves behind, for inspection:
+ *   out[0] qkv   [tokens, (nh + 2 nkv) hd] dtype: q (after RoPE), k (before RoPE), v
+ *   out[1] h     [tokens, dim] dtype: the second RMSNorm's output
+ *   out[2] attn  [tokens, nh hd] dtype: attention output (heads concatenated)
+ *   out[3] m     [tokens, ffn_dim] dtype: silu(gate) * up
+ * Writes min(n, 4) entries.  Errors: INVALID_ARG. */
+llama_status llama_workspace_offsets(const llama_dims* dims, int32_t batch, int32_t seq_len, size_t* out,
+                                     int32_t n);
+
+/* Read (and optionally clear) the device status word at the start of
+ * `workspace`.  Synchronous device-to-host copy: call after the work has
+ * been synchronised.  Returns LLAMA_OK or the first device-side error
+ * (LLAMA_ERR_DEVICE_TIMEOUT); LLAMA_ERR_CUDA if the copy itself fails. */
+llama_status llama_device_status(const void* workspace, int32_t clear);
+
+/* ------------------------------------------------------------------ layer calls */
+
+/* Prefill: one decoder block over `seq_len` new tokens of each of `batch`
+ * sequences, positions cache.length .. cache.length+seq_len-1 (chunked
+ * prefill when the cache is not empty: query p sees keys 0..p).
+ *   h   = attn_norm * x / sqrt(mean(x^2) + eps)        [MLX-13B] 4. RMSNorm; [DeepDive] LLaMARMSNorm
+ *   q,k,v = h Wq^T, h Wk^T, h Wv^T; RoPE on q and k     [DeepDive] LLaMAAttention, LLaMARoPE
+ *   cache <- append(k, v)                               [MLX-13B] KV 缓存实现片段
+ *   o   = softmax(q k^T / sqrt(hd), causal) v, GQA     [MLX-13B] 2. 注意力机制, 5. 因果掩码
+ *   x1  = x + o Wo^T                                    [DeepDive] LLaMABlock
+ *   x_out = x1 + W2(silu(h2 W1^T) * (h2 W3^T)), h2 = ffn_norm-RMSNorm(x1)
+ *                                                        [MLX-13B] 3. 前馈网络; [Decoder] 数据流动
+ * x_in, x_out: device float32 [batch*seq_len, dim]; they must not overlap.
+ * The cache length advances by seq_len when the call is enqueued.
+ * Errors: INVALID_ARG (null, bad sizes, batch != cache batch, aliasing),
+ *   UNSUPPORTED, ALIGNMENT, CACHE_FULL, WORKSPACE_TOO_SMALL, CUDA. */
+llama_status llama_layer_prefill(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                 int32_t batch, int32_t seq_len, const float* x_in, float* x_out, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* Decode: the same block for ONE new token per sequence at position
+ * cache.length ([HandsOn] 第三章: decode reads the KV cache and processes
+ * only the new token).  x_in, x_out: device float32 [batch, dim].
+ * Same errors as llama_layer_prefill. */
+llama_status llama_layer_decode(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------ whole model */
+
+/* A whole model ([DeepDive] class LLaMA; [HandsOn] Phi3ForCausalLM tree).
+ *   embed   [vocab, dim] (dtype), final_norm float32 [dim], lm_head [vocab, dim] (dtype)
+ *   layers  HOST array of n_layers weight sets (device pointers inside). */
+typedef struct llama_model {
+  llama_dims dims;
+  int32_t n_layers;
+  int32_t vocab;
+  const void* embed;
+  const float* final_norm;
+  const void* lm_head;
+  const llama_layer_weights* layers;
+} llama_model;
+
+size_t llama_model_workspace_size(const llama_model* model, int32_t batch, int32_t seq_len);
+
+/* Embedding lookup, all blocks (prefill when seq_len > 1 or the caches are
+ * empty, decode otherwise), final RMSNorm, lm_head on the LAST row of each
+ * sequence, greedy argmax ([HandsOn] 第三章: argmax of the last position's
+ * scores; [MLX-13B] 生成过程: temp 0 is argmax).
+ *   caches       HOST array of n_layers cache handles (all the same length)
+ *   tokens       device int32 [batch, seq_len], each in [0, vocab)
+ *   logits_or_null  device float32 [batch, vocab] or NULL
+ *   next_ids     device int32 [batch]; ties resolve to the lowest index
+ * Errors: as llama_layer_prefill. */
+llama_status llama_model_forward(const llama_model* model, llama_kv_cache* const* caches, const int32_t* tokens,
+                                 int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ misc */
+
+const char* llama_status_string(llama_status s);
+int32_t llama_abi_version(void);
+
+/* Upper bound, in nanoseconds, on every device-side wait of later launches
+ * (default 2e9).  A test may lower it.  Returns the previous value. */
+uint64_t llama_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the failure path: launches one CTA that waits on an
+ * mbarrier nothing will ever arrive on, with a limit of `limit_ns`; the wait
+ * runs out, the kernel records LLAMA_ERR_DEVICE_TIMEOUT in the workspace
+ * status word and returns.  No page counterpart: failure detection only. */
+llama_status llama_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_B200_H */

@@ -1,0 +1,224 @@
+"""Python binding of the B200 decoder-block library (argument marshalling only).
+
+Every call goes through the C ABI declared in ``include/llama_b200.h`` and
+implemented by ``libllama_b200.so`` (built in-tree by ``build.py``).  There is
+no fallback: if the library is missing or cannot be loaded, every entry point
+raises ``LlamaError``.  PyTorch is used only to own device memory and to name
+the CUDA stream.
+
+The ``llama_*`` functions mirror the C names one to one and take raw
+pointers / integers; the lower-case helpers (``layer_prefill`` ...) accept
+torch tensors and pass their ``data_ptr()``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB
+
+__all__ = [
+    "LlamaError", "Dims", "LayerWeights", "Model", "lib", "EXPORTS",
+    "F32", "BF16", "ROPE_HALF", "ROPE_INTERLEAVED",
+    "make_dims", "layer_weights", "model_struct", "KVCache",
+    "workspace_size", "model_workspace_size", "layer_prefill", "layer_decode",
+    "model_forward", "device_status", "workspace_offsets", "set_wait_limit_ns", "selftest_wait_timeout",
+]
+
+F32, BF16 = 0, 1
+ROPE_HALF, ROPE_INTERLEAVED = 0, 1
+
+STATUS = {
+    0: "LLAMA_OK", 1: "LLAMA_ERR_INVALID_ARG", 2: "LLAMA_ERR_UNSUPPORTED", 3: "LLAMA_ERR_CACHE_FULL",
+    4: "LLAMA_ERR_ALIGNMENT", 5: "LLAMA_ERR_WORKSPACE_TOO_SMALL", 6: "LLAMA_ERR_CUDA",
+    7: "LLAMA_ERR_DEVICE_TIMEOUT",
+}
+
+
+class LlamaError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = int(status)
+        super().__init__(f"{what}: {STATUS.get(self.status, self.status)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("dim", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("ffn_dim", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("rope_style", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w1", "w3", "w2")]
+
+
+class Model(ctypes.Structure):
+    _fields_ = [("dims", Dims), ("n_layers", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p), ("lm_head", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(LayerWeights))]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_S = ctypes.c_size_t
+_U64 = ctypes.c_uint64
+_DP = ctypes.POINTER(Dims)
+_WP = ctypes.POINTER(LayerWeights)
+_MP = ctypes.POINTER(Model)
+
+# name -> (restype, argtypes); the full export list of include/llama_b200.h
+EXPORTS = {
+    "llama_abi_version": (_I, []),
+    "llama_status_string": (ctypes.c_char_p, [_I]),
+    "llama_set_wait_limit_ns": (_U64, [_U64]),
+    "llama_kv_cache_create": (_I, [_DP, _I, _I, _P, _P, ctypes.POINTER(_P)]),
+    "llama_kv_cache_set_length": (_I, [_P, _I]),
+    "llama_kv_cache_length": (_I, [_P]),
+    "llama_kv_cache_capacity": (_I, [_P]),
+    "llama_kv_cache_destroy": (None, [_P]),
+    "llama_workspace_size": (_S, [_DP, _I, _I]),
+    "llama_device_status": (_I, [_P, _I]),
+    "llama_workspace_offsets": (_I, [_DP, _I, _I, ctypes.POINTER(_S), _I]),
+    "llama_layer_prefill": (_I, [_DP, _WP, _P, _I, _I, _P, _P, _P, _S, _P]),
+    "llama_layer_decode": (_I, [_DP, _WP, _P, _I, _P, _P, _P, _S, _P]),
+    "llama_model_workspace_size": (_S, [_MP, _I, _I]),
+    "llama_model_forward": (_I, [_MP, ctypes.POINTER(_P), _P, _I, _I, _P, _P, _P, _S, _P]),
+    "llama_selftest_wait_timeout": (_I, [_P, _U64, _P]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises ``LlamaError`` if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise LlamaError(6, f"CUDA library not built ({LIB}); run python -m llama_decoder_only_b200.build")
+        handle = ctypes.CDLL(LIB)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status, what):
+    if status != 0:
+        raise LlamaError(status, what)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+# ------------------------------------------------------------------ structures
+
+def make_dims(dim, n_heads, n_kv_heads, head_dim, ffn_dim, eps, rope_theta=10000.0,
+              rope_style=ROPE_HALF, dtype=BF16):
+    if isinstance(rope_style, str):
+        rope_style = ROPE_HALF if rope_style == "half" else ROPE_INTERLEAVED
+    if isinstance(dtype, str):
+        dtype = BF16 if dtype == "bf16" else F32
+    return Dims(dim, n_heads, n_kv_heads, head_dim, ffn_dim, eps, rope_theta, rope_style, dtype)
+
+
+def layer_weights(t):
+    """``LayerWeights`` from a dict of device tensors (keys attn_norm, wq, ... w2)."""
+    return LayerWeights(*[_ptr(t[k]) for k in
+                          ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w1", "w3", "w2")])
+
+
+def model_struct(dims, embed, final_norm, lm_head, layers):
+    """``Model`` struct plus the ctypes array that must stay alive with it."""
+    arr = (LayerWeights * len(layers))(*[layer_weights(w) for w in layers])
+    m = Model(dims, len(layers), embed.shape[0], _ptr(embed), _ptr(final_norm), _ptr(lm_head),
+              ctypes.cast(arr, ctypes.POINTER(LayerWeights)))
+    return m, arr
+
+
+class KVCache:
+    """One layer's cache: device buffers (torch-owned) plus the library handle."""
+
+    def __init__(self, dims, batch, capacity, device="cuda", k=None, v=None):
+        import torch
+        dt = torch.bfloat16 if dims.dtype == BF16 else torch.float32
+        shape = (batch, dims.n_kv_heads, capacity, dims.head_dim)
+        self.k = k if k is not None else torch.zeros(shape, dtype=dt, device=device)
+        self.v = v if v is not None else torch.zeros(shape, dtype=dt, device=device)
+        h = ctypes.c_void_p()
+        _check(lib().llama_kv_cache_create(ctypes.byref(dims), batch, capacity, _ptr(self.k), _ptr(self.v),
+                                           ctypes.byref(h)), "llama_kv_cache_create")
+        self.handle = h
+        self.batch, self.capacity = batch, capacity
+
+    @property
+    def length(self):
+        return lib().llama_kv_cache_length(self.handle)
+
+    def set_length(self, n):
+        _check(lib().llama_kv_cache_set_length(self.handle, n), "llama_kv_cache_set_length")
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and _lib is not None:
+            _lib.llama_kv_cache_destroy(h)
+            self.handle = None
+
+
+# ------------------------------------------------------------------ calls
+
+def workspace_size(dims, batch, seq_len):
+    return lib().llama_workspace_size(ctypes.byref(dims), batch, seq_len)
+
+
+def model_workspace_size(model, batch, seq_len):
+    return lib().llama_model_workspace_size(ctypes.byref(model), batch, seq_len)
+
+
+def layer_prefill(dims, w, cache, batch, seq_len, x_in, x_out, ws, stream=None):
+    _check(lib().llama_layer_prefill(ctypes.byref(dims), ctypes.byref(w), cache.handle, batch, seq_len,
+                                     _ptr(x_in), _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream)), "llama_layer_prefill")
+
+
+def layer_decode(dims, w, cache, batch, x_in, x_out, ws, stream=None):
+    _check(lib().llama_layer_decode(ctypes.byref(dims), ctypes.byref(w), cache.handle, batch, _ptr(x_in),
+                                    _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "llama_layer_decode")
+
+
+def model_forward(model, caches, tokens, batch, seq_len, logits, next_ids, ws, stream=None):
+    arr = (ctypes.c_void_p * len(caches))(*[c.handle.value for c in caches])
+    _check(lib().llama_model_forward(ctypes.byref(model), arr, _ptr(tokens), batch, seq_len, _ptr(logits),
+                                     _ptr(next_ids), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "llama_model_forward")
+
+
+def workspace_offsets(dims, batch, seq_len):
+    """Offsets (bytes) of qkv, h, attn and m inside a layer call's workspace."""
+    out = (_S * 4)()
+    _check(lib().llama_workspace_offsets(ctypes.byref(dims), batch, seq_len, out, 4), "llama_workspace_offsets")
+    return list(out)
+
+
+def device_status(ws, clear=False):
+    return lib().llama_device_status(_ptr(ws), 1 if clear else 0)
+
+
+def set_wait_limit_ns(ns):
+    return lib().llama_set_wait_limit_ns(int(ns))
+
+
+def selftest_wait_timeout(ws, limit_ns, stream=None):
+    _check(lib().llama_selftest_wait_timeout(_ptr(ws), int(limit_ns), _stream(stream)),
+           "llama_selftest_wait_timeout")

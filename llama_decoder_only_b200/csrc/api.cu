@@ -1,0 +1,773 @@
+// C-ABI host library: argument checks, workspace layout, tensor maps and the
+// launch sequence of one decoder block (prefill / decode) and of a whole
+// model.  Every step of the block runs in the kernels of this library; the
+// host only validates, plans and enqueues.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "f32_path.cuh"
+#include "gemm_tc.cuh"
+#include "small_kernels.cuh"
+
+using namespace llama;
+
+struct llama_kv_cache {
+  llama_dims dims;
+  int32_t batch;
+  int32_t capacity;
+  int32_t length;
+  void* k;
+  void* v;
+};
+
+namespace {
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+constexpr int kMaxSkGrid = 192;     // upper bound on stream-K CTAs (workspace sizing)
+constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
+constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K form up to here
+
+#define CUDA_TRY(x)                           \
+  do {                                        \
+    if ((x) != cudaSuccess) {                 \
+      (void)cudaGetLastError();               \
+      return LLAMA_ERR_CUDA;                  \
+    }                                         \
+  } while (0)
+
+#define LAUNCH_CHECK()                        \
+  do {                                        \
+    if (cudaGetLastError() != cudaSuccess) return LLAMA_ERR_CUDA; \
+  } while (0)
+
+#define TRY(x)                                \
+  do {                                        \
+    llama_status _s = (x);                    \
+    if (_s != LLAMA_OK) return _s;            \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// ------------------------------------------------------------------ driver entry point for tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
+// dims[0] is the contiguous dimension; strides are in bytes for dims 1..rank-1.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t d[5], s[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides[i];
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s, bx, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[2] = {inner, rows};
+  const uint64_t strides[1] = {inner * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return make_map(m, base, 2, dims, strides, box);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+// ------------------------------------------------------------------ validation
+
+llama_status check_dims(const llama_dims* d) {
+  if (d == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (d->dim <= 0 || d->n_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 || d->ffn_dim <= 0)
+    return LLAMA_ERR_INVALID_ARG;
+  if (d->n_heads % d->n_kv_heads != 0) return LLAMA_ERR_INVALID_ARG;
+  if (!(d->eps > 0.f) || !(d->eps < 1.f)) return LLAMA_ERR_INVALID_ARG;
+  if (!(d->rope_theta > 1.f) || !(d->rope_theta < 1e30f)) return LLAMA_ERR_INVALID_ARG;
+  if (d->rope_style != LLAMA_ROPE_HALF && d->rope_style != LLAMA_ROPE_INTERLEAVED) return LLAMA_ERR_INVALID_ARG;
+  if (d->dtype != LLAMA_F32 && d->dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (d->dim % 8 || d->ffn_dim % 8) return LLAMA_ERR_UNSUPPORTED;
+  const int hd = d->head_dim;
+  if (d->dtype == LLAMA_BF16) {
+    if (hd != 64 && hd != 96 && hd != 128) return LLAMA_ERR_UNSUPPORTED;
+    const int grp = d->n_heads / d->n_kv_heads;
+    if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return LLAMA_ERR_UNSUPPORTED;
+  } else {
+    if (hd != 32 && hd != 64 && hd != 96 && hd != 128) return LLAMA_ERR_UNSUPPORTED;
+  }
+  return LLAMA_OK;
+}
+
+bool same_dims(const llama_dims& a, const llama_dims& b) { return std::memcmp(&a, &b, sizeof(llama_dims)) == 0; }
+
+llama_status check_weights(const llama_layer_weights* w) {
+  if (w == nullptr) return LLAMA_ERR_INVALID_ARG;
+  const void* ps[9] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->ffn_norm, w->w1, w->w3, w->w2};
+  for (const void* p : ps)
+    if (p == nullptr) return LLAMA_ERR_INVALID_ARG;
+  for (const void* p : ps)
+    if (!aligned16(p)) return LLAMA_ERR_ALIGNMENT;
+  return LLAMA_OK;
+}
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// ------------------------------------------------------------------ workspace layout
+
+struct WsLayout {
+  size_t qkv, h, attn, mbuf, partial, att_ml, att_o;        // layer scratch
+  size_t xa, xb, xl, hl, logits;                            // model scratch
+  size_t total;
+};
+
+int swap_bn(int tokens) { return tokens <= 16 ? 16 : tokens <= 32 ? 32 : tokens <= 64 ? 64 : 128; }
+
+// Bound on the stream-K partial buffer of one decode GEMM (floats).
+size_t sk_partial_floats(int n_rows_total, int tokens) {
+  const long long n_tiles = cdiv(n_rows_total, 128) + 3;  // + segment padding
+  return (size_t)(n_tiles + 3LL * kMaxSkGrid) * swap_bn(tokens) * 128;
+}
+
+WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
+  WsLayout w{};
+  const size_t es = d.dtype == LLAMA_BF16 ? 2 : 4;
+  const size_t M = (size_t)batch * seq_len;
+  const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
+  size_t off = 256;  // status word
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  w.qkv = take(M * qkvn * es);
+  w.h = take(M * (size_t)d.dim * es);
+  w.attn = take(M * (size_t)d.n_heads * d.head_dim * es);
+  w.mbuf = take(M * (size_t)d.ffn_dim * es);
+  size_t pf = 0;
+  if (d.dtype == LLAMA_BF16 && batch <= kSwapMaxTokens) {
+    // decode GEMMs (M = batch) and the lm_head on the last rows (M = batch)
+    pf = sk_partial_floats(qkvn, batch);
+    pf = std::max(pf, sk_partial_floats(d.dim, batch));
+    pf = std::max(pf, sk_partial_floats(2 * d.ffn_dim, batch));
+    if (vocab > 0) pf = std::max(pf, sk_partial_floats(vocab, batch));
+  }
+  w.partial = take(pf * 4);
+  w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
+  w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
+  if (vocab > 0) {
+    w.xa = take(M * (size_t)d.dim * 4);
+    w.xb = take(M * (size_t)d.dim * 4);
+    w.xl = take((size_t)batch * d.dim * 4);
+    w.hl = take((size_t)batch * d.dim * es);
+    w.logits = take((size_t)batch * vocab * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// ------------------------------------------------------------------ GEMM launchers (bf16, tcgen05)
+
+struct WSeg {
+  const void* ptr;
+  int rows;
+  int col0;
+};
+
+template <int BN, bool SWAP, int EPI>
+llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
+                            cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES));
+    attr_set = true;
+  }
+  gemm_tc_kernel<BN, SWAP, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(a, w[0], w[1], w[2], p);
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+// Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
+llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
+                          void* out, int ldo, const float* resid, int ldr, DevStatus* status) {
+  constexpr int BN = 256;
+  GemmParams p{};
+  p.K = K;
+  p.num_kb = cdiv(K, 64);
+  p.act_rows = M;
+  p.m_tiles = cdiv(M, 128);
+  p.nseg = nseg;
+  p.out = out;
+  p.ldo = ldo;
+  p.resid = resid;
+  p.ldr = ldr;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  CUtensorMap ta, tw[3];
+  std::memset(tw, 0, sizeof(tw));
+  if (!make_map_2d(&ta, act, K, M, 128)) return LLAMA_ERR_CUDA;
+  if (epi == EPI_SWIGLU_BF16) {
+    // segs[0] = gate (w1), segs[1] = up (w3), both [ffn, K]; one tile = 128 gate + 128 up rows
+    p.nseg = 2;
+    p.seg_rows[0] = segs[0].rows;
+    p.seg_tile0[0] = 0;
+    p.n_tiles = cdiv(segs[0].rows, BN / 2);
+    p.seg_tile0[1] = p.n_tiles;
+    p.seg_tile0[2] = p.n_tiles;
+    p.seg_tile0[3] = p.n_tiles;
+    if (!make_map_2d(&tw[0], segs[0].ptr, K, segs[0].rows, BN / 2)) return LLAMA_ERR_CUDA;
+    if (!make_map_2d(&tw[1], segs[1].ptr, K, segs[1].rows, BN / 2)) return LLAMA_ERR_CUDA;
+    tw[2] = tw[1];
+  } else {
+    int t = 0;
+    for (int s = 0; s < nseg; ++s) {
+      p.seg_rows[s] = segs[s].rows;
+      p.seg_col0[s] = segs[s].col0;
+      p.seg_tile0[s] = t;
+      t += cdiv(segs[s].rows, BN);
+      if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, BN)) return LLAMA_ERR_CUDA;
+    }
+    for (int s = nseg; s < 3; ++s) tw[s] = tw[0];
+    for (int s = nseg; s < 4; ++s) p.seg_tile0[s] = t;
+    p.n_tiles = t;
+  }
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = std::min(tiles, num_sms());
+  switch (epi) {
+    case EPI_BF16:
+      return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st);
+    case EPI_RESID_F32:
+      return launch_gemm_tc<BN, false, EPI_RESID_F32>(ta, tw, p, grid, st);
+    case EPI_SWIGLU_BF16:
+      return launch_gemm_tc<BN, false, EPI_SWIGLU_BF16>(ta, tw, p, grid, st);
+    case EPI_F32:
+      return launch_gemm_tc<BN, false, EPI_F32>(ta, tw, p, grid, st);
+  }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+// Stream-K (decode) GEMM: partials = act[M, K] · W^T with W as the MMA's A
+// operand, then the reduce kernel applies `dec_epi`.
+llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int dec_epi,
+                         void* out, int ldo, const float* resid, int ldr, float* partial, DevStatus* status) {
+  const int BN = swap_bn(M);
+  GemmParams p{};
+  p.K = K;
+  p.num_kb = cdiv(K, 64);
+  p.act_rows = M;
+  p.m_tiles = 1;
+  p.nseg = nseg;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  p.partial = partial;
+  CUtensorMap ta, tw[3];
+  std::memset(tw, 0, sizeof(tw));
+  if (!make_map_2d(&ta, act, K, M, BN)) return LLAMA_ERR_CUDA;
+  int t = 0;
+  int n_out = 0;
+  for (int s = 0; s < nseg; ++s) {
+    p.seg_rows[s] = segs[s].rows;
+    p.seg_col0[s] = segs[s].col0;
+    p.seg_tile0[s] = t;
+    t += cdiv(segs[s].rows, 128);
+    n_out = std::max(n_out, segs[s].col0 + segs[s].rows);
+    if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, 128)) return LLAMA_ERR_CUDA;
+  }
+  for (int s = nseg; s < 3; ++s) tw[s] = tw[0];
+  for (int s = nseg; s < 4; ++s) p.seg_tile0[s] = t;
+  p.n_tiles = t;
+  p.units = (long long)p.n_tiles * p.num_kb;
+  const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
+  const long long per = (p.units + grid - 1) / grid;
+  p.max_pieces = (int)((per + p.num_kb - 1) / p.num_kb) + 1;
+  llama_status s = LLAMA_OK;
+  switch (BN) {
+    case 16: s = launch_gemm_tc<16, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
+    case 32: s = launch_gemm_tc<32, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
+    case 64: s = launch_gemm_tc<64, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
+    default: s = launch_gemm_tc<128, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
+  }
+  if (s != LLAMA_OK) return s;
+  ReduceParams r{};
+  r.act_rows = M;
+  r.num_kb = p.num_kb;
+  r.units = p.units;
+  r.grid = grid;
+  r.max_pieces = p.max_pieces;
+  r.BN = BN;
+  r.nseg = nseg;
+  for (int i = 0; i < 3; ++i) {
+    r.seg_rows[i] = p.seg_rows[i];
+    r.seg_col0[i] = p.seg_col0[i];
+  }
+  for (int i = 0; i < 4; ++i) r.seg_tile0[i] = p.seg_tile0[i];
+  r.partial = partial;
+  r.out = out;
+  r.ldo = ldo;
+  r.resid = resid;
+  r.ldr = ldr;
+  if (dec_epi == DEC_SWIGLU_BF16) {
+    r.ffn = segs[0].rows;
+    n_out = segs[0].rows;
+  }
+  r.n_out = n_out;
+  dim3 grid_r(cdiv(n_out, 256), M);
+  switch (dec_epi) {
+    case DEC_BF16: splitk_reduce_kernel<DEC_BF16><<<grid_r, 256, 0, st>>>(r); break;
+    case DEC_RESID_F32: splitk_reduce_kernel<DEC_RESID_F32><<<grid_r, 256, 0, st>>>(r); break;
+    case DEC_SWIGLU_BF16: splitk_reduce_kernel<DEC_SWIGLU_BF16><<<grid_r, 256, 0, st>>>(r); break;
+    default: splitk_reduce_kernel<DEC_F32><<<grid_r, 256, 0, st>>>(r); break;
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+// Prefill-or-decode dispatch of one projection.
+llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
+                       int epi, void* out, int ldo, const float* resid, int ldr, float* partial,
+                       DevStatus* status) {
+  if (decode && M <= kSwapMaxTokens) {
+    const int dec = epi == EPI_BF16 ? DEC_BF16 : epi == EPI_RESID_F32 ? DEC_RESID_F32
+                  : epi == EPI_SWIGLU_BF16 ? DEC_SWIGLU_BF16 : DEC_F32;
+    WSeg s2[3];
+    for (int i = 0; i < nseg; ++i) s2[i] = segs[i];
+    if (epi == EPI_SWIGLU_BF16) s2[1].col0 = segs[0].rows;  // up rows follow the gate rows
+    return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status);
+  }
+  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status);
+}
+
+// ------------------------------------------------------------------ attention launchers
+
+llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int L, int p0,
+                               const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM));
+    attr_set = true;
+  }
+  const int hd = d.head_dim;
+  const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
+  const int T = p0 + L;
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[3] = {(uint64_t)qkvn, (uint64_t)L, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)qkvn * 2, (uint64_t)L * qkvn * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tq, qkv, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)T, (uint64_t)B * d.n_kv_heads};
+    const uint64_t strides[2] = {(uint64_t)hd * 2, (uint64_t)kv->capacity * hd * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tk, kv->k, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+    if (!make_map(&tv, kv->v, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  }
+  AttnPrefillParams p{};
+  p.L = L;
+  p.p0 = p0;
+  p.nh = d.n_heads;
+  p.nkv = d.n_kv_heads;
+  p.hd = hd;
+  p.n_qtiles = cdiv(L, 128);
+  p.scale_log2 = kLog2e / sqrtf((float)hd);
+  p.out = out;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  dim3 grid(p.n_qtiles, d.n_heads, B);
+  attn_prefill_kernel<<<grid, 192, ATT_SMEM, st>>>(tq, tk, tv, p);
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+template <int HD, int G>
+void launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st) {
+  attn_decode_kernel<HD, G><<<grid, 128, 0, st>>>(p);
+}
+
+llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int T,
+                              const __nv_bfloat16* qkv, __nv_bfloat16* out, float* part_ml, float* part_o) {
+  const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  AttnDecodeParams p{};
+  p.qkv = qkv;
+  p.ld_qkv = (d.n_heads + 2 * d.n_kv_heads) * hd;
+  p.kc = reinterpret_cast<const __nv_bfloat16*>(kv->k);
+  p.vc = reinterpret_cast<const __nv_bfloat16*>(kv->v);
+  p.cap = kv->capacity;
+  p.T = T;
+  p.nh = d.n_heads;
+  p.nkv = d.n_kv_heads;
+  p.scale_log2 = kLog2e / sqrtf((float)hd);
+  p.part_ml = part_ml;
+  p.part_o = part_o;
+  p.out = out;
+  // split the keys so that about 4 CTAs per SM run, with >= 128 keys per split
+  const int base = B * d.n_kv_heads;
+  int splits = cdiv(4 * num_sms(), base);
+  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 128))));
+  int kps = cdiv(T, splits);
+  kps = cdiv(kps, 32) * 32;
+  splits = cdiv(T, kps);
+  p.splits = splits;
+  p.keys_per_split = kps;
+  dim3 grid(splits, d.n_kv_heads, B);
+#define DEC_CASE(HD_, G_) \
+  if (hd == HD_ && grp == G_) launch_attn_decode<HD_, G_>(p, grid, st);
+  DEC_CASE(64, 1) DEC_CASE(64, 2) DEC_CASE(64, 4) DEC_CASE(64, 8)
+  DEC_CASE(96, 1) DEC_CASE(96, 2) DEC_CASE(96, 4) DEC_CASE(96, 8)
+  DEC_CASE(128, 1) DEC_CASE(128, 2) DEC_CASE(128, 4) DEC_CASE(128, 8)
+#undef DEC_CASE
+  LAUNCH_CHECK();
+  if (splits > 1) {
+    attn_decode_combine_kernel<<<dim3(d.n_heads, B), 128, 0, st>>>(part_ml, part_o, out, d.n_heads, hd, splits);
+    LAUNCH_CHECK();
+  }
+  return LLAMA_OK;
+}
+
+// ------------------------------------------------------------------ one block
+
+llama_status check_layer_call(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* kv, int B,
+                              int L, const float* x_in, float* x_out, void* ws, size_t ws_bytes, int vocab) {
+  TRY(check_dims(dims));
+  TRY(check_weights(w));
+  if (kv == nullptr || x_in == nullptr || x_out == nullptr || ws == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (B <= 0 || L <= 0) return LLAMA_ERR_INVALID_ARG;
+  if (!same_dims(*dims, kv->dims) || B != kv->batch) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(ws)) return LLAMA_ERR_ALIGNMENT;
+  const size_t xb = (size_t)B * L * dims->dim * 4;
+  if (overlap(x_in, xb, x_out, xb)) return LLAMA_ERR_INVALID_ARG;
+  if ((long long)kv->length + L > kv->capacity) return LLAMA_ERR_CACHE_FULL;
+  if (ws_bytes < plan_ws(*dims, B, L, vocab).total) return LLAMA_ERR_WORKSPACE_TOO_SMALL;
+  return LLAMA_OK;
+}
+
+// Enqueue one block.  `decode` selects the one-token-per-sequence kernels.
+llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_kv_cache* kv, int B, int L,
+                       const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay, cudaStream_t st) {
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  const int M = B * L;
+  const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+  const int qkvn = (nh + 2 * nkv) * hd;
+  const int p0 = kv->length;
+  const bool decode = (L == 1);
+  const int rows_per_block = 256 / 32;
+  if (d.dtype == LLAMA_BF16) {
+    using bf = __nv_bfloat16;
+    bf* qkv = reinterpret_cast<bf*>(ws + lay.qkv);
+    bf* h = reinterpret_cast<bf*>(ws + lay.h);
+    bf* att = reinterpret_cast<bf*>(ws + lay.attn);
+    bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
+    float* part = reinterpret_cast<float*>(ws + lay.partial);
+    // a2: RMSNorm-1 -> h (bf16)
+    rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    LAUNCH_CHECK();
+    // a3: QKV projection
+    const size_t rb = (size_t)d.dim * 2;  // bytes per weight row
+    WSeg segs[3];
+    int nseg;
+    if (w.wk == (const uint8_t*)w.wq + (size_t)nh * hd * rb && w.wv == (const uint8_t*)w.wk + (size_t)nkv * hd * rb) {
+      segs[0] = {w.wq, qkvn, 0};
+      nseg = 1;
+    } else {
+      segs[0] = {w.wq, nh * hd, 0};
+      segs[1] = {w.wk, nkv * hd, nh * hd};
+      segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
+      nseg = 3;
+    }
+    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status));
+    // a4: RoPE + KV append
+    rope_append_kernel<bf><<<M, 256, 0, st>>>(qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
+                                               p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    LAUNCH_CHECK();
+    // a5 / a6: attention
+    if (decode) {
+      TRY(attn_decode_bf16(st, d, kv, B, p0 + 1, qkv, att, reinterpret_cast<float*>(ws + lay.att_ml),
+                           reinterpret_cast<float*>(ws + lay.att_o)));
+    } else {
+      TRY(attn_prefill_bf16(st, d, kv, B, L, p0, qkv, att, status));
+    }
+    // a7: o_proj + residual -> x_out holds x_mid
+    WSeg so{w.wo, d.dim, 0};
+    TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status));
+    // a8: RMSNorm-2 + gate_up + SiLU·mul
+    rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+    LAUNCH_CHECK();
+    WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
+    TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status));
+    // a9: down + residual (in place on x_out)
+    WSeg sd{w.w2, d.dim, 0};
+    TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status));
+  } else {
+    float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
+    float* h = reinterpret_cast<float*>(ws + lay.h);
+    float* att = reinterpret_cast<float*>(ws + lay.attn);
+    float* mb = reinterpret_cast<float*>(ws + lay.mbuf);
+    const float* wq = static_cast<const float*>(w.wq);
+    const float* wk = static_cast<const float*>(w.wk);
+    const float* wv = static_cast<const float*>(w.wv);
+    auto grid_for = [](int M_, int N_) { return dim3(cdiv(N_, 64), cdiv(M_, 64)); };
+    rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    LAUNCH_CHECK();
+    gemm_f32_kernel<F32_STORE><<<grid_for(M, nh * hd), 256, 0, st>>>(h, d.dim, wq, nullptr, d.dim, M, nh * hd,
+                                                                      d.dim, qkv, qkvn, nullptr, 0);
+    gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(h, d.dim, wk, nullptr, d.dim, M, nkv * hd,
+                                                                       d.dim, qkv + nh * hd, qkvn, nullptr, 0);
+    gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(
+        h, d.dim, wv, nullptr, d.dim, M, nkv * hd, d.dim, qkv + (nh + nkv) * hd, qkvn, nullptr, 0);
+    LAUNCH_CHECK();
+    rope_append_kernel<float><<<M, 256, 0, st>>>(qkv, static_cast<float*>(kv->k), static_cast<float*>(kv->v), L, p0,
+                                                  nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    LAUNCH_CHECK();
+    const int Tmax = p0 + L;
+    const size_t smem = (size_t)Tmax * 4;
+    if (smem > 48 * 1024) {
+      CUDA_TRY(cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      if (smem > 200 * 1024) return LLAMA_ERR_UNSUPPORTED;
+    }
+    attn_f32_kernel<<<dim3(L, nh, B), 128, smem, st>>>(qkv, qkvn, static_cast<const float*>(kv->k),
+                                                       static_cast<const float*>(kv->v), att, L, p0, nh, nkv, hd,
+                                                       kv->capacity);
+    LAUNCH_CHECK();
+    gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(att, nh * hd, static_cast<const float*>(w.wo),
+                                                                   nullptr, nh * hd, M, d.dim, nh * hd, x_out,
+                                                                   d.dim, x_in, d.dim);
+    LAUNCH_CHECK();
+    rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+    gemm_f32_kernel<F32_SWIGLU><<<grid_for(M, d.ffn_dim), 256, 0, st>>>(
+        h, d.dim, static_cast<const float*>(w.w1), static_cast<const float*>(w.w3), d.dim, M, d.ffn_dim, d.dim, mb,
+        d.ffn_dim, nullptr, 0);
+    gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(mb, d.ffn_dim, static_cast<const float*>(w.w2),
+                                                                   nullptr, d.ffn_dim, M, d.dim, d.ffn_dim, x_out,
+                                                                   d.dim, x_out, d.dim);
+    LAUNCH_CHECK();
+  }
+  kv->length = p0 + L;
+  return LLAMA_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+int32_t llama_abi_version(void) { return LLAMA_B200_ABI_VERSION; }
+
+const char* llama_status_string(llama_status s) {
+  switch (s) {
+    case LLAMA_OK: return "ok";
+    case LLAMA_ERR_INVALID_ARG: return "invalid argument";
+    case LLAMA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LLAMA_ERR_CACHE_FULL: return "KV cache full";
+    case LLAMA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case LLAMA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case LLAMA_ERR_CUDA: return "CUDA error";
+    case LLAMA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+uint64_t llama_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns == 0 ? 1 : ns); }
+
+llama_status llama_kv_cache_create(const llama_dims* dims, int32_t batch, int32_t capacity, void* k_buf,
+                                   void* v_buf, llama_kv_cache** out) {
+  if (out == nullptr) return LLAMA_ERR_INVALID_ARG;
+  *out = nullptr;
+  TRY(check_dims(dims));
+  if (batch <= 0 || capacity <= 0 || k_buf == nullptr || v_buf == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(k_buf) || !aligned16(v_buf)) return LLAMA_ERR_ALIGNMENT;
+  auto* c = new (std::nothrow) llama_kv_cache;
+  if (c == nullptr) return LLAMA_ERR_INVALID_ARG;
+  c->dims = *dims;
+  c->batch = batch;
+  c->capacity = capacity;
+  c->length = 0;
+  c->k = k_buf;
+  c->v = v_buf;
+  *out = c;
+  return LLAMA_OK;
+}
+
+llama_status llama_kv_cache_set_length(llama_kv_cache* c, int32_t len) {
+  if (c == nullptr || len < 0) return LLAMA_ERR_INVALID_ARG;
+  if (len > c->capacity) return LLAMA_ERR_CACHE_FULL;
+  c->length = len;
+  return LLAMA_OK;
+}
+
+int32_t llama_kv_cache_length(const llama_kv_cache* c) { return c ? c->length : -1; }
+int32_t llama_kv_cache_capacity(const llama_kv_cache* c) { return c ? c->capacity : -1; }
+void llama_kv_cache_destroy(llama_kv_cache* c) { delete c; }
+
+size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_len) {
+  if (check_dims(dims) != LLAMA_OK || batch <= 0 || seq_len <= 0) return 0;
+  return plan_ws(*dims, batch, seq_len, 0).total;
+}
+
+llama_status llama_workspace_offsets(const llama_dims* dims, int32_t batch, int32_t seq_len, size_t* out,
+                                     int32_t n) {
+  TRY(check_dims(dims));
+  if (batch <= 0 || seq_len <= 0 || out == nullptr || n < 0) return LLAMA_ERR_INVALID_ARG;
+  const WsLayout w = plan_ws(*dims, batch, seq_len, 0);
+  const size_t v[4] = {w.qkv, w.h, w.attn, w.mbuf};
+  for (int i = 0; i < n && i < 4; ++i) out[i] = v[i];
+  return LLAMA_OK;
+}
+
+llama_status llama_device_status(const void* workspace, int32_t clear) {
+  if (workspace == nullptr) return LLAMA_ERR_INVALID_ARG;
+  DevStatus s{};
+  CUDA_TRY(cudaMemcpy(&s, workspace, sizeof(s), cudaMemcpyDeviceToHost));
+  if (clear) {
+    DevStatus z{};
+    CUDA_TRY(cudaMemcpy(const_cast<void*>(workspace), &z, sizeof(z), cudaMemcpyHostToDevice));
+  }
+  return static_cast<llama_status>(s.code);
+}
+
+llama_status llama_layer_prefill(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                 int32_t batch, int32_t seq_len, const float* x_in, float* x_out, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  TRY(check_layer_call(dims, w, cache, batch, seq_len, x_in, x_out, workspace, ws_bytes, 0));
+  const WsLayout lay = plan_ws(*dims, batch, seq_len, 0);
+  return run_layer(*dims, *w, cache, batch, seq_len, x_in, x_out, static_cast<uint8_t*>(workspace), lay,
+                   static_cast<cudaStream_t>(stream));
+}
+
+llama_status llama_layer_decode(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  TRY(check_layer_call(dims, w, cache, batch, 1, x_in, x_out, workspace, ws_bytes, 0));
+  const WsLayout lay = plan_ws(*dims, batch, 1, 0);
+  return run_layer(*dims, *w, cache, batch, 1, x_in, x_out, static_cast<uint8_t*>(workspace), lay,
+                   static_cast<cudaStream_t>(stream));
+}
+
+size_t llama_model_workspace_size(const llama_model* m, int32_t batch, int32_t seq_len) {
+  if (m == nullptr || check_dims(&m->dims) != LLAMA_OK || batch <= 0 || seq_len <= 0 || m->vocab <= 0) return 0;
+  return plan_ws(m->dims, batch, seq_len, m->vocab).total;
+}
+
+llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* caches, const int32_t* tokens,
+                                 int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  if (m == nullptr || caches == nullptr || tokens == nullptr || next_ids == nullptr || workspace == nullptr)
+    return LLAMA_ERR_INVALID_ARG;
+  TRY(check_dims(&m->dims));
+  const llama_dims& d = m->dims;
+  if (m->n_layers <= 0 || m->vocab <= 0 || m->layers == nullptr || m->embed == nullptr ||
+      m->final_norm == nullptr || m->lm_head == nullptr)
+    return LLAMA_ERR_INVALID_ARG;
+  if (batch <= 0 || seq_len <= 0) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(m->embed) || !aligned16(m->final_norm) || !aligned16(m->lm_head) || !aligned16(tokens) ||
+      !aligned16(next_ids) || !aligned16(workspace) || (logits_or_null && !aligned16(logits_or_null)))
+    return LLAMA_ERR_ALIGNMENT;
+  const WsLayout lay = plan_ws(d, batch, seq_len, m->vocab);
+  if (ws_bytes < lay.total) return LLAMA_ERR_WORKSPACE_TOO_SMALL;
+  const int len0 = caches[0] ? caches[0]->length : -1;
+  for (int l = 0; l < m->n_layers; ++l) {
+    llama_kv_cache* c = caches[l];
+    if (c == nullptr || !same_dims(c->dims, d) || c->batch != batch || c->length != len0)
+      return LLAMA_ERR_INVALID_ARG;
+    if ((long long)c->length + seq_len > c->capacity) return LLAMA_ERR_CACHE_FULL;
+    TRY(check_weights(&m->layers[l]));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  const int M = batch * seq_len;
+  float* xa = reinterpret_cast<float*>(ws + lay.xa);
+  float* xb = reinterpret_cast<float*>(ws + lay.xb);
+  // a1: embedding
+  if (d.dtype == LLAMA_BF16)
+    embed_kernel<__nv_bfloat16><<<cdiv(M, 8), 256, 0, st>>>(
+        tokens, static_cast<const __nv_bfloat16*>(m->embed), xa, M, d.dim, m->vocab, status);
+  else
+    embed_kernel<float><<<cdiv(M, 8), 256, 0, st>>>(tokens, static_cast<const float*>(m->embed), xa, M, d.dim,
+                                                    m->vocab, status);
+  LAUNCH_CHECK();
+  // blocks
+  for (int l = 0; l < m->n_layers; ++l) {
+    TRY(run_layer(d, m->layers[l], caches[l], batch, seq_len, xa, xb, ws, lay, st));
+    std::swap(xa, xb);
+  }
+  // a10: final norm + lm_head on the last row of each sequence + argmax
+  const float* xl = xa;
+  if (seq_len > 1) {
+    float* g = reinterpret_cast<float*>(ws + lay.xl);
+    gather_last_rows_kernel<<<dim3(cdiv(d.dim, 256), batch), 256, 0, st>>>(xa, g, seq_len, d.dim);
+    LAUNCH_CHECK();
+    xl = g;
+  }
+  float* logits = logits_or_null ? logits_or_null : reinterpret_cast<float*>(ws + lay.logits);
+  if (d.dtype == LLAMA_BF16) {
+    __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
+    rmsnorm_kernel<__nv_bfloat16><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
+                                                                   d.eps);
+    LAUNCH_CHECK();
+    WSeg s{m->lm_head, m->vocab, 0};
+    TRY(gemm_bf16(st, true, hl, batch, d.dim, &s, 1, EPI_F32, logits, m->vocab, nullptr, 0,
+                  reinterpret_cast<float*>(ws + lay.partial), status));
+  } else {
+    float* hl = reinterpret_cast<float*>(ws + lay.hl);
+    rmsnorm_kernel<float><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
+    gemm_f32_kernel<F32_STORE><<<dim3(cdiv(m->vocab, 64), cdiv(batch, 64)), 256, 0, st>>>(
+        hl, d.dim, static_cast<const float*>(m->lm_head), nullptr, d.dim, batch, m->vocab, d.dim, logits, m->vocab,
+        nullptr, 0);
+    LAUNCH_CHECK();
+  }
+  argmax_kernel<<<batch, 1024, 0, st>>>(logits, m->vocab, next_ids);
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+llama_status llama_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
+  if (workspace == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return LLAMA_ERR_ALIGNMENT;
+  if (limit_ns > 5000000000ull) return LLAMA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<DevStatus*>(workspace),
+                                                                      limit_ns);
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+}  // extern "C"

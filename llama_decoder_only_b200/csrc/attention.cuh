@@ -1,0 +1,523 @@
+// Causal grouped-query attention over the KV cache, bf16 operands.
+//
+//  * attn_prefill_kernel: flash attention on tcgen05 ([HandsOn] "Transformer
+//    块的内部结构" names FlashAttention: tile Q/K/V through on-chip memory
+//    instead of materialising the score matrix in HBM).  One CTA per
+//    (128-query tile, head, sequence); K/V tiles of 128 keys arrive by TMA
+//    into a 2-stage ring; S = Q K^T lands in TMEM (double-buffered), the
+//    softmax warps read it with tcgen05.ld, keep the running max / sum in
+//    fp32 (online softmax), write P as bf16 into shared memory and the MMA
+//    warp accumulates O += P V in TMEM.  The running max is only moved (and
+//    O rescaled) when it grows by more than 2^8, which is exact because the
+//    final division uses the same stale maximum for numerator and sum.
+//  * attn_decode_kernel + attn_decode_combine_kernel: one new query per
+//    sequence; the cache of each (sequence, KV head) is split along the key
+//    axis over several CTAs; the query heads of a GQA group share every K/V
+//    load; partial (max, sum, output) are merged with the usual log-sum-exp
+//    rule.  CUDA-core FMAs, 16-byte loads; bound by HBM bandwidth.
+//
+// Definition followed: softmax(q k^T / sqrt(hd)) v over keys j <= p
+// ([MLX-13B] 2. 注意力机制 and 5. 因果掩码; [DeepDive] LLaMAAttention),
+// query head h reads KV head h / (nh / nkv).
+#pragma once
+
+#include "common.cuh"
+
+namespace llama {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ====================================================================== prefill
+
+struct AttnPrefillParams {
+  int L;         // new tokens per sequence
+  int p0;        // position of token 0 (cache length before the call)
+  int nh, nkv, hd;
+  int n_qtiles;
+  float scale_log2;   // log2(e) / sqrt(hd)
+  __nv_bfloat16* out; // [B*L, nh*hd]
+  DevStatus* status;
+  unsigned long long limit_ns;
+};
+
+constexpr int ATT_NS = 2;                       // K/V ring stages
+constexpr int ATT_REGION = 128 * 128;           // bytes of a [128 rows x 64 bf16] region
+constexpr int ATT_SMEM = 1024 + 2 * ATT_REGION        // Q
+                         + ATT_NS * 4 * ATT_REGION    // K, V (2 regions each)
+                         + 2 * ATT_REGION             // P
+                         + 256;
+
+__global__ void __launch_bounds__(192, 1)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const AttnPrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + 2 * ATT_REGION;          // stage s: K at s*4R, V at s*4R + 2R
+  uint8_t* sP = sKV + ATT_NS * 4 * ATT_REGION;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * ATT_REGION);
+  // bars: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full, pv_done, drain
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.n_qtiles - 1 - blockIdx.x;   // heavy (late) tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (p.nh / p.nkv);
+  const int hd = p.hd;
+  const int nreg = hd > 64 ? 2 : 1;             // 64-column regions per head row
+  const int hd_pad = nreg * 64;
+  const int q_row0 = qt * 128;                  // first token of the tile
+  const int last_q = min(p.L, q_row0 + 128) - 1;
+  const int n_kv = (p.p0 + last_q) / 128 + 1;   // kv tiles with any visible key
+  const int pos_min = p.p0 + q_row0;
+
+  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t q_full = bar0;
+  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (1 + ATT_NS + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * ATT_NS + s); };
+  auto s_full = [&](int i) { return bar0 + 8u * (1 + 3 * ATT_NS + i); };
+  auto s_free = [&](int i) { return bar0 + 8u * (3 + 3 * ATT_NS + i); };
+  const uint32_t p_full = bar0 + 8u * (5 + 3 * ATT_NS);
+  const uint32_t pv_done = bar0 + 8u * (6 + 3 * ATT_NS);
+  const uint32_t drain = bar0 + 8u * (7 + 3 * ATT_NS);
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ATT_NS; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(s_free(i), 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;   // S0 at col 0, S1 at col 128, O at col 256
+  WaitCtx wc{&abort_sh, p.status, p.limit_ns, 3};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int filled[ATT_NS] = {};
+      mbar_arrive_expect_tx(q_full, nreg * ATT_REGION);
+      for (int r = 0; r < nreg; ++r)
+        tma_load_3d(smem_u32(sQ + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64, q_row0, b);
+      const int zkv = b * p.nkv + g;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % ATT_NS;
+        if (!mbar_wait(kv_empty(s), ((j / ATT_NS) & 1) ^ 1u, wc, 1)) break;
+        uint8_t* st = sKV + s * 4 * ATT_REGION;
+        mbar_arrive_expect_tx(k_full(s), nreg * ATT_REGION);
+        for (int r = 0; r < nreg; ++r) tma_load_3d(smem_u32(st + r * ATT_REGION), &tmK, k_full(s), r * 64, j * 128, zkv);
+        mbar_arrive_expect_tx(v_full(s), nreg * ATT_REGION);
+        for (int r = 0; r < nreg; ++r)
+          tma_load_3d(smem_u32(st + (2 + r) * ATT_REGION), &tmV, v_full(s), r * 64, j * 128, zkv);
+        filled[s] = j + 1;
+      }
+      // drain own copies before exit
+      mbar_wait(q_full, 0, wc, 9, false);
+      for (int s = 0; s < ATT_NS; ++s)
+        if (filled[s] > 0) {
+          const uint32_t par = ((filled[s] - 1) / ATT_NS) & 1;
+          mbar_wait(k_full(s), par, wc, 9, false);
+          mbar_wait(v_full(s), par, wc, 9, false);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(128, hd_pad, 0, 1);   // V is MN-major
+      const int ksteps = hd / 16;
+      bool ok = mbar_wait(q_full, 0, wc, 2);
+      bool issued = false;
+      const uint32_t aQ = smem_u32(sQ);
+      const uint32_t aP = smem_u32(sP);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % ATT_NS, sb = j & 1;
+        if (!mbar_wait(k_full(s), (j / ATT_NS) & 1, wc, 3)) return false;
+        if (!mbar_wait(s_free(sb), ((j >> 1) & 1) ^ 1u, wc, 4)) return false;
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sKV + s * 4 * ATT_REGION);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t off = (ks >> 2) * ATT_REGION + (ks & 3) * 32;
+          umma_bf16(tmem + sb * 128, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(aK + off, 16, 1024),
+                    idesc_s, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full(sb));
+        issued = true;
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % ATT_NS;
+        if (!mbar_wait(p_full, j & 1, wc, 5)) return false;
+        if (!mbar_wait(v_full(s), (j / ATT_NS) & 1, wc, 6)) return false;
+        tc_fence_after();
+        const uint32_t aV = smem_u32(sKV + s * 4 * ATT_REGION + 2 * ATT_REGION);
+        for (int ks = 0; ks < 8; ++ks) {   // 128 keys, 16 per MMA
+          const uint32_t pa = aP + (ks >> 2) * ATT_REGION + (ks & 3) * 32;
+          const uint32_t va = aV + ks * 16 * 128;
+          umma_bf16(tmem + 256, smem_desc_sw128(pa, 16, 1024), smem_desc_sw128(va, ATT_REGION, 1024), idesc_o,
+                    (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done);
+        umma_commit(kv_empty(s));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 1; ok && j < n_kv; ++j) {
+        ok = issue_s(j);
+        if (ok) ok = issue_pv(j - 1);
+      }
+      if (ok) issue_pv(n_kv - 1);
+      if (issued) {
+        umma_commit(drain);
+        mbar_wait(drain, 0, wc, 8, false);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / correction / epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int t = q_row0 + row;                // token within the sequence
+    const int pos = p.p0 + t;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint8_t* prow0 = sP + row * 128;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int sb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(sb), (j >> 1) & 1, wc, 10))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + sb * 128 + c * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
+      }
+      tc_fence_before();
+      mbar_arrive(s_free(sb));
+      const bool need_mask = j * 128 + 127 > pos_min;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float x = s[i] * p.scale_log2;
+        if (need_mask && (j * 128 + i > pos)) x = -INFINITY;
+        s[i] = x;
+        mx = fmaxf(mx, x);
+      }
+      bool rescale = false;
+      float alpha = 1.f;
+      if (mx > m_used + 8.0f) {
+        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - mx);
+        m_used = mx;
+        rescale = j > 0;
+      }
+      // wait until the previous P·V has finished (O stable, P buffer free)
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, wc, 11))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (rescale) {
+        l *= alpha;
+        for (int c = 0; c < hd_pad; c += 32) {
+          float v[32];
+          tmem_ld32(tmem + lane_off + 256 + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st32(tmem + lane_off + 256 + c, v);
+        }
+        tmem_st_wait();
+      }
+      // P = exp2(s - m_used) as bf16 into the swizzled K-major A tile
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {   // 16-byte chunk c holds keys 8c .. 8c+7
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = (m_used == -INFINITY) ? 0.f : exp2f(s[8 * c + 2 * e] - m_used);
+          const float bb = (m_used == -INFINITY) ? 0.f : exp2f(s[8 * c + 2 * e + 1] - m_used);
+          __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
+          const float2 back = __bfloat1622float2(hv);
+          psum += back.x + back.y;
+          w[e] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        const int region = c >> 3, cc = c & 7;
+        uint8_t* dst = prow0 + region * ATT_REGION + ((cc ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += psum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, wc, 12))) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((size_t)b * p.L + t) * (size_t)(p.nh * hd) + (size_t)h * hd;
+      for (int c = 0; c < hd_pad; c += 32) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + 256 + c, v);
+        tmem_ld_wait();
+        if (t < p.L) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (c + 8 * q < hd) {
+              uint4 w;
+              w.x = pack_bf16x2(v[8 * q + 0] * inv, v[8 * q + 1] * inv);
+              w.y = pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv);
+              w.z = pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv);
+              w.w = pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c + 8 * q) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ====================================================================== decode
+
+struct AttnDecodeParams {
+  const __nv_bfloat16* qkv;   // [B, ld_qkv], q heads at columns h*hd (already rotated)
+  int ld_qkv;
+  const __nv_bfloat16* kc;    // [B][nkv][cap][hd]
+  const __nv_bfloat16* vc;
+  int cap, T;                 // capacity, visible keys (cache length after the append)
+  int nh, nkv;
+  int splits, keys_per_split;
+  float scale_log2;
+  float* part_ml;             // [B*nh][splits][2]   (splits > 1)
+  float* part_o;              // [B*nh][splits][hd]
+  __nv_bfloat16* out;         // [B, nh*hd]
+};
+
+template <int HD, int G>
+__global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams p) {
+  constexpr int LPK = HD == 96 ? 4 : HD / 8;    // lanes per key (power of two)
+  constexpr int VEC = HD / LPK;                 // elements per lane
+  constexpr int NV = VEC / 8;                   // 16-byte loads per lane per row
+  constexpr int KPW = 32 / LPK;                 // keys per warp step
+  constexpr int NK = 4;                         // keys per lane group per step
+  constexpr int NW = 4;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane / LPK, sub = lane % LPK;
+  const int j0 = split * p.keys_per_split;
+  const int j1 = min(p.T, j0 + p.keys_per_split);
+
+  float q[G][VEC];
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi) {
+    const __nv_bfloat16* qr = p.qkv + (size_t)b * p.ld_qkv + (size_t)(g * G + gi) * HD + sub * VEC;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      uint4 u = *reinterpret_cast<const uint4*>(qr + 8 * v);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        q[gi][8 * v + 2 * e] = f.x * p.scale_log2;
+        q[gi][8 * v + 2 * e + 1] = f.y * p.scale_log2;
+      }
+    }
+  }
+  float m[G], l[G], o[G][VEC];
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi) {
+    m[gi] = -INFINITY;
+    l[gi] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) o[gi][e] = 0.f;
+  }
+  const size_t head_off = ((size_t)b * p.nkv + g) * (size_t)p.cap * HD + sub * VEC;
+  const __nv_bfloat16* K = p.kc + head_off;
+  const __nv_bfloat16* V = p.vc + head_off;
+  constexpr int STEP = NW * KPW * NK;
+  for (int wb = j0 + warp * KPW * NK; wb < j1; wb += STEP) {
+    uint4 kr[NK][NV], vr[NK][NV];
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+      const int j = wb + grp * NK + kk;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        if (j < j1) {
+          kr[kk][v] = __ldg(reinterpret_cast<const uint4*>(K + (size_t)j * HD) + v);
+          vr[kk][v] = __ldg(reinterpret_cast<const uint4*>(V + (size_t)j * HD) + v);
+        } else {
+          kr[kk][v] = make_uint4(0, 0, 0, 0);
+          vr[kk][v] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    float s[NK][G];
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+      float kf[VEC];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[kk][v]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          kf[8 * v + 2 * e] = f.x;
+          kf[8 * v + 2 * e + 1] = f.y;
+        }
+      }
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) {
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) d = fmaf(q[gi][e], kf[e], d);
+#pragma unroll
+        for (int off = LPK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        s[kk][gi] = (wb + grp * NK + kk < j1) ? d : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      float mx = s[0][gi];
+#pragma unroll
+      for (int kk = 1; kk < NK; ++kk) mx = fmaxf(mx, s[kk][gi]);
+      const float mn = fmaxf(m[gi], mx);
+      if (mn == -INFINITY) continue;
+      const float alpha = exp2f(m[gi] - mn);
+      m[gi] = mn;
+      l[gi] *= alpha;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[gi][e] *= alpha;
+#pragma unroll
+      for (int kk = 0; kk < NK; ++kk) {
+        const float pk = exp2f(s[kk][gi] - mn);
+        l[gi] += pk;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&vr[kk][v]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            o[gi][8 * v + 2 * e] = fmaf(pk, f.x, o[gi][8 * v + 2 * e]);
+            o[gi][8 * v + 2 * e + 1] = fmaf(pk, f.y, o[gi][8 * v + 2 * e + 1]);
+          }
+        }
+      }
+    }
+  }
+  // merge the lane groups of the warp (same `sub`, different keys)
+#pragma unroll
+  for (int off = LPK; off < 32; off <<= 1) {
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[gi], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[gi], off);
+      const float mn = fmaxf(m[gi], mo);
+      const float a = mn == -INFINITY ? 0.f : exp2f(m[gi] - mn);
+      const float c = mn == -INFINITY ? 0.f : exp2f(mo - mn);
+      l[gi] = l[gi] * a + lo * c;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float oo = __shfl_xor_sync(0xffffffffu, o[gi][e], off);
+        o[gi][e] = o[gi][e] * a + oo * c;
+      }
+      m[gi] = mn;
+    }
+  }
+  // merge the warps through shared memory
+  __shared__ float sm_m[NW][G], sm_l[NW][G];
+  __shared__ float sm_o[NW][G][HD];
+  if (grp == 0) {
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      if (sub == 0) {
+        sm_m[warp][gi] = m[gi];
+        sm_l[warp][gi] = l[gi];
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) sm_o[warp][gi][sub * VEC + e] = o[gi][e];
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
+    const int gi = idx / HD, d = idx % HD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][gi]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float c = exp2f(sm_m[w][gi] - M);
+        Lsum += sm_l[w][gi] * c;
+        O += sm_o[w][gi][d] * c;
+      }
+    }
+    const int hq = g * G + gi;
+    if (p.splits == 1) {
+      p.out[(size_t)b * p.nh * HD + (size_t)hq * HD + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+    } else {
+      const size_t r = ((size_t)b * p.nh + hq) * p.splits + split;
+      p.part_o[r * HD + d] = O;
+      if (d == 0) {
+        p.part_ml[2 * r] = M;
+        p.part_ml[2 * r + 1] = Lsum;
+      }
+    }
+  }
+}
+
+// out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
+__global__ void attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
+                                           __nv_bfloat16* __restrict__ out, int nh, int hd, int splits) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const size_t r0 = ((size_t)b * nh + h) * splits;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[2 * (r0 + s)]);
+  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < splits; ++s) {
+        const float c = exp2f(part_ml[2 * (r0 + s)] - M);
+        Lsum += part_ml[2 * (r0 + s) + 1] * c;
+        O += part_o[(r0 + s) * hd + d] * c;
+      }
+    }
+    out[(size_t)b * nh * hd + (size_t)h * hd + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+  }
+}
+
+}  // namespace llama

@@ -1,0 +1,234 @@
+// Bandwidth-bound kernels of the block: RMSNorm, fused RoPE + KV-cache
+// append, embedding gather, last-row gather and greedy argmax.
+#pragma once
+
+#include "common.cuh"
+
+namespace llama {
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// ------------------------------------------------------------------ RMSNorm (K1)
+// h[m, :] = g * (x[m, :] * rsqrt(mean(x[m, :]^2) + eps)), one warp per row,
+// 16-byte loads, warp-shuffle reduction ([MLX-13B] 4. RMSNorm; [DeepDive]
+// LLaMARMSNorm).  `x_row_stride` lets the final norm read the last row of
+// each sequence only.  dim % 4 == 0.
+template <typename OutT>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, long long x_row_stride,
+                                                      const float* __restrict__ g, OutT* __restrict__ h, int rows,
+                                                      int dim, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)warp * x_row_stride);
+  const int n4 = dim >> 2;
+  float ss = 0.f;
+  for (int i = lane; i < n4; i += 32) {
+    float4 v = __ldg(xr + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float rstd = rsqrtf(ss / (float)dim + eps);
+  OutT* hr = h + (size_t)warp * dim;
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  for (int i = lane; i < n4; i += 32) {
+    float4 v = __ldg(xr + i);
+    float4 w = __ldg(g4 + i);
+    float a = w.x * (v.x * rstd), b = w.y * (v.y * rstd), c = w.z * (v.z * rstd), d = w.w * (v.w * rstd);
+    if constexpr (sizeof(OutT) == 2) {
+      uint2 o;
+      o.x = pack_bf16x2(a, b);
+      o.y = pack_bf16x2(c, d);
+      reinterpret_cast<uint2*>(hr)[i] = o;
+    } else {
+      reinterpret_cast<float4*>(hr)[i] = make_float4(a, b, c, d);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ RoPE + KV append (K3)
+// One CTA per token.  The token's cos/sin ladder is computed once in fp64
+// (angle p * theta^(-2i/hd), [DeepDive] LLaMARoPE) into shared memory, then
+// every (head, pair) of q and k is rotated; q is rotated in place in the
+// projection buffer, rotated k and plain v are written to the cache at
+// position p0 + t ([MLX-13B] KV 缓存实现片段: concatenate after the cached
+// entries, RoPE offset = cache length).
+//   qkv   [M, (nh + 2 nkv) hd] row-major (q | k | v), M = batch * L
+//   cache [batch][nkv][cap][hd]
+// style 0: rotate-half pairs (i, i + hd/2); style 1: adjacent pairs (2i, 2i+1).
+template <typename T>
+__global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T* __restrict__ kc,
+                                                          T* __restrict__ vc, int L, int p0, int nh, int nkv,
+                                                          int hd, int cap, float theta, int style) {
+  __shared__ float cs[64], sn[64];
+  const int m = blockIdx.x;
+  const int b = m / L;
+  const int t = m % L;
+  const int p = p0 + t;
+  const int half = hd >> 1;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double inv = pow((double)theta, -2.0 * (double)i / (double)hd);
+    double s, c;
+    sincos((double)p * inv, &s, &c);
+    cs[i] = (float)c;
+    sn[i] = (float)s;
+  }
+  __syncthreads();
+  const int qkvn = (nh + 2 * nkv) * hd;
+  T* row = qkv + (size_t)m * qkvn;
+  // rotate q (heads 0..nh-1) and k (heads nh..nh+nkv-1)
+  const int nrot = (nh + nkv) * half;
+  for (int e = threadIdx.x; e < nrot; e += blockDim.x) {
+    const int head = e / half;
+    const int i = e % half;
+    const int i0 = style == 0 ? i : 2 * i;
+    const int i1 = style == 0 ? i + half : 2 * i + 1;
+    T* hv = row + head * hd;
+    const float x0 = to_f32(hv[i0]), x1 = to_f32(hv[i1]);
+    const float c = cs[i], s = sn[i];
+    const float y0 = x0 * c - x1 * s;
+    const float y1 = x1 * c + x0 * s;
+    if (head < nh) {
+      hv[i0] = from_f32<T>(y0);
+      hv[i1] = from_f32<T>(y1);
+    } else {
+      const int g = head - nh;
+      T* dst = kc + (((size_t)b * nkv + g) * cap + p) * hd;
+      dst[i0] = from_f32<T>(y0);
+      dst[i1] = from_f32<T>(y1);
+    }
+  }
+  // copy v
+  const int nv = nkv * hd;
+  const T* vsrc = row + (nh + nkv) * hd;
+  for (int e = threadIdx.x; e < nv; e += blockDim.x) {
+    const int g = e / hd, d = e % hd;
+    vc[(((size_t)b * nkv + g) * cap + p) * hd + d] = vsrc[e];
+  }
+}
+
+// ------------------------------------------------------------------ embedding gather (K6)
+// x[m, :] = float(E[tok[m], :]) ([DeepDive] class LLaMA: nn.Embedding).
+// One warp per token, 16-byte loads.  Out-of-range ids record INVALID_ARG
+// in the status word and produce a zero row.
+template <typename T>
+__global__ void __launch_bounds__(256) embed_kernel(const int32_t* __restrict__ tok, const T* __restrict__ E,
+                                                    float* __restrict__ x, int M, int dim, int vocab,
+                                                    DevStatus* st) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= M) return;
+  const int id = tok[warp];
+  float* xr = x + (size_t)warp * dim;
+  if (id < 0 || id >= vocab) {
+    if (lane == 0) record_error(st, LLAMA_ERR_INVALID_ARG, 20, warp);
+    for (int i = lane; i < dim; i += 32) xr[i] = 0.f;
+    return;
+  }
+  const T* er = E + (size_t)id * dim;
+  if constexpr (sizeof(T) == 2) {
+    for (int i = lane; i < dim / 8; i += 32) {
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(er) + i);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      float4 a, b;
+      float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+      float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
+      a = make_float4(f0.x, f0.y, f1.x, f1.y);
+      b = make_float4(f2.x, f2.y, f3.x, f3.y);
+      reinterpret_cast<float4*>(xr)[2 * i] = a;
+      reinterpret_cast<float4*>(xr)[2 * i + 1] = b;
+    }
+  } else {
+    for (int i = lane; i < dim / 4; i += 32)
+      reinterpret_cast<float4*>(xr)[i] = __ldg(reinterpret_cast<const float4*>(er) + i);
+  }
+}
+
+// ------------------------------------------------------------------ greedy argmax (K7)
+// ids[b] = argmax_v logits[b, v]; ties resolve to the lowest index
+// ([HandsOn] 第三章: argmax of the last position; numpy/torch convention).
+// One CTA per row; NaN never wins.
+__global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ logits, int vocab,
+                                                      int32_t* __restrict__ ids) {
+  const int b = blockIdx.x;
+  const float* r = logits + (size_t)b * vocab;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int v = threadIdx.x; v < vocab; v += blockDim.x) {
+    const float x = r[v];
+    if (x > best || (x == best && v < bi)) {
+      best = x;
+      bi = v;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob > best || (ob == best && oi < bi)) {
+      best = ob;
+      bi = oi;
+    }
+  }
+  __shared__ float sb[32];
+  __shared__ int si[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sb[warp] = best;
+    si[warp] = bi;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    best = lane < nw ? sb[lane] : -INFINITY;
+    bi = lane < nw ? si[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    if (lane == 0) ids[b] = bi == 0x7fffffff ? 0 : bi;
+  }
+}
+
+// Gather the last row of each of `batch` sequences of length L: dst[b] = src[b*L + L-1].
+__global__ void gather_last_rows_kernel(const float* __restrict__ src, float* __restrict__ dst, int L, int dim) {
+  const int b = blockIdx.y;
+  const float* s = src + ((size_t)b * L + (L - 1)) * dim;
+  float* d = dst + (size_t)b * dim;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < dim; i += gridDim.x * blockDim.x) d[i] = s[i];
+}
+
+// Device-side failure self-test: wait on an mbarrier that nothing arrives on;
+// the bounded wait runs out, records LLAMA_ERR_DEVICE_TIMEOUT and returns.
+__global__ void selftest_wait_kernel(DevStatus* st, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_sh;
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx wc{&abort_sh, st, limit_ns, 99};
+    mbar_wait(smem_u32(&bar), 0, wc, 0);
+  }
+}
+
+}  // namespace llama

@@ -237,8 +237,11 @@ def layer_forward(d: Dims, W, x, cache: KVCache, rounding=None, rows=None):
     rows are pushed through attention, o_proj and the FFN (all rows still
     feed the cache), and the returned arrays hold just those rows.
 
-    Returns ``(x_out, parts)`` with ``parts["x_mid"]`` the residual stream
-    after the attention branch.
+    Returns ``(x_out, parts)``: ``parts`` holds the intermediates ``h``
+    (norm-1 output), ``q`` (after RoPE, selected rows), ``k`` (after RoPE),
+    ``v``, ``attn`` (attention output, heads concatenated), ``x_mid`` (residual
+    stream after the attention branch), ``h2`` (norm-2 output) and ``m``
+    (SwiGLU product).
     """
     rnd = to_bf16 if rounding == "bf16" else _identity
     x = np.asarray(x, dtype=np.float64)
@@ -248,9 +251,9 @@ def layer_forward(d: Dims, W, x, cache: KVCache, rounding=None, rows=None):
     pos = p0 + np.arange(L)
 
     h = rnd(rms_norm(x, W["attn_norm"], d.eps))
-    k = rnd(h @ np.asarray(W["wk"], np.float64).T).reshape(B, L, nkv, hd)
+    k_raw = rnd(h @ np.asarray(W["wk"], np.float64).T).reshape(B, L, nkv, hd)
     v = rnd(h @ np.asarray(W["wv"], np.float64).T).reshape(B, L, nkv, hd)
-    k = rnd(apply_rope(k, pos, d.rope_theta, d.rope_style))
+    k = rnd(apply_rope(k_raw, pos, d.rope_theta, d.rope_style))
     cache.append(k, v)
 
     sel = np.arange(L) if rows is None else np.asarray(rows)
@@ -271,7 +274,8 @@ def layer_forward(d: Dims, W, x, cache: KVCache, rounding=None, rows=None):
     up = h2 @ np.asarray(W["w3"], np.float64).T
     m = rnd(silu(gate) * up)
     x_out = x_mid + m @ np.asarray(W["w2"], np.float64).T
-    return x_out, {"x_mid": x_mid, "attn": o, "m": m}
+    return x_out, {"h": h, "q": q, "k_raw": k_raw, "k": k, "v": v, "attn": o, "x_mid": x_mid,
+                   "h2": h2, "m": m}
 
 
 def embed(E, tokens):

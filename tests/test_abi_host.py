@@ -1,0 +1,196 @@
+"""Host-side checks of the C ABI (CPU only: nothing here launches a kernel).
+
+* the library loads and exports every function ``include/llama_b200.h`` declares;
+* argument validation rejects bad input before anything is enqueued
+  (null pointers, unsupported shapes, misalignment, aliasing, cache overflow,
+  a too-small workspace) and leaves the cache length unchanged;
+* workspace sizing is monotone in the token count.
+
+Fake device addresses are fine here: every rejected call returns before its
+first CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import llama_decoder_only_b200 as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "llama_b200.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(llama_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    lib = L.lib()
+    declared = header_functions()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(L.EXPORTS)
+
+
+def test_abi_version_and_status_strings():
+    lib = L.lib()
+    assert lib.llama_abi_version() == 1
+    for s in range(8):
+        assert lib.llama_status_string(s)
+    assert lib.llama_status_string(99) == b"unknown status"
+
+
+BF = dict(dim=512, n_heads=8, n_kv_heads=2, head_dim=64, ffn_dim=1376, eps=1e-5)
+FAKE = 0x10000000  # aligned fake device address, never dereferenced
+
+
+def dims(**kw):
+    a = dict(BF, rope_theta=1e4, rope_style=L.ROPE_HALF, dtype=L.BF16)
+    a.update(kw)
+    return L.make_dims(**a)
+
+
+def fake_weights(base=FAKE):
+    return L.LayerWeights(*[base + i * 0x100000 for i in range(9)])
+
+
+def cache(d, batch=2, cap=64):
+    h = ctypes.c_void_p()
+    st = L.lib().llama_kv_cache_create(ctypes.byref(d), batch, cap, FAKE, FAKE + 0x1000000, ctypes.byref(h))
+    assert st == 0
+    return h
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(n_heads=6, n_kv_heads=4), 1),       # not a multiple
+    (dict(head_dim=48), 2),                   # unsupported head dim
+    (dict(head_dim=32), 2),                   # 32 only on the fp32 path
+    (dict(dim=100), 2),                       # dim % 8
+    (dict(eps=0.0), 1),
+    (dict(rope_theta=1.0), 1),
+    (dict(rope_style=3), 1),
+    (dict(dtype=7), 1),
+    (dict(n_heads=24, n_kv_heads=2), 2),      # GQA group 12 not instantiated
+])
+def test_bad_dims_rejected(kw, expect):
+    d = dims(**kw)
+    assert L.lib().llama_workspace_size(ctypes.byref(d), 1, 16) == 0
+    h = ctypes.c_void_p()
+    assert L.lib().llama_kv_cache_create(ctypes.byref(d), 1, 16, FAKE, FAKE, ctypes.byref(h)) == expect
+
+
+def test_fp32_head_dim_32_supported():
+    d = dims(dtype=L.F32, head_dim=32)
+    assert L.lib().llama_workspace_size(ctypes.byref(d), 1, 64) > 0
+
+
+def test_cache_handle_lifecycle():
+    d = dims()
+    h = cache(d)
+    lib = L.lib()
+    assert lib.llama_kv_cache_length(h) == 0
+    assert lib.llama_kv_cache_capacity(h) == 64
+    assert lib.llama_kv_cache_set_length(h, 64) == 0
+    assert lib.llama_kv_cache_set_length(h, 65) == 3        # LLAMA_ERR_CACHE_FULL
+    assert lib.llama_kv_cache_set_length(h, -1) == 1
+    assert lib.llama_kv_cache_length(None) == -1
+    lib.llama_kv_cache_destroy(h)
+
+
+def test_cache_create_rejects_null_and_misaligned():
+    d = dims()
+    h = ctypes.c_void_p()
+    lib = L.lib()
+    assert lib.llama_kv_cache_create(ctypes.byref(d), 1, 16, None, FAKE, ctypes.byref(h)) == 1
+    assert lib.llama_kv_cache_create(ctypes.byref(d), 1, 16, FAKE + 8, FAKE, ctypes.byref(h)) == 4
+    assert lib.llama_kv_cache_create(ctypes.byref(d), 0, 16, FAKE, FAKE, ctypes.byref(h)) == 1
+    assert lib.llama_kv_cache_create(ctypes.byref(d), 1, 16, FAKE, FAKE, None) == 1
+
+
+def _prefill(d, w, h, B, Lq, x_in, x_out, ws, ws_bytes):
+    return L.lib().llama_layer_prefill(ctypes.byref(d), ctypes.byref(w), h, B, Lq, x_in, x_out, ws, ws_bytes, None)
+
+
+def test_layer_call_validation_before_launch():
+    d = dims()
+    h = cache(d, batch=2, cap=64)
+    w = fake_weights()
+    lib = L.lib()
+    need = lib.llama_workspace_size(ctypes.byref(d), 2, 16)
+    X, Y, WS = 0x20000000, 0x30000000, 0x40000000
+    assert _prefill(d, w, h, 2, 16, X, Y, WS, need - 1) == 5            # workspace too small
+    assert _prefill(d, w, h, 2, 16, X, X + 256, WS, need) == 1          # x_out overlaps x_in
+    assert _prefill(d, w, h, 2, 16, X + 4, Y, WS, need) == 4            # misaligned input
+    assert _prefill(d, w, h, 3, 16, X, Y, WS, need) == 1                # batch != cache batch
+    assert _prefill(d, w, h, 2, 0, X, Y, WS, need) == 1                 # empty call
+    assert _prefill(d, w, h, 2, 65, X, Y, WS, 1 << 40) == 3             # exceeds capacity
+    bad = fake_weights()
+    bad.wk = None
+    assert _prefill(d, bad, h, 2, 16, X, Y, WS, need) == 1              # null weight
+    bad = fake_weights()
+    bad.w2 = FAKE + 2
+    assert _prefill(d, bad, h, 2, 16, X, Y, WS, need) == 4              # misaligned weight
+    d2 = dims(ffn_dim=1408)
+    assert _prefill(d2, w, h, 2, 16, X, Y, WS, need) == 1               # dims differ from the cache's
+    assert lib.llama_kv_cache_length(h) == 0                            # nothing advanced
+    lib.llama_kv_cache_destroy(h)
+
+
+def test_decode_rejects_full_cache():
+    d = dims()
+    h = cache(d, batch=1, cap=8)
+    lib = L.lib()
+    lib.llama_kv_cache_set_length(h, 8)
+    w = fake_weights()
+    st = lib.llama_layer_decode(ctypes.byref(d), ctypes.byref(w), h, 1, 0x20000000, 0x30000000, 0x40000000,
+                                1 << 40, None)
+    assert st == 3
+    assert lib.llama_kv_cache_length(h) == 8
+    lib.llama_kv_cache_destroy(h)
+
+
+def test_workspace_grows_with_tokens():
+    d = dims()
+    lib = L.lib()
+    sizes = [lib.llama_workspace_size(ctypes.byref(d), 1, n) for n in (1, 64, 512, 4096)]
+    assert all(a < b for a, b in zip(sizes, sizes[1:]))
+
+
+def test_model_call_validation():
+    d = dims()
+    lib = L.lib()
+    layers = (L.LayerWeights * 2)(fake_weights(), fake_weights())
+    m = L.Model(d, 2, 1000, FAKE, FAKE, FAKE, ctypes.cast(layers, ctypes.POINTER(L.LayerWeights)))
+    need = lib.llama_model_workspace_size(ctypes.byref(m), 2, 8)
+    assert need > lib.llama_workspace_size(ctypes.byref(d), 2, 8)
+    h0, h1 = cache(d, 2, 16), cache(d, 2, 16)
+    arr = (ctypes.c_void_p * 2)(h0.value, h1.value)
+    call = lambda ws_bytes, tok=0x50000000: lib.llama_model_forward(  # noqa: E731
+        ctypes.byref(m), arr, tok, 2, 8, None, 0x60000000, 0x40000000, ws_bytes, None)
+    assert call(need - 1) == 5
+    assert call(need, tok=0x50000004) == 4
+    lib.llama_kv_cache_set_length(h1, 3)                                # lengths disagree
+    assert call(need) == 1
+    lib.llama_kv_cache_destroy(h0)
+    lib.llama_kv_cache_destroy(h1)
+
+
+def test_selftest_rejects_bad_args():
+    lib = L.lib()
+    assert lib.llama_selftest_wait_timeout(None, 1000, None) == 1
+    assert lib.llama_selftest_wait_timeout(FAKE + 4, 1000, None) == 4
+    assert lib.llama_selftest_wait_timeout(FAKE, 10 ** 10, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "LIB", str(tmp_path / "missing.so"))
+    with pytest.raises(L.LlamaError):
+        L.lib()
+    importlib.reload(L)
