@@ -222,6 +222,27 @@ int32_t llama_abi_version(void);
  * (default 2e9).  A test may lower it.  Returns the previous value. */
 uint64_t llama_set_wait_limit_ns(uint64_t ns);
 
+/* ------------------------------------------------------------------ tracing */
+
+/* Number of kernels the library has enqueued since it was loaded. */
+uint64_t llama_launch_count(void);
+
+/* Turn per-launch tracing on or off.  While on, every kernel launch is
+ * bracketed by two CUDA events on its stream (a few microseconds of host
+ * work per launch).  No page counterpart: measurement only. */
+llama_status llama_profile_enable(int32_t on);
+
+/* Accumulated device time and launch count per kernel kind of the traced
+ * launches (synchronises on their events).  Fills up to n entries of each
+ * non-null array; names point to static strings.  Returns the number of
+ * kinds.  reset != 0 clears the accumulators afterwards. */
+int32_t llama_profile_read(const char** names, double* total_ms, long long* launches, int32_t n, int32_t reset);
+
+/* Traced launches that have not finished yet (non-blocking query of their end
+ * events), oldest first: writes up to n kind names and returns the count.
+ * Names a kernel that does not complete without waiting on it. */
+int32_t llama_profile_inflight(const char** names, int32_t n);
+
 /* Self-test of the failure path: launches one CTA that waits on an
  * mbarrier nothing will ever arrive on, with a limit of `limit_ns`; the wait
  * runs out, the kernel records LLAMA_ERR_DEVICE_TIMEOUT in the workspace

@@ -24,6 +24,7 @@ __all__ = [
     "make_dims", "layer_weights", "model_struct", "KVCache",
     "workspace_size", "model_workspace_size", "layer_prefill", "layer_decode",
     "model_forward", "device_status", "workspace_offsets", "set_wait_limit_ns", "selftest_wait_timeout",
+    "launch_count", "profile_enable", "profile_read", "profile_inflight",
 ]
 
 F32, BF16 = 0, 1
@@ -85,6 +86,11 @@ EXPORTS = {
     "llama_model_workspace_size": (_S, [_MP, _I, _I]),
     "llama_model_forward": (_I, [_MP, ctypes.POINTER(_P), _P, _I, _I, _P, _P, _P, _S, _P]),
     "llama_selftest_wait_timeout": (_I, [_P, _U64, _P]),
+    "llama_launch_count": (_U64, []),
+    "llama_profile_enable": (_I, [_I]),
+    "llama_profile_inflight": (_I, [ctypes.POINTER(ctypes.c_char_p), _I]),
+    "llama_profile_read": (_I, [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                ctypes.POINTER(ctypes.c_longlong), _I, _I]),
 }
 
 _lib = None
@@ -213,6 +219,31 @@ def workspace_offsets(dims, batch, seq_len):
 
 def device_status(ws, clear=False):
     return lib().llama_device_status(_ptr(ws), 1 if clear else 0)
+
+
+def launch_count():
+    return int(lib().llama_launch_count())
+
+
+def profile_enable(on=True):
+    _check(lib().llama_profile_enable(1 if on else 0), "llama_profile_enable")
+
+
+def profile_read(reset=True):
+    """{kernel kind: (total ms, launches)} of the traced launches."""
+    n = 32
+    names = (ctypes.c_char_p * n)()
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    k = lib().llama_profile_read(names, ms, cnt, n, 1 if reset else 0)
+    return {names[i].decode(): (ms[i], cnt[i]) for i in range(min(k, n)) if cnt[i] > 0}
+
+
+def profile_inflight(n=64):
+    """Kinds of traced launches still running (non-blocking), oldest first."""
+    names = (ctypes.c_char_p * n)()
+    k = lib().llama_profile_inflight(names, n)
+    return k, [names[i].decode() for i in range(min(k, n))]
 
 
 def set_wait_limit_ns(ns):

@@ -6,9 +6,12 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "attention.cuh"
 #include "common.cuh"
@@ -33,6 +36,78 @@ std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 constexpr int kMaxSkGrid = 192;     // upper bound on stream-K CTAs (workspace sizing)
 constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
 constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K form up to here
+
+// ------------------------------------------------------------------ tracing
+// Every kernel launch of the library is counted; when tracing is on it is
+// also bracketed by two CUDA events on its stream, and llama_profile_read
+// sums the elapsed times per kernel kind.
+
+enum KernelKind : int {
+  K_RMSNORM = 0, K_GEMM_QKV, K_ROPE_APPEND, K_ATTN_PREFILL, K_ATTN_DECODE, K_ATTN_COMBINE, K_GEMM_O,
+  K_GEMM_GATE_UP, K_GEMM_DOWN, K_SPLITK_REDUCE, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
+  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_COUNT
+};
+const char* const kKindNames[K_COUNT] = {
+  "rmsnorm", "gemm_qkv", "rope_kv_append", "attn_prefill", "attn_decode", "attn_decode_combine", "gemm_o_proj",
+  "gemm_gate_up_swiglu", "gemm_down", "splitk_reduce", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
+  "gemm_f32", "attn_f32", "selftest"};
+
+struct ProfRec {
+  cudaEvent_t a, b;
+  int kind;
+};
+
+struct Tracer {
+  std::mutex mu;
+  bool on = false;
+  std::vector<ProfRec> pending;
+  double total_ms[K_COUNT] = {};
+  long long launches[K_COUNT] = {};
+};
+Tracer& tracer() {
+  static Tracer t;
+  return t;
+}
+std::atomic<unsigned long long> g_launch_count{0};
+
+// LLAMA_SYNC_TRACE=1 (debugging aid): print every launch to stderr and wait
+// for it to finish before returning, so a failing kernel is named.
+bool sync_trace() {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_SYNC_TRACE");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+
+struct LaunchScope {
+  cudaStream_t st;
+  int kind;
+  cudaEvent_t a = nullptr, b = nullptr;
+  LaunchScope(cudaStream_t s, int k) : st(s), kind(k) {
+    g_launch_count.fetch_add(1, std::memory_order_relaxed);
+    if (sync_trace()) std::fprintf(stderr, "[llama] launch %s\n", kKindNames[kind]);
+    Tracer& t = tracer();
+    if (t.on && cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess) {
+      cudaEventRecord(a, st);
+    } else {
+      a = b = nullptr;
+    }
+  }
+  ~LaunchScope() {
+    if (sync_trace()) {
+      const cudaError_t e = cudaStreamSynchronize(st);
+      std::fprintf(stderr, "[llama] done %s: %s\n", kKindNames[kind], cudaGetErrorString(e));
+    }
+    if (a != nullptr) {
+      cudaEventRecord(b, st);
+      Tracer& t = tracer();
+      std::lock_guard<std::mutex> g(t.mu);
+      t.pending.push_back({a, b, kind});
+    }
+  }
+};
+#define TRACE(kind, stream) LaunchScope _trace_scope_(stream, kind)
 
 #define CUDA_TRY(x)                           \
   do {                                        \
@@ -212,7 +287,7 @@ struct WSeg {
 
 template <int BN, bool SWAP, int EPI>
 llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
-                            cudaStream_t st) {
+                            cudaStream_t st, int kind) {
   using C = GemmCfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -220,14 +295,17 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
                                   C::SMEM_BYTES));
     attr_set = true;
   }
-  gemm_tc_kernel<BN, SWAP, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(a, w[0], w[1], w[2], p);
+  {
+    TRACE(kind, st);
+    gemm_tc_kernel<BN, SWAP, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(a, w[0], w[1], w[2], p);
+  }
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
 
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
 llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
-                          void* out, int ldo, const float* resid, int ldr, DevStatus* status) {
+                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind) {
   constexpr int BN = 256;
   GemmParams p{};
   p.K = K;
@@ -273,13 +351,13 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
   const int grid = std::min(tiles, num_sms());
   switch (epi) {
     case EPI_BF16:
-      return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st);
+      return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st, kind);
     case EPI_RESID_F32:
-      return launch_gemm_tc<BN, false, EPI_RESID_F32>(ta, tw, p, grid, st);
+      return launch_gemm_tc<BN, false, EPI_RESID_F32>(ta, tw, p, grid, st, kind);
     case EPI_SWIGLU_BF16:
-      return launch_gemm_tc<BN, false, EPI_SWIGLU_BF16>(ta, tw, p, grid, st);
+      return launch_gemm_tc<BN, false, EPI_SWIGLU_BF16>(ta, tw, p, grid, st, kind);
     case EPI_F32:
-      return launch_gemm_tc<BN, false, EPI_F32>(ta, tw, p, grid, st);
+      return launch_gemm_tc<BN, false, EPI_F32>(ta, tw, p, grid, st, kind);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -287,7 +365,8 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
 // Stream-K (decode) GEMM: partials = act[M, K] · W^T with W as the MMA's A
 // operand, then the reduce kernel applies `dec_epi`.
 llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int dec_epi,
-                         void* out, int ldo, const float* resid, int ldr, float* partial, DevStatus* status) {
+                         void* out, int ldo, const float* resid, int ldr, float* partial, DevStatus* status,
+                         int kind) {
   const int BN = swap_bn(M);
   GemmParams p{};
   p.K = K;
@@ -320,10 +399,10 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.max_pieces = (int)((per + p.num_kb - 1) / p.num_kb) + 1;
   llama_status s = LLAMA_OK;
   switch (BN) {
-    case 16: s = launch_gemm_tc<16, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
-    case 32: s = launch_gemm_tc<32, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
-    case 64: s = launch_gemm_tc<64, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
-    default: s = launch_gemm_tc<128, true, EPI_PARTIAL>(ta, tw, p, grid, st); break;
+    case 16: s = launch_gemm_tc<16, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
+    case 32: s = launch_gemm_tc<32, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
+    case 64: s = launch_gemm_tc<64, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
+    default: s = launch_gemm_tc<128, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
   }
   if (s != LLAMA_OK) return s;
   ReduceParams r{};
@@ -350,6 +429,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   }
   r.n_out = n_out;
   dim3 grid_r(cdiv(n_out, 256), M);
+  TRACE(K_SPLITK_REDUCE, st);
   switch (dec_epi) {
     case DEC_BF16: splitk_reduce_kernel<DEC_BF16><<<grid_r, 256, 0, st>>>(r); break;
     case DEC_RESID_F32: splitk_reduce_kernel<DEC_RESID_F32><<<grid_r, 256, 0, st>>>(r); break;
@@ -363,16 +443,16 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
                        int epi, void* out, int ldo, const float* resid, int ldr, float* partial,
-                       DevStatus* status) {
+                       DevStatus* status, int kind) {
   if (decode && M <= kSwapMaxTokens) {
     const int dec = epi == EPI_BF16 ? DEC_BF16 : epi == EPI_RESID_F32 ? DEC_RESID_F32
                   : epi == EPI_SWIGLU_BF16 ? DEC_SWIGLU_BF16 : DEC_F32;
     WSeg s2[3];
     for (int i = 0; i < nseg; ++i) s2[i] = segs[i];
     if (epi == EPI_SWIGLU_BF16) s2[1].col0 = segs[0].rows;  // up rows follow the gate rows
-    return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status);
+    return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status, kind);
   }
-  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status);
+  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
 }
 
 // ------------------------------------------------------------------ attention launchers
@@ -413,6 +493,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
   dim3 grid(p.n_qtiles, d.n_heads, B);
+  TRACE(K_ATTN_PREFILL, st);
   attn_prefill_kernel<<<grid, 192, ATT_SMEM, st>>>(tq, tk, tv, p);
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -449,14 +530,18 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cac
   p.splits = splits;
   p.keys_per_split = kps;
   dim3 grid(splits, d.n_kv_heads, B);
+  {
+  TRACE(K_ATTN_DECODE, st);
 #define DEC_CASE(HD_, G_) \
   if (hd == HD_ && grp == G_) launch_attn_decode<HD_, G_>(p, grid, st);
   DEC_CASE(64, 1) DEC_CASE(64, 2) DEC_CASE(64, 4) DEC_CASE(64, 8)
   DEC_CASE(96, 1) DEC_CASE(96, 2) DEC_CASE(96, 4) DEC_CASE(96, 8)
   DEC_CASE(128, 1) DEC_CASE(128, 2) DEC_CASE(128, 4) DEC_CASE(128, 8)
 #undef DEC_CASE
+  }
   LAUNCH_CHECK();
   if (splits > 1) {
+    TRACE(K_ATTN_COMBINE, st);
     attn_decode_combine_kernel<<<dim3(d.n_heads, B), 128, 0, st>>>(part_ml, part_o, out, d.n_heads, hd, splits);
     LAUNCH_CHECK();
   }
@@ -498,7 +583,10 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
     float* part = reinterpret_cast<float*>(ws + lay.partial);
     // a2: RMSNorm-1 -> h (bf16)
-    rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    }
     LAUNCH_CHECK();
     // a3: QKV projection
     const size_t rb = (size_t)d.dim * 2;  // bytes per weight row
@@ -513,10 +601,13 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
-    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status));
+    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
     // a4: RoPE + KV append
-    rope_append_kernel<bf><<<M, 256, 0, st>>>(qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
-                                               p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    {
+      TRACE(K_ROPE_APPEND, st);
+      rope_append_kernel<bf><<<M, 256, 0, st>>>(qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
+                                                 p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    }
     LAUNCH_CHECK();
     // a5 / a6: attention
     if (decode) {
@@ -527,15 +618,21 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     }
     // a7: o_proj + residual -> x_out holds x_mid
     WSeg so{w.wo, d.dim, 0};
-    TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status));
+    TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status,
+                  K_GEMM_O));
     // a8: RMSNorm-2 + gate_up + SiLU·mul
-    rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+    }
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
-    TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status));
+    TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
+                  K_GEMM_GATE_UP));
     // a9: down + residual (in place on x_out)
     WSeg sd{w.w2, d.dim, 0};
-    TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status));
+    TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
+                  K_GEMM_DOWN));
   } else {
     float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
     float* h = reinterpret_cast<float*>(ws + lay.h);
@@ -545,39 +642,67 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     const float* wk = static_cast<const float*>(w.wk);
     const float* wv = static_cast<const float*>(w.wv);
     auto grid_for = [](int M_, int N_) { return dim3(cdiv(N_, 64), cdiv(M_, 64)); };
-    rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+    }
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_STORE><<<grid_for(M, nh * hd), 256, 0, st>>>(h, d.dim, wq, nullptr, d.dim, M, nh * hd,
+                                                                        d.dim, qkv, qkvn, nullptr, 0);
+    }
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(h, d.dim, wk, nullptr, d.dim, M, nkv * hd,
+                                                                         d.dim, qkv + nh * hd, qkvn, nullptr, 0);
+    }
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(
+          h, d.dim, wv, nullptr, d.dim, M, nkv * hd, d.dim, qkv + (nh + nkv) * hd, qkvn, nullptr, 0);
+    }
     LAUNCH_CHECK();
-    gemm_f32_kernel<F32_STORE><<<grid_for(M, nh * hd), 256, 0, st>>>(h, d.dim, wq, nullptr, d.dim, M, nh * hd,
-                                                                      d.dim, qkv, qkvn, nullptr, 0);
-    gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(h, d.dim, wk, nullptr, d.dim, M, nkv * hd,
-                                                                       d.dim, qkv + nh * hd, qkvn, nullptr, 0);
-    gemm_f32_kernel<F32_STORE><<<grid_for(M, nkv * hd), 256, 0, st>>>(
-        h, d.dim, wv, nullptr, d.dim, M, nkv * hd, d.dim, qkv + (nh + nkv) * hd, qkvn, nullptr, 0);
-    LAUNCH_CHECK();
-    rope_append_kernel<float><<<M, 256, 0, st>>>(qkv, static_cast<float*>(kv->k), static_cast<float*>(kv->v), L, p0,
-                                                  nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    {
+      TRACE(K_ROPE_APPEND, st);
+      rope_append_kernel<float><<<M, 256, 0, st>>>(qkv, static_cast<float*>(kv->k), static_cast<float*>(kv->v), L,
+                                                    p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+    }
     LAUNCH_CHECK();
     const int Tmax = p0 + L;
     const size_t smem = (size_t)Tmax * 4;
-    if (smem > 48 * 1024) {
+    if (smem > 200 * 1024) return LLAMA_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024)
       CUDA_TRY(cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-      if (smem > 200 * 1024) return LLAMA_ERR_UNSUPPORTED;
+    {
+      TRACE(K_ATTN_F32, st);
+      attn_f32_kernel<<<dim3(L, nh, B), 128, smem, st>>>(qkv, qkvn, static_cast<const float*>(kv->k),
+                                                         static_cast<const float*>(kv->v), att, L, p0, nh, nkv, hd,
+                                                         kv->capacity);
     }
-    attn_f32_kernel<<<dim3(L, nh, B), 128, smem, st>>>(qkv, qkvn, static_cast<const float*>(kv->k),
-                                                       static_cast<const float*>(kv->v), att, L, p0, nh, nkv, hd,
-                                                       kv->capacity);
     LAUNCH_CHECK();
-    gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(att, nh * hd, static_cast<const float*>(w.wo),
-                                                                   nullptr, nh * hd, M, d.dim, nh * hd, x_out,
-                                                                   d.dim, x_in, d.dim);
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(att, nh * hd, static_cast<const float*>(w.wo),
+                                                                     nullptr, nh * hd, M, d.dim, nh * hd, x_out,
+                                                                     d.dim, x_in, d.dim);
+    }
     LAUNCH_CHECK();
-    rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
-    gemm_f32_kernel<F32_SWIGLU><<<grid_for(M, d.ffn_dim), 256, 0, st>>>(
-        h, d.dim, static_cast<const float*>(w.w1), static_cast<const float*>(w.w3), d.dim, M, d.ffn_dim, d.dim, mb,
-        d.ffn_dim, nullptr, 0);
-    gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(mb, d.ffn_dim, static_cast<const float*>(w.w2),
-                                                                   nullptr, d.ffn_dim, M, d.dim, d.ffn_dim, x_out,
-                                                                   d.dim, x_out, d.dim);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+    }
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_SWIGLU><<<grid_for(M, d.ffn_dim), 256, 0, st>>>(
+          h, d.dim, static_cast<const float*>(w.w1), static_cast<const float*>(w.w3), d.dim, M, d.ffn_dim, d.dim,
+          mb, d.ffn_dim, nullptr, 0);
+    }
+    {
+      TRACE(K_GEMM_F32, st);
+      gemm_f32_kernel<F32_RESID><<<grid_for(M, d.dim), 256, 0, st>>>(mb, d.ffn_dim, static_cast<const float*>(w.w2),
+                                                                     nullptr, d.ffn_dim, M, d.dim, d.ffn_dim, x_out,
+                                                                     d.dim, x_out, d.dim);
+    }
     LAUNCH_CHECK();
   }
   kv->length = p0 + L;
@@ -607,6 +732,60 @@ const char* llama_status_string(llama_status s) {
 }
 
 uint64_t llama_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns == 0 ? 1 : ns); }
+
+uint64_t llama_launch_count(void) { return g_launch_count.load(); }
+
+llama_status llama_profile_enable(int32_t on) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> g(t.mu);
+  t.on = on != 0;
+  return LLAMA_OK;
+}
+
+int32_t llama_profile_inflight(const char** names, int32_t n) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> g(t.mu);
+  int32_t k = 0;
+  for (const ProfRec& r : t.pending) {
+    const cudaError_t e = cudaEventQuery(r.b);
+    if (e == cudaErrorNotReady) {
+      if (names && k < n) names[k] = kKindNames[r.kind];
+      ++k;
+    } else if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+    }
+  }
+  return k;
+}
+
+int32_t llama_profile_read(const char** names, double* total_ms, long long* launches, int32_t n, int32_t reset) {
+  Tracer& t = tracer();
+  std::lock_guard<std::mutex> g(t.mu);
+  for (ProfRec& r : t.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      t.total_ms[r.kind] += ms;
+      t.launches[r.kind] += 1;
+    } else {
+      (void)cudaGetLastError();
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  t.pending.clear();
+  for (int i = 0; i < n && i < K_COUNT; ++i) {
+    if (names) names[i] = kKindNames[i];
+    if (total_ms) total_ms[i] = t.total_ms[i];
+    if (launches) launches[i] = t.launches[i];
+  }
+  if (reset) {
+    for (int i = 0; i < K_COUNT; ++i) {
+      t.total_ms[i] = 0.0;
+      t.launches[i] = 0;
+    }
+  }
+  return K_COUNT;
+}
 
 llama_status llama_kv_cache_create(const llama_dims* dims, int32_t batch, int32_t capacity, void* k_buf,
                                    void* v_buf, llama_kv_cache** out) {
@@ -718,12 +897,15 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
   float* xa = reinterpret_cast<float*>(ws + lay.xa);
   float* xb = reinterpret_cast<float*>(ws + lay.xb);
   // a1: embedding
+  {
+  TRACE(K_EMBED, st);
   if (d.dtype == LLAMA_BF16)
     embed_kernel<__nv_bfloat16><<<cdiv(M, 8), 256, 0, st>>>(
         tokens, static_cast<const __nv_bfloat16*>(m->embed), xa, M, d.dim, m->vocab, status);
   else
     embed_kernel<float><<<cdiv(M, 8), 256, 0, st>>>(tokens, static_cast<const float*>(m->embed), xa, M, d.dim,
                                                     m->vocab, status);
+  }
   LAUNCH_CHECK();
   // blocks
   for (int l = 0; l < m->n_layers; ++l) {
@@ -734,28 +916,43 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
   const float* xl = xa;
   if (seq_len > 1) {
     float* g = reinterpret_cast<float*>(ws + lay.xl);
-    gather_last_rows_kernel<<<dim3(cdiv(d.dim, 256), batch), 256, 0, st>>>(xa, g, seq_len, d.dim);
+    {
+      TRACE(K_GATHER_LAST, st);
+      gather_last_rows_kernel<<<dim3(cdiv(d.dim, 256), batch), 256, 0, st>>>(xa, g, seq_len, d.dim);
+    }
     LAUNCH_CHECK();
     xl = g;
   }
   float* logits = logits_or_null ? logits_or_null : reinterpret_cast<float*>(ws + lay.logits);
   if (d.dtype == LLAMA_BF16) {
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
-    rmsnorm_kernel<__nv_bfloat16><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
-                                                                   d.eps);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<__nv_bfloat16><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
+                                                                     d.eps);
+    }
     LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};
     TRY(gemm_bf16(st, true, hl, batch, d.dim, &s, 1, EPI_F32, logits, m->vocab, nullptr, 0,
-                  reinterpret_cast<float*>(ws + lay.partial), status));
+                  reinterpret_cast<float*>(ws + lay.partial), status, K_GEMM_LM_HEAD));
   } else {
     float* hl = reinterpret_cast<float*>(ws + lay.hl);
-    rmsnorm_kernel<float><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
-    gemm_f32_kernel<F32_STORE><<<dim3(cdiv(m->vocab, 64), cdiv(batch, 64)), 256, 0, st>>>(
-        hl, d.dim, static_cast<const float*>(m->lm_head), nullptr, d.dim, batch, m->vocab, d.dim, logits, m->vocab,
-        nullptr, 0);
+    {
+      TRACE(K_RMSNORM, st);
+      rmsnorm_kernel<float><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
+    }
+    {
+      TRACE(K_GEMM_LM_HEAD, st);
+      gemm_f32_kernel<F32_STORE><<<dim3(cdiv(m->vocab, 64), cdiv(batch, 64)), 256, 0, st>>>(
+          hl, d.dim, static_cast<const float*>(m->lm_head), nullptr, d.dim, batch, m->vocab, d.dim, logits,
+          m->vocab, nullptr, 0);
+    }
     LAUNCH_CHECK();
   }
-  argmax_kernel<<<batch, 1024, 0, st>>>(logits, m->vocab, next_ids);
+  {
+    TRACE(K_ARGMAX, st);
+    argmax_kernel<<<batch, 1024, 0, st>>>(logits, m->vocab, next_ids);
+  }
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
@@ -764,8 +961,11 @@ llama_status llama_selftest_wait_timeout(void* workspace, uint64_t limit_ns, voi
   if (workspace == nullptr) return LLAMA_ERR_INVALID_ARG;
   if (!aligned16(workspace)) return LLAMA_ERR_ALIGNMENT;
   if (limit_ns > 5000000000ull) return LLAMA_ERR_INVALID_ARG;
-  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<DevStatus*>(workspace),
-                                                                      limit_ns);
+  {
+    TRACE(K_SELFTEST, static_cast<cudaStream_t>(stream));
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<DevStatus*>(workspace),
+                                                                        limit_ns);
+  }
   LAUNCH_CHECK();
   return LLAMA_OK;
 }

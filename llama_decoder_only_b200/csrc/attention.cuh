@@ -232,13 +232,17 @@ __global__ void __launch_bounds__(192, 1)
         s[i] = x;
         mx = fmaxf(mx, x);
       }
-      bool rescale = false;
+      // Move this row's reference maximum only when it grew by more than
+      // 2^8; rows that keep theirs use alpha = 1.  The O rescale below is a
+      // warp-collective TMEM read-modify-write, so the warp does it when any
+      // of its rows needs it.
       float alpha = 1.f;
-      if (mx > m_used + 8.0f) {
+      const bool need = mx > m_used + 8.0f;
+      if (need) {
         alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - mx);
         m_used = mx;
-        rescale = j > 0;
       }
+      const bool rescale = __any_sync(0xffffffffu, need && j > 0);
       // wait until the previous P·V has finished (O stable, P buffer free)
       if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, wc, 11))) {
         ok = false;

@@ -29,12 +29,24 @@ def rel_errors(gpu, ref):
     return float(np.max(np.abs(d))) / rms, float(np.sqrt(np.mean(d * d))) / rms
 
 
-def ulp_err(gpu, ref):
-    """Largest |gpu - ref| / (|ref| + 0.05 RMS(ref)): about 2**-8 per bf16 ulp."""
+def ulp_rms_err(gpu, ref, ulps=2, rms_frac=1e-2):
+    """Largest |gpu - ref| / (ulps * 2**-8 |ref| + rms_frac RMS(ref)); <= 1 passes."""
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     rms = float(np.sqrt(np.mean(ref * ref)))
-    return float(np.max(np.abs(gpu - ref) / (np.abs(ref) + 0.05 * rms)))
+    return float(np.max(np.abs(gpu - ref) / (ulps * 2.0 ** -8 * np.abs(ref) + rms_frac * rms)))
+
+
+def floor_ratios(gpu, rounded, exact):
+    """Error of ``gpu`` against ``exact`` divided by the error of the bf16-rounded
+    oracle against ``exact``: (RMS ratio, max-abs ratio)."""
+    gpu, rounded, exact = (np.asarray(a, np.float64) for a in (gpu, rounded, exact))
+    rms = float(np.sqrt(np.mean(exact * exact)))
+    eg, eb = gpu - exact, rounded - exact
+    tiny = 1e-4 * rms
+    r_rms = float(np.sqrt(np.mean(eg * eg))) / (float(np.sqrt(np.mean(eb * eb))) + tiny)
+    r_max = float(np.max(np.abs(eg))) / (float(np.max(np.abs(eb))) + tiny)
+    return r_rms, r_max
 
 
 class LayerRun:

@@ -7,7 +7,14 @@ Tolerances (written here, derived in the design notes):
   against the exact oracle the RMS error must stay <= 1e-2 x RMS and the
   max-abs error <= 5e-2 x RMS (bf16 operand rounding alone reaches ~3e-2).
 * intermediates (q, k, v, attention output, norm output, SwiGLU product):
-  within two bf16 ulps of the rounded oracle value (``ulp_err <= 2**-7``).
+  their error against the EXACT oracle, measured as RMS and as max-abs, must
+  stay within 1.5x (RMS) and 2x (max) of the bf16 rounding floor -- the same
+  error of the bf16-rounded oracle.  (Both sides round these tensors to bf16,
+  but not always the same way: the GPU rounds the attention probabilities
+  unnormalised, in flash form, and the oracle rounds them normalised; and an
+  element that sits within fp32 accumulation error of a rounding boundary can
+  land one ulp apart.  An element-wise comparison of the two rounded tensors
+  therefore mostly measures rounding noise, not the kernel.)
 """
 
 import numpy as np
@@ -15,7 +22,7 @@ import pytest
 
 import synth
 from oracle import block as ob
-from tests.harness import LayerRun, oracle_dims, rel_errors, ulp_err
+from tests.harness import LayerRun, floor_ratios, oracle_dims, rel_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -24,20 +31,32 @@ torch = pytest.importorskip("torch")
 BF16_MAX = 1e-2
 BF16_EXACT_RMS = 1e-2
 BF16_EXACT_MAX = 5e-2
-ULP2 = 2.0 ** -7
 F32_MAX = 1e-4
+FLOOR_RMS = 1.5
+FLOOR_MAX = 2.0
 
 
-def check_bf16_block(run, W, x, d, cache_b, cache_x, label):
+def check_bf16_block(run, W, x, d, cache_b, cache_x, label, absolute=True):
     y = run.step(x)
     inter = run.intermediates()
     yb, pb = ob.layer_forward(d, W, x, cache_b, rounding="bf16")
-    ye, _ = ob.layer_forward(d, W, x, cache_x)
-    mx, _ = rel_errors(y, yb)
+    ye, pe = ob.layer_forward(d, W, x, cache_x)
+    mx, rmsb = rel_errors(y, yb)
     mxe, rmse = rel_errors(y, ye)
-    for name in ("q", "k", "v", "attn", "h2", "m"):
-        e = ulp_err(inter[name], pb[name])
-        assert e <= ULP2, f"{label}: intermediate {name} off by {e:.3g} (relative)"
+    inter_err = {n: floor_ratios(inter[n], pb[n], pe[n]) for n in ("q", "k", "v", "attn", "h2", "m")}
+    print(f"[parity] {label}: out max/RMS vs bf16-oracle {mx:.3g} (rms {rmsb:.3g}); vs exact {mxe:.3g} "
+          f"(rms {rmse:.3g}); intermediates (rms, max) / bf16 floor: "
+          + " ".join(f"{k}=({v[0]:.2f},{v[1]:.2f})" for k, v in inter_err.items()))
+    for name, (r_rms, r_max) in inter_err.items():
+        assert r_rms <= FLOOR_RMS and r_max <= FLOOR_MAX, \
+            f"{label}: intermediate {name} error / bf16 floor = rms {r_rms:.3g}, max {r_max:.3g}"
+    if not absolute:
+        # stress inputs outside the workloads' distributions: the output is held
+        # to the bf16 floor instead of the absolute bar
+        r_rms, r_max = floor_ratios(y, yb, ye)
+        print(f"[parity] {label}: output error / bf16 floor = rms {r_rms:.2f}, max {r_max:.2f}")
+        assert r_rms <= FLOOR_RMS and r_max <= FLOOR_MAX
+        return mx, mxe, rmse
     assert mx <= BF16_MAX, f"{label}: max-abs/RMS vs bf16-rounded oracle {mx:.3g}"
     assert rmse <= BF16_EXACT_RMS, f"{label}: rms/RMS vs exact oracle {rmse:.3g}"
     assert mxe <= BF16_EXACT_MAX, f"{label}: max-abs/RMS vs exact oracle {mxe:.3g}"
@@ -94,6 +113,20 @@ def test_bf16_prefill_parity(case):
     cb = ob.KVCache(w.batch, w.n_kv_heads, w.head_dim, 512)
     ce = ob.KVCache(w.batch, w.n_kv_heads, w.head_dim, 512)
     check_bf16_block(run, inp.weights, inp.x, d, cb, ce, case[0])
+
+
+def test_bf16_prefill_large_scores_rescale_path():
+    # Large weights give attention scores with a std of ~10 (log2 units), so the
+    # running row maximum jumps past the 2^8 threshold at different tiles for
+    # different rows of one warp: exercises the warp-uniform O rescale.
+    w = synth.Workload("large_scores", 512, 8, 2, 64, 1376, 1e-5, 1e4, "half", "bf16", 0.08, 5,
+                       batch=1, prefill_len=700)
+    inp = synth.prefill_inputs(w, with_steps=False)
+    d = oracle_dims(w)
+    run = LayerRun(w, inp.weights, 1, 768, 700)
+    cb = ob.KVCache(1, w.n_kv_heads, w.head_dim, 768)
+    ce = ob.KVCache(1, w.n_kv_heads, w.head_dim, 768)
+    check_bf16_block(run, inp.weights, inp.x, d, cb, ce, "large_scores", absolute=False)
 
 
 def test_bf16_prefill_separate_weight_buffers():
