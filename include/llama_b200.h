@@ -54,7 +54,8 @@ typedef enum llama_status {
   LLAMA_ERR_ALIGNMENT = 4,           /* a device pointer is not 16-byte aligned */
   LLAMA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < the *_workspace_size query */
   LLAMA_ERR_CUDA = 6,                /* a CUDA runtime/driver call failed */
-  LLAMA_ERR_DEVICE_TIMEOUT = 7       /* a bounded device wait ran out (read via llama_device_status) */
+  LLAMA_ERR_DEVICE_TIMEOUT = 7,      /* a bounded device wait ran out (read via llama_device_status) */
+  LLAMA_ERR_SCRATCH_LIMIT = 8        /* llama_attention_decode_noalloc: more than its fixed scratch */
 } llama_status;
 
 /* RoPE variant.  HALF: rotate-half, x*cos(emb) + cat(-x2, x1)*sin(emb) with
@@ -212,6 +213,38 @@ size_t llama_model_workspace_size(const llama_model* model, int32_t batch, int32
 llama_status llama_model_forward(const llama_model* model, llama_kv_cache* const* caches, const int32_t* tokens,
                                  int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ allocation-free decode attention */
+
+/* The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory -- a plug-in inside a serving framework
+ * that reserved all GPU memory for its own pool and hands out no workspace,
+ * or a latency-critical loop that must not call cudaMalloc (which may
+ * synchronise the device).  It is the split-KV decode attention of
+ * llama_layer_decode on its own, with its partial results kept in a fixed
+ * 8 MiB array that is part of the library (every GPU that loads the library
+ * holds it until the process exits) instead of in a workspace.  It allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *
+ *   q        device bf16 [batch, ld_q]: query head h of sequence b at
+ *            q[b*ld_q + h*head_dim ...] (already rotated); ld_q >= n_heads*head_dim,
+ *            ld_q % 8 == 0 (e.g. the q part of a packed q|k|v row)
+ *   k_cache, v_cache  device bf16 [batch][n_kv_heads][capacity][head_dim]
+ *   length   keys 0 .. length-1 are attended (1 <= length <= capacity)
+ *   out      device bf16 [batch, n_heads*head_dim]
+ * out[b, h] = softmax(q_bh k^T / sqrt(head_dim)) v over those keys, KV head
+ * h / (n_heads/n_kv_heads).  dims->dtype must be LLAMA_BF16.
+ * Limit: batch * n_heads * (head_dim + 2) * 8 bytes <= 8 MiB (two key
+ * splits), else LLAMA_ERR_SCRATCH_LIMIT; the call then enqueues nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and nothing in it needs to start
+ * at zero; two calls that overlap on the GPU (different streams, or
+ * different host threads without ordering) race on it.
+ * Errors: INVALID_ARG, UNSUPPORTED (fp32 dims), ALIGNMENT, SCRATCH_LIMIT, CUDA. */
+llama_status llama_attention_decode_noalloc(const llama_dims* dims, int32_t batch, const void* q, int32_t ld_q,
+                                            const void* k_cache, const void* v_cache, int32_t capacity,
+                                            int32_t length, void* out, void* stream);
 
 /* ------------------------------------------------------------------ misc */
 

@@ -24,7 +24,7 @@ __all__ = [
     "make_dims", "layer_weights", "model_struct", "KVCache",
     "workspace_size", "model_workspace_size", "layer_prefill", "layer_decode",
     "model_forward", "device_status", "workspace_offsets", "set_wait_limit_ns", "selftest_wait_timeout",
-    "launch_count", "profile_enable", "profile_read", "profile_inflight",
+    "launch_count", "profile_enable", "profile_read", "profile_inflight", "attention_decode_noalloc",
 ]
 
 F32, BF16 = 0, 1
@@ -33,7 +33,7 @@ ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 STATUS = {
     0: "LLAMA_OK", 1: "LLAMA_ERR_INVALID_ARG", 2: "LLAMA_ERR_UNSUPPORTED", 3: "LLAMA_ERR_CACHE_FULL",
     4: "LLAMA_ERR_ALIGNMENT", 5: "LLAMA_ERR_WORKSPACE_TOO_SMALL", 6: "LLAMA_ERR_CUDA",
-    7: "LLAMA_ERR_DEVICE_TIMEOUT",
+    7: "LLAMA_ERR_DEVICE_TIMEOUT", 8: "LLAMA_ERR_SCRATCH_LIMIT",
 }
 
 
@@ -86,6 +86,7 @@ EXPORTS = {
     "llama_model_workspace_size": (_S, [_MP, _I, _I]),
     "llama_model_forward": (_I, [_MP, ctypes.POINTER(_P), _P, _I, _I, _P, _P, _P, _S, _P]),
     "llama_selftest_wait_timeout": (_I, [_P, _U64, _P]),
+    "llama_attention_decode_noalloc": (_I, [_DP, _I, _P, _I, _P, _P, _I, _I, _P, _P]),
     "llama_launch_count": (_U64, []),
     "llama_profile_enable": (_I, [_I]),
     "llama_profile_inflight": (_I, [ctypes.POINTER(ctypes.c_char_p), _I]),
@@ -244,6 +245,13 @@ def profile_inflight(n=64):
     names = (ctypes.c_char_p * n)()
     k = lib().llama_profile_inflight(names, n)
     return k, [names[i].decode() for i in range(min(k, n))]
+
+
+def attention_decode_noalloc(dims, batch, q, ld_q, k_cache, v_cache, capacity, length, out, stream=None):
+    """Decode attention with its scratch in the library's fixed array (see the C header)."""
+    _check(lib().llama_attention_decode_noalloc(ctypes.byref(dims), batch, _ptr(q), ld_q, _ptr(k_cache),
+                                                _ptr(v_cache), capacity, length, _ptr(out), _stream(stream)),
+           "llama_attention_decode_noalloc")
 
 
 def set_wait_limit_ns(ns):

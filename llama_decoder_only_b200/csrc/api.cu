@@ -727,6 +727,7 @@ const char* llama_status_string(llama_status s) {
     case LLAMA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case LLAMA_ERR_CUDA: return "CUDA error";
     case LLAMA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case LLAMA_ERR_SCRATCH_LIMIT: return "request exceeds the fixed scratch of the allocation-free entry point";
   }
   return "unknown status";
 }
@@ -971,3 +972,97 @@ llama_status llama_selftest_wait_timeout(void* workspace, uint64_t limit_ns, voi
 }
 
 }  // extern "C"
+
+// ====================================================================== decode attention, no allocation
+//
+// For callers that cannot allocate device memory at all -- for example code
+// running inside a serving framework that has reserved all GPU memory for its
+// own pool and gives a plug-in no workspace, or a real-time loop that must not
+// call cudaMalloc (which can synchronise the device) -- this variant of the
+// split-KV decode attention keeps its partial results in a fixed array that is
+// part of the library image instead of in a caller-provided workspace.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB, held on every GPU that loads the library
+__device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+llama_status noalloc_scratch(float** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return LLAMA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return LLAMA_OK;
+}
+
+}  // namespace
+
+extern "C" llama_status llama_attention_decode_noalloc(const llama_dims* dims, int32_t batch, const void* q,
+                                                       int32_t ld_q, const void* k_cache, const void* v_cache,
+                                                       int32_t capacity, int32_t length, void* out, void* stream) {
+  TRY(check_dims(dims));
+  const llama_dims& d = *dims;
+  if (d.dtype != LLAMA_BF16) return LLAMA_ERR_UNSUPPORTED;
+  if (batch <= 0 || q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr)
+    return LLAMA_ERR_INVALID_ARG;
+  if (length <= 0 || capacity < length || ld_q < d.n_heads * d.head_dim) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || (ld_q % 8) != 0)
+    return LLAMA_ERR_ALIGNMENT;
+  const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  // partials of `splits` key ranges per (sequence, query head): (max, sum) and hd outputs
+  const size_t per_split = (size_t)batch * d.n_heads * (hd + 2) * sizeof(float);
+  const size_t max_splits = kNoAllocScratchBytes / per_split;
+  if (max_splits < 2) return LLAMA_ERR_SCRATCH_LIMIT;
+  int splits = cdiv(4 * num_sms(), batch * d.n_kv_heads);
+  splits = std::max(2, std::min({splits, (int)std::min<size_t>(max_splits, kMaxAttnSplits), cdiv(length, 32)}));
+  int kps = cdiv(cdiv(length, splits), 32) * 32;
+  splits = cdiv(length, kps);
+  float* scratch = nullptr;
+  TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnDecodeParams p{};
+  p.qkv = static_cast<const __nv_bfloat16*>(q);
+  p.ld_qkv = ld_q;
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.cap = capacity;
+  p.T = length;
+  p.nh = d.n_heads;
+  p.nkv = d.n_kv_heads;
+  p.scale_log2 = kLog2e / sqrtf((float)hd);
+  p.splits = splits;
+  p.keys_per_split = kps;
+  p.part_ml = scratch;
+  p.part_o = scratch + (size_t)batch * d.n_heads * splits * 2;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  dim3 grid(splits, d.n_kv_heads, batch);
+  {
+    TRACE(K_ATTN_DECODE, st);
+#define NOALLOC_CASE(HD_, G_) \
+  if (hd == HD_ && grp == G_) launch_attn_decode<HD_, G_>(p, grid, st);
+    NOALLOC_CASE(64, 1) NOALLOC_CASE(64, 2) NOALLOC_CASE(64, 4) NOALLOC_CASE(64, 8)
+    NOALLOC_CASE(96, 1) NOALLOC_CASE(96, 2) NOALLOC_CASE(96, 4) NOALLOC_CASE(96, 8)
+    NOALLOC_CASE(128, 1) NOALLOC_CASE(128, 2) NOALLOC_CASE(128, 4) NOALLOC_CASE(128, 8)
+#undef NOALLOC_CASE
+  }
+  LAUNCH_CHECK();
+  if (splits > 1) {
+    TRACE(K_ATTN_COMBINE, st);
+    attn_decode_combine_kernel<<<dim3(d.n_heads, batch), 128, 0, st>>>(p.part_ml, p.part_o, p.out, d.n_heads, hd,
+                                                                        splits);
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
