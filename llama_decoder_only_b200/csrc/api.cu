@@ -487,14 +487,14 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.nh = d.n_heads;
   p.nkv = d.n_kv_heads;
   p.hd = hd;
-  p.n_qtiles = cdiv(L, 128);
+  p.n_qblocks = cdiv(L, 256);
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
-  dim3 grid(p.n_qtiles, d.n_heads, B);
+  dim3 grid(p.n_qblocks, d.n_heads, B);
   TRACE(K_ATTN_PREFILL, st);
-  attn_prefill_kernel<<<grid, 192, ATT_SMEM, st>>>(tq, tk, tv, p);
+  attn_prefill_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(tq, tk, tv, p);
   LAUNCH_CHECK();
   return LLAMA_OK;
 }

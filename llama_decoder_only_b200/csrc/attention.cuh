@@ -3,11 +3,13 @@
 //  * attn_prefill_kernel: flash attention on tcgen05 ([HandsOn] "Transformer
 //    块的内部结构" names FlashAttention: tile Q/K/V through on-chip memory
 //    instead of materialising the score matrix in HBM).  One CTA per
-//    (128-query tile, head, sequence); K/V tiles of 128 keys arrive by TMA
-//    into a 2-stage ring; S = Q K^T lands in TMEM (double-buffered), the
-//    softmax warps read it with tcgen05.ld, keep the running max / sum in
-//    fp32 (online softmax), write P as bf16 into shared memory and the MMA
-//    warp accumulates O += P V in TMEM.  The running max is only moved (and
+//    (256-query block, head, sequence) = two 128-row query tiles that share
+//    every K/V tile; K/V tiles of 128 keys arrive by TMA into a 3-slot ring;
+//    S_t = Q_t K^T lands in TMEM, a softmax warpgroup per tile reads it with
+//    tcgen05.ld, keeps the running max / sum in fp32 (online softmax), writes
+//    P_t as bf16 into shared memory, and the MMA warp accumulates
+//    O_t += P_t V in TMEM; the two tiles ping-pong so one tile's softmax
+//    overlaps the other tile's MMAs.  The running max is only moved (and
 //    O rescaled) when it grows by more than 2^8, which is exact because the
 //    final division uses the same stale maximum for numerator and sum.
 //  * attn_decode_kernel + attn_decode_combine_kernel: one new query per
@@ -33,70 +35,81 @@ struct AttnPrefillParams {
   int L;         // new tokens per sequence
   int p0;        // position of token 0 (cache length before the call)
   int nh, nkv, hd;
-  int n_qtiles;
+  int n_qblocks; // blocks of 256 query rows (two 128-row tiles)
   float scale_log2;   // log2(e) / sqrt(hd)
   __nv_bfloat16* out; // [B*L, nh*hd]
   DevStatus* status;
   unsigned long long limit_ns;
 };
 
-constexpr int ATT_NS = 2;                       // K/V ring stages
 constexpr int ATT_REGION = 128 * 128;           // bytes of a [128 rows x 64 bf16] region
-constexpr int ATT_SMEM = 1024 + 2 * ATT_REGION        // Q
-                         + ATT_NS * 4 * ATT_REGION    // K, V (2 regions each)
-                         + 2 * ATT_REGION             // P
+constexpr int ATT_TILE = 2 * ATT_REGION;        // one 128-row tile of a head (two 64-column regions)
+constexpr int ATT_SLOTS = 3;                    // K/V ring: K_j, V_j, K_{j+1} in flight
+constexpr int ATT_THREADS = 320;                // producer, MMA, 2 softmax warpgroups
+constexpr int ATT_SMEM = 1024 + 2 * ATT_TILE    // Q0, Q1
+                         + ATT_SLOTS * ATT_TILE  // K/V ring
+                         + 2 * ATT_TILE          // P0, P1
                          + 256;
 
-__global__ void __launch_bounds__(192, 1)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two 128-row query tiles (t = 0, 1) of one head share every K/V tile.  The
+// MMA warp interleaves S1_j, P0·V_j, S0_{j+1}, P1·V_j, so while one softmax
+// warpgroup turns S_t into P_t the tensor core works on the other tile.
+__global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnPrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + 2 * ATT_REGION;          // stage s: K at s*4R, V at s*4R + 2R
-  uint8_t* sP = sKV + ATT_NS * 4 * ATT_REGION;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * ATT_REGION);
-  // bars: q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full, pv_done, drain
+  uint8_t* sQ = smem;                                   // tile t at t * ATT_TILE
+  uint8_t* sKV = sQ + 2 * ATT_TILE;                     // slot s at s * ATT_TILE
+  uint8_t* sP = sKV + ATT_SLOTS * ATT_TILE;             // tile t at t * ATT_TILE
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * ATT_TILE);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.n_qtiles - 1 - blockIdx.x;   // heavy (late) tiles first
+  const int qb = p.n_qblocks - 1 - blockIdx.x;   // heavy (late) blocks first
   const int h = blockIdx.y, b = blockIdx.z;
   const int g = h / (p.nh / p.nkv);
   const int hd = p.hd;
   const int nreg = hd > 64 ? 2 : 1;             // 64-column regions per head row
   const int hd_pad = nreg * 64;
-  const int q_row0 = qt * 128;                  // first token of the tile
-  const int last_q = min(p.L, q_row0 + 128) - 1;
-  const int n_kv = (p.p0 + last_q) / 128 + 1;   // kv tiles with any visible key
-  const int pos_min = p.p0 + q_row0;
+  const int q_row0 = qb * 256;
+  const bool q1_valid = q_row0 + 128 < p.L;
+  // kv tiles with any key visible to tile t (0 for an empty tile)
+  const int last0 = min(p.L, q_row0 + 128) - 1;
+  const int n_kv0 = (p.p0 + last0) / 128 + 1;
+  const int n_kv1 = q1_valid ? (p.p0 + min(p.L, q_row0 + 256) - 1) / 128 + 1 : 0;
+  const int n_kv = max(n_kv0, n_kv1);
 
   const uint32_t bar0 = smem_u32(bars);
   const uint32_t q_full = bar0;
-  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (1 + ATT_NS + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * ATT_NS + s); };
-  auto s_full = [&](int i) { return bar0 + 8u * (1 + 3 * ATT_NS + i); };
-  auto s_free = [&](int i) { return bar0 + 8u * (3 + 3 * ATT_NS + i); };
-  const uint32_t p_full = bar0 + 8u * (5 + 3 * ATT_NS);
-  const uint32_t pv_done = bar0 + 8u * (6 + 3 * ATT_NS);
-  const uint32_t drain = bar0 + 8u * (7 + 3 * ATT_NS);
+  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ATT_SLOTS + s); };
+  auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * ATT_SLOTS + t); };
+  auto s_free = [&](int t) { return bar0 + 8u * (3 + 2 * ATT_SLOTS + t); };
+  auto p_full = [&](int t) { return bar0 + 8u * (5 + 2 * ATT_SLOTS + t); };
+  auto pv_done = [&](int t) { return bar0 + 8u * (7 + 2 * ATT_SLOTS + t); };
+  const uint32_t drain = bar0 + 8u * (9 + 2 * ATT_SLOTS);
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(q_full, 1);
-    for (int s = 0; s < ATT_NS; ++s) {
-      mbar_init(k_full(s), 1);
-      mbar_init(v_full(s), 1);
+    for (int s = 0; s < ATT_SLOTS; ++s) {
+      mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(s_free(t), 128);
+      mbar_init(p_full(t), 128);
+      mbar_init(pv_done(t), 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -112,36 +125,33 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_base_sh;   // S0 at col 0, S1 at col 128, O at col 256
+  const uint32_t tmem = tmem_base_sh;   // S_t at col 128 t, O_t at col 256 + 128 t
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, 3};
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int filled[ATT_NS] = {};
-      mbar_arrive_expect_tx(q_full, nreg * ATT_REGION);
-      for (int r = 0; r < nreg; ++r)
-        tma_load_3d(smem_u32(sQ + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64, q_row0, b);
-      const int zkv = b * p.nkv + g;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % ATT_NS;
-        if (!mbar_wait(kv_empty(s), ((j / ATT_NS) & 1) ^ 1u, wc, 1)) break;
-        uint8_t* st = sKV + s * 4 * ATT_REGION;
-        mbar_arrive_expect_tx(k_full(s), nreg * ATT_REGION);
-        for (int r = 0; r < nreg; ++r) tma_load_3d(smem_u32(st + r * ATT_REGION), &tmK, k_full(s), r * 64, j * 128, zkv);
-        mbar_arrive_expect_tx(v_full(s), nreg * ATT_REGION);
+      int last_fill[ATT_SLOTS] = {-1, -1, -1};
+      const int nq = q1_valid ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * nreg * ATT_REGION);
+      for (int t = 0; t < nq; ++t)
         for (int r = 0; r < nreg; ++r)
-          tma_load_3d(smem_u32(st + (2 + r) * ATT_REGION), &tmV, v_full(s), r * 64, j * 128, zkv);
-        filled[s] = j + 1;
+          tma_load_3d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64,
+                      q_row0 + t * 128, b);
+      const int zkv = b * p.nkv + g;
+      for (int f = 0; f < 2 * n_kv; ++f) {   // fill f: K_{f/2} (f even) or V_{f/2} (f odd)
+        const int s = f % ATT_SLOTS;
+        if (!mbar_wait(kv_empty(s), ((f / ATT_SLOTS) & 1) ^ 1u, wc, 1)) break;
+        const CUtensorMap* m = (f & 1) ? &tmV : &tmK;
+        mbar_arrive_expect_tx(kv_full(s), nreg * ATT_REGION);
+        for (int r = 0; r < nreg; ++r)
+          tma_load_3d(smem_u32(sKV + s * ATT_TILE + r * ATT_REGION), m, kv_full(s), r * 64, (f >> 1) * 128, zkv);
+        last_fill[s] = f;
       }
       // drain own copies before exit
       mbar_wait(q_full, 0, wc, 9, false);
-      for (int s = 0; s < ATT_NS; ++s)
-        if (filled[s] > 0) {
-          const uint32_t par = ((filled[s] - 1) / ATT_NS) & 1;
-          mbar_wait(k_full(s), par, wc, 9, false);
-          mbar_wait(v_full(s), par, wc, 9, false);
-        }
+      for (int s = 0; s < ATT_SLOTS; ++s)
+        if (last_fill[s] >= 0) mbar_wait(kv_full(s), (last_fill[s] / ATT_SLOTS) & 1, wc, 9, false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -151,45 +161,54 @@ __global__ void __launch_bounds__(192, 1)
       const int ksteps = hd / 16;
       bool ok = mbar_wait(q_full, 0, wc, 2);
       bool issued = false;
-      const uint32_t aQ = smem_u32(sQ);
-      const uint32_t aP = smem_u32(sP);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % ATT_NS, sb = j & 1;
-        if (!mbar_wait(k_full(s), (j / ATT_NS) & 1, wc, 3)) return false;
-        if (!mbar_wait(s_free(sb), ((j >> 1) & 1) ^ 1u, wc, 4)) return false;
+      int s_count[2] = {0, 0};
+      auto slot_ready = [&](int f) -> bool {   // wait for fill f of the ring
+        return mbar_wait(kv_full(f % ATT_SLOTS), (f / ATT_SLOTS) & 1, wc, 3);
+      };
+      auto issue_s = [&](int t, int j) -> bool {
+        if (!mbar_wait(s_free(t), (s_count[t] & 1) ^ 1u, wc, 4)) return false;
         tc_fence_after();
-        const uint32_t aK = smem_u32(sKV + s * 4 * ATT_REGION);
+        const uint32_t aQ = smem_u32(sQ + t * ATT_TILE);
+        const uint32_t aK = smem_u32(sKV + ((2 * j) % ATT_SLOTS) * ATT_TILE);
         for (int ks = 0; ks < ksteps; ++ks) {
           const uint32_t off = (ks >> 2) * ATT_REGION + (ks & 3) * 32;
-          umma_bf16(tmem + sb * 128, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(aK + off, 16, 1024),
+          umma_bf16(tmem + t * 128, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(aK + off, 16, 1024),
                     idesc_s, ks > 0 ? 1u : 0u);
         }
-        umma_commit(s_full(sb));
+        umma_commit(s_full(t));
+        ++s_count[t];
         issued = true;
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int s = j % ATT_NS;
-        if (!mbar_wait(p_full, j & 1, wc, 5)) return false;
-        if (!mbar_wait(v_full(s), (j / ATT_NS) & 1, wc, 6)) return false;
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait(p_full(t), j & 1, wc, 5)) return false;
         tc_fence_after();
-        const uint32_t aV = smem_u32(sKV + s * 4 * ATT_REGION + 2 * ATT_REGION);
+        const uint32_t aP = smem_u32(sP + t * ATT_TILE);
+        const uint32_t aV = smem_u32(sKV + ((2 * j + 1) % ATT_SLOTS) * ATT_TILE);
         for (int ks = 0; ks < 8; ++ks) {   // 128 keys, 16 per MMA
           const uint32_t pa = aP + (ks >> 2) * ATT_REGION + (ks & 3) * 32;
           const uint32_t va = aV + ks * 16 * 128;
-          umma_bf16(tmem + 256, smem_desc_sw128(pa, 16, 1024), smem_desc_sw128(va, ATT_REGION, 1024), idesc_o,
-                    (j > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16(tmem + 256 + t * 128, smem_desc_sw128(pa, 16, 1024), smem_desc_sw128(va, ATT_REGION, 1024),
+                    idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(pv_done);
-        umma_commit(kv_empty(s));
+        umma_commit(pv_done(t));
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 1; ok && j < n_kv; ++j) {
-        ok = issue_s(j);
-        if (ok) ok = issue_pv(j - 1);
+      if (ok && n_kv0 > 0) ok = slot_ready(0) && issue_s(0, 0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const bool a0 = j < n_kv0, a1 = j < n_kv1;
+        if (a1) {
+          if (!a0) ok = slot_ready(2 * j);   // K_j not waited for by tile 0
+          if (ok) ok = issue_s(1, j);
+        }
+        if (!ok) break;
+        umma_commit(kv_empty((2 * j) % ATT_SLOTS));          // K_j free once its S MMAs finish
+        if (!slot_ready(2 * j + 1)) break;                  // V_j
+        if (a0 && !issue_pv(0, j)) break;
+        if (j + 1 < n_kv0 && !(slot_ready(2 * j + 2) && issue_s(0, j + 1))) break;
+        if (a1 && !issue_pv(1, j)) break;
+        umma_commit(kv_empty((2 * j + 1) % ATT_SLOTS));      // V_j free once its P·V MMAs finish
       }
-      if (ok) issue_pv(n_kv - 1);
       if (issued) {
         umma_commit(drain);
         mbar_wait(drain, 0, wc, 8, false);
@@ -197,17 +216,21 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / correction / epilogue
+    const int t = (warp - 2) >> 2;             // query tile of this warpgroup
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int t = q_row0 + row;                // token within the sequence
-    const int pos = p.p0 + t;
+    const int tok = q_row0 + t * 128 + row;    // token within the sequence
+    const int pos = p.p0 + tok;
+    const int pos_min = p.p0 + q_row0 + t * 128;
+    const int my_kv = t == 0 ? n_kv0 : n_kv1;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow0 = sP + row * 128;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(sb), (j >> 1) & 1, wc, 10))) {
+    uint8_t* prow0 = sP + t * ATT_TILE + row * 128;
+    for (int j = 0; j < my_kv && ok; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(t), j & 1, wc, 10))) {
         ok = false;
         break;
       }
@@ -216,13 +239,13 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_off + sb * 128 + c * 32, v);
+        tmem_ld32(tS + c * 32, v);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
       }
       tc_fence_before();
-      mbar_arrive(s_free(sb));
+      mbar_arrive(s_free(t));
       const bool need_mask = j * 128 + 127 > pos_min;
       float mx = -INFINITY;
 #pragma unroll
@@ -239,12 +262,12 @@ __global__ void __launch_bounds__(192, 1)
       float alpha = 1.f;
       const bool need = mx > m_used + 8.0f;
       if (need) {
-        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - mx);
+        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mx);
         m_used = mx;
       }
       const bool rescale = __any_sync(0xffffffffu, need && j > 0);
-      // wait until the previous P·V has finished (O stable, P buffer free)
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, wc, 11))) {
+      // the previous P·V of this tile must be done (O stable, P buffer free)
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done(t), (j - 1) & 1, wc, 11))) {
         ok = false;
         break;
       }
@@ -253,27 +276,26 @@ __global__ void __launch_bounds__(192, 1)
         l *= alpha;
         for (int c = 0; c < hd_pad; c += 32) {
           float v[32];
-          tmem_ld32(tmem + lane_off + 256 + c, v);
+          tmem_ld32(tO + c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(tmem + lane_off + 256 + c, v);
+          tmem_st32(tO + c, v);
         }
         tmem_st_wait();
       }
-      // P = exp2(s - m_used) as bf16 into the swizzled K-major A tile
+      // P = 2^(s - m_used) as bf16 into the swizzled K-major A tile
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
       float psum = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {   // 16-byte chunk c holds keys 8c .. 8c+7
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = (m_used == -INFINITY) ? 0.f : exp2f(s[8 * c + 2 * e] - m_used);
-          const float bb = (m_used == -INFINITY) ? 0.f : exp2f(s[8 * c + 2 * e + 1] - m_used);
-          __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
-          const float2 back = __bfloat1622float2(hv);
-          psum += back.x + back.y;
-          w[e] = *reinterpret_cast<uint32_t*>(&hv);
+          const float a = ex2_approx(s[8 * c + 2 * e] - mref);
+          const float bb = ex2_approx(s[8 * c + 2 * e + 1] - mref);
+          psum += a + bb;
+          w[e] = pack_bf16x2(a, bb);
         }
         const int region = c >> 3, cc = c & 7;
         uint8_t* dst = prow0 + region * ATT_REGION + ((cc ^ (row & 7)) << 4);
@@ -282,17 +304,17 @@ __global__ void __launch_bounds__(192, 1)
       l += psum;
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(t));
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (n_kv - 1) & 1, wc, 12))) {
+    if (ok && my_kv > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done(t), (my_kv - 1) & 1, wc, 12))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((size_t)b * p.L + t) * (size_t)(p.nh * hd) + (size_t)h * hd;
+      __nv_bfloat16* orow = p.out + ((size_t)b * p.L + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
       for (int c = 0; c < hd_pad; c += 32) {
         float v[32];
-        tmem_ld32(tmem + lane_off + 256 + c, v);
+        tmem_ld32(tO + c, v);
         tmem_ld_wait();
-        if (t < p.L) {
+        if (tok < p.L) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (c + 8 * q < hd) {
