@@ -436,10 +436,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOAD_RUNNERS),
+                    help="run one workload alone and print its own line (for profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload:
+        return run_single_workload(args)
 
     import torch
 
@@ -497,6 +501,50 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def _single_decode(L, torch, name, args):
+    r = bench_decode_layer(L, torch, synth.WORKLOADS[name], args.steps, args.warmup, 1, seed=11)
+    by = r["weight_bytes"] + r["kv_bytes"] + r["append_bytes"]
+    return {"metric": "decode tokens/s per layer", "unit": UNIT, "value": r["tokens_per_step"] / r["t_step_s"],
+            "ms_per_step": 1e3 * r["t_step_s"], "gbs": by / r["t_step_s"] / 1e9,
+            "kernels_us": {k: round(v["avg_us"], 2) for k, v in r["kernels"].items()}}
+
+
+def _single_prefill(L, torch, name, args):
+    w = synth.WORKLOADS[name]
+    r = bench_prefill_layer(L, torch, w, args.steps, args.warmup, 1, seed=7, with_e2e=False)
+    fl = r["gemm_flops"] + r["attn_flops"]
+    return {"metric": "prefill tokens/s per layer", "unit": UNIT, "value": r["tokens_per_step"] / r["t_step_s"],
+            "ms_per_step": 1e3 * r["t_step_s"], "tflops": fl / r["t_step_s"] / 1e12,
+            "kernels_us": {k: round(v["avg_us"], 2) for k, v in r["kernels"].items()}}
+
+
+def _single_model(L, torch, phase, args):
+    r = bench_model(L, torch, synth.WORKLOADS["phi3mini_model"], args.steps, args.warmup, 1, seed=21)[phase]
+    return {"metric": f"model {phase} tokens/s", "unit": "tokens/s", "value": r["tokens_per_step"] / r["t_step_s"],
+            "ms_per_step": 1e3 * r["t_step_s"]}
+
+
+WORKLOAD_RUNNERS = {
+    "llama7b_prefill": lambda L, t, a: _single_prefill(L, t, "llama7b_prefill", a),
+    "llama13b_decode": lambda L, t, a: _single_decode(L, t, "llama13b_decode", a),
+    "gqa70b_prefill": lambda L, t, a: _single_prefill(L, t, "gqa70b", a),
+    "gqa70b_decode": lambda L, t, a: _single_decode(L, t, "gqa70b", a),
+    "phi3_prefill": lambda L, t, a: _single_model(L, t, "prefill", a),
+    "phi3_decode": lambda L, t, a: _single_model(L, t, "decode", a),
+}
+
+
+def run_single_workload(args):
+    import torch
+
+    import llama_decoder_only_b200 as L
+    torch.cuda.set_device(0)
+    line = {"workload": args.workload, "steps": args.steps, "warmup": args.warmup}
+    line.update(WORKLOAD_RUNNERS[args.workload](L, torch, args))
+    print(json.dumps(line))
     return 0
 
 

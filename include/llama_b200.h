@@ -234,8 +234,12 @@ llama_status llama_model_forward(const llama_model* model, llama_kv_cache* const
  *   out      device bf16 [batch, n_heads*head_dim]
  * out[b, h] = softmax(q_bh k^T / sqrt(head_dim)) v over those keys, KV head
  * h / (n_heads/n_kv_heads).  dims->dtype must be LLAMA_BF16.
+ * It runs the same kernels and key-split choice as llama_layer_decode, with
+ * at least two key splits whenever the length allows.
  * Limit: batch * n_heads * (head_dim + 2) * 8 bytes <= 8 MiB (two key
  * splits), else LLAMA_ERR_SCRATCH_LIMIT; the call then enqueues nothing.
+ * With no workspace there is no device status word: a device-side wait that
+ * runs out is not reported by this entry point.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  All calls share the one array and nothing in it needs to start

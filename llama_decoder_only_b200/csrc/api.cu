@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "attention.cuh"
@@ -167,20 +168,58 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
   return r == CUDA_SUCCESS;
 }
 
+// Encoded 2-D maps are cached by (base, inner, rows, box rows): weights and
+// workspace buffers recur every call, and encoding is host work on the
+// launch path.  The cache is cleared when it grows past a bound.
+struct MapKey {
+  uintptr_t base;
+  uint64_t inner, rows;
+  uint32_t box_rows;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && inner == o.inner && rows == o.rows && box_rows == o.box_rows;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+    h ^= (k.inner + 0x632BE59BD9B4E019ull) * 0xC2B2AE3D27D4EB4Full + (h << 6) + (h >> 2);
+    h ^= (k.rows * 31 + k.box_rows) * 0x165667B19E3779F9ull + (h << 6) + (h >> 2);
+    return (size_t)h;
+  }
+};
+
 bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  const MapKey key{reinterpret_cast<uintptr_t>(base), inner, rows, box_rows};
+  {
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *m = it->second;
+      return true;
+    }
+  }
   const uint64_t dims[2] = {inner, rows};
   const uint64_t strides[1] = {inner * 2};
   const uint32_t box[2] = {64, box_rows};
-  return make_map(m, base, 2, dims, strides, box);
+  if (!make_map(m, base, 2, dims, strides, box)) return false;
+  std::lock_guard<std::mutex> g(mu);
+  if (cache.size() > 8192) cache.clear();
+  cache.emplace(key, *m);
+  return true;
 }
 
 int num_sms() {
+  static int cached[64] = {};
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return 148;
   }
+  if (dev >= 0 && dev < 64) cached[dev] = n;
   return n;
 }
 
@@ -504,15 +543,86 @@ void launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st) {
   attn_decode_kernel<HD, G><<<grid, 128, 0, st>>>(p);
 }
 
-llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int T,
-                              const __nv_bfloat16* qkv, __nv_bfloat16* out, float* part_ml, float* part_o) {
+template <int HD, int G>
+llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
+                                    dim3 grid, cudaStream_t st) {
+  using C = DecMmaCfg<HD>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(attn_decode_mma_kernel<HD, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM));
+    attr_set = true;
+  }
+  attn_decode_mma_kernel<HD, G><<<grid, 160, C::SMEM, st>>>(tk, tv, p);
+  return LLAMA_OK;
+}
+
+// Decode attention for GQA groups of 4 or 8 on the tensor cores.
+llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
+                             int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
+                             float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  CUtensorMap tk, tv;
+  const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)T, (uint64_t)B * d.n_kv_heads};
+  const uint64_t strides[2] = {(uint64_t)hd * 2, (uint64_t)capacity * hd * 2};
+  const uint32_t box[3] = {64, (uint32_t)DEC_CHUNK, 1};
+  if (!make_map(&tk, kc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  if (!make_map(&tv, vc, 3, dims, strides, box)) return LLAMA_ERR_CUDA;
+  AttnDecodeMmaParams p{};
+  p.qkv = qkv;
+  p.ld_qkv = ld_qkv;
+  p.T = T;
+  p.nh = d.n_heads;
+  p.nkv = d.n_kv_heads;
+  p.scale_log2 = kLog2e / sqrtf((float)hd);
+  p.part_ml = part_ml;
+  p.part_o = part_o;
+  p.out = out;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  const int base = B * d.n_kv_heads;
+  int splits = cdiv(2 * num_sms(), base);
+  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 256))));
+  splits = std::max(std::min(min_splits, cdiv(T, DEC_CHUNK)), std::min(splits, max_splits));
+  int kps = cdiv(cdiv(T, splits), DEC_CHUNK) * DEC_CHUNK;
+  splits = cdiv(T, kps);
+  p.splits = splits;
+  p.keys_per_split = kps;
+  dim3 grid(splits, d.n_kv_heads, B);
+  llama_status r = LLAMA_ERR_UNSUPPORTED;
+  {
+    TRACE(K_ATTN_DECODE, st);
+    if (hd == 128 && grp == 8) r = launch_attn_decode_mma<128, 8>(tk, tv, p, grid, st);
+    else if (hd == 128 && grp == 4) r = launch_attn_decode_mma<128, 4>(tk, tv, p, grid, st);
+    else if (hd == 64 && grp == 8) r = launch_attn_decode_mma<64, 8>(tk, tv, p, grid, st);
+    else if (hd == 64 && grp == 4) r = launch_attn_decode_mma<64, 4>(tk, tv, p, grid, st);
+  }
+  if (r != LLAMA_OK) return r;
+  LAUNCH_CHECK();
+  if (splits > 1) {
+    TRACE(K_ATTN_COMBINE, st);
+    attn_decode_combine_kernel<<<dim3(d.n_heads, B), 128, 0, st>>>(part_ml, part_o, out, d.n_heads, hd, splits);
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+// Decode attention of one new token per sequence over keys [0, T).  Splits of
+// the key range are chosen by a heuristic, clamped to [min_splits, max_splits].
+llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
+                              int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
+                              float* part_ml, float* part_o, DevStatus* status, int min_splits = 1,
+                              int max_splits = kMaxAttnSplits) {
+  const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  if (grp >= 4 && (hd == 64 || hd == 128))
+    return attn_decode_mma(st, d, kc, vc, capacity, B, T, qkv, ld_qkv, out, part_ml, part_o, status, min_splits,
+                           max_splits);
   AttnDecodeParams p{};
   p.qkv = qkv;
-  p.ld_qkv = (d.n_heads + 2 * d.n_kv_heads) * hd;
-  p.kc = reinterpret_cast<const __nv_bfloat16*>(kv->k);
-  p.vc = reinterpret_cast<const __nv_bfloat16*>(kv->v);
-  p.cap = kv->capacity;
+  p.ld_qkv = ld_qkv;
+  p.kc = reinterpret_cast<const __nv_bfloat16*>(kc);
+  p.vc = reinterpret_cast<const __nv_bfloat16*>(vc);
+  p.cap = capacity;
   p.T = T;
   p.nh = d.n_heads;
   p.nkv = d.n_kv_heads;
@@ -524,6 +634,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cac
   const int base = B * d.n_kv_heads;
   int splits = cdiv(4 * num_sms(), base);
   splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 128))));
+  splits = std::max(std::min(min_splits, cdiv(T, 32)), std::min(splits, max_splits));
   int kps = cdiv(T, splits);
   kps = cdiv(kps, 32) * 32;
   splits = cdiv(T, kps);
@@ -611,8 +722,9 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     LAUNCH_CHECK();
     // a5 / a6: attention
     if (decode) {
-      TRY(attn_decode_bf16(st, d, kv, B, p0 + 1, qkv, att, reinterpret_cast<float*>(ws + lay.att_ml),
-                           reinterpret_cast<float*>(ws + lay.att_o)));
+      TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
+                           reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o),
+                           status));
     } else {
       TRY(attn_prefill_bf16(st, d, kv, B, L, p0, qkv, att, status));
     }
@@ -1020,49 +1132,19 @@ extern "C" llama_status llama_attention_decode_noalloc(const llama_dims* dims, i
   if (length <= 0 || capacity < length || ld_q < d.n_heads * d.head_dim) return LLAMA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || (ld_q % 8) != 0)
     return LLAMA_ERR_ALIGNMENT;
-  const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  const int hd = d.head_dim;
   // partials of `splits` key ranges per (sequence, query head): (max, sum) and hd outputs
   const size_t per_split = (size_t)batch * d.n_heads * (hd + 2) * sizeof(float);
   const size_t max_splits = kNoAllocScratchBytes / per_split;
   if (max_splits < 2) return LLAMA_ERR_SCRATCH_LIMIT;
-  int splits = cdiv(4 * num_sms(), batch * d.n_kv_heads);
-  splits = std::max(2, std::min({splits, (int)std::min<size_t>(max_splits, kMaxAttnSplits), cdiv(length, 32)}));
-  int kps = cdiv(cdiv(length, splits), 32) * 32;
-  splits = cdiv(length, kps);
+  const int cap_splits = (int)std::min<size_t>(max_splits, kMaxAttnSplits);
   float* scratch = nullptr;
   TRY(noalloc_scratch(&scratch));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  AttnDecodeParams p{};
-  p.qkv = static_cast<const __nv_bfloat16*>(q);
-  p.ld_qkv = ld_q;
-  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
-  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
-  p.cap = capacity;
-  p.T = length;
-  p.nh = d.n_heads;
-  p.nkv = d.n_kv_heads;
-  p.scale_log2 = kLog2e / sqrtf((float)hd);
-  p.splits = splits;
-  p.keys_per_split = kps;
-  p.part_ml = scratch;
-  p.part_o = scratch + (size_t)batch * d.n_heads * splits * 2;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  dim3 grid(splits, d.n_kv_heads, batch);
-  {
-    TRACE(K_ATTN_DECODE, st);
-#define NOALLOC_CASE(HD_, G_) \
-  if (hd == HD_ && grp == G_) launch_attn_decode<HD_, G_>(p, grid, st);
-    NOALLOC_CASE(64, 1) NOALLOC_CASE(64, 2) NOALLOC_CASE(64, 4) NOALLOC_CASE(64, 8)
-    NOALLOC_CASE(96, 1) NOALLOC_CASE(96, 2) NOALLOC_CASE(96, 4) NOALLOC_CASE(96, 8)
-    NOALLOC_CASE(128, 1) NOALLOC_CASE(128, 2) NOALLOC_CASE(128, 4) NOALLOC_CASE(128, 8)
-#undef NOALLOC_CASE
-  }
-  LAUNCH_CHECK();
-  if (splits > 1) {
-    TRACE(K_ATTN_COMBINE, st);
-    attn_decode_combine_kernel<<<dim3(d.n_heads, batch), 128, 0, st>>>(p.part_ml, p.part_o, p.out, d.n_heads, hd,
-                                                                        splits);
-  }
-  LAUNCH_CHECK();
-  return LLAMA_OK;
+  float* part_ml = scratch;
+  float* part_o = scratch + (size_t)batch * d.n_heads * cap_splits * 2;
+  // the same kernels and split heuristic as llama_layer_decode, with at least two splits (the
+  // partials live in the fixed array); no workspace, so no device status word is written
+  return attn_decode_bf16(static_cast<cudaStream_t>(stream), d, k_cache, v_cache, capacity, batch, length,
+                          static_cast<const __nv_bfloat16*>(q), ld_q, static_cast<__nv_bfloat16*>(out), part_ml,
+                          part_o, nullptr, 2, cap_splits);
 }

@@ -526,6 +526,286 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
   }
 }
 
+// ---------------------------------------------------------------------- decode, GQA groups >= 4
+// The G query heads of a KV head are the rows of a 16-row MMA tile (rows
+// G..15 are zero), so S = Q K^T and O += P V run on the tensor cores
+// (mma.sync m16n8k16, bf16 -> fp32) and the kernel stays bound by the K/V
+// stream.  One producer warp stages 64-key chunks of K and V by TMA (128-byte
+// swizzle, 3-D maps over [head_dim, length, batch*n_kv]); four consumer warps
+// take chunks round robin, each with its own online-softmax state; the warps'
+// states are merged through shared memory at the end.
+
+constexpr int DEC_CHUNK = 64;                          // keys per chunk
+constexpr int DEC_STAGES = 4;
+constexpr int DEC_REGION = DEC_CHUNK * 128;            // [64 keys x 64 dims] bf16 = 8 KB
+
+template <int HD>
+struct DecMmaCfg {
+  static constexpr int NREG = HD / 64;                 // 64-dim regions per key row
+  static constexpr int STAGE = 2 * NREG * DEC_REGION;  // K then V
+  static constexpr int SMEM = 1024 + DEC_STAGES * STAGE + 256;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte offset of (key, 16-byte chunk) inside a swizzled [64 keys x 128 B] region
+__device__ __forceinline__ uint32_t sw128(int key, int chunk) {
+  return (uint32_t)(key * 128 + ((chunk ^ (key & 7)) << 4));
+}
+
+struct AttnDecodeMmaParams {
+  const __nv_bfloat16* qkv;
+  int ld_qkv;
+  int T;
+  int nh, nkv;
+  int splits, keys_per_split;
+  float scale_log2;
+  float* part_ml;
+  float* part_o;
+  __nv_bfloat16* out;
+  DevStatus* status;
+  unsigned long long limit_ns;
+};
+
+template <int HD, int G>
+__global__ void __launch_bounds__(160, 1)
+    attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const AttnDecodeMmaParams p) {
+  using C = DecMmaCfg<HD>;
+  constexpr int NW = 4;                // consumer warps
+  constexpr int KS = HD / 16;          // k-steps of S = Q K^T
+  constexpr int NT_O = HD / 8;         // 8-dim output tiles
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DEC_STAGES * C::STAGE);
+  __shared__ int abort_sh;
+  __shared__ float sm_m[NW][16], sm_l[NW][16];
+  __shared__ float sm_o[NW][G][HD];
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = split * p.keys_per_split;
+  const int j1 = min(p.T, j0 + p.keys_per_split);
+  const int n_chunks = j1 > j0 ? (j1 - j0 + DEC_CHUNK - 1) / DEC_CHUNK : 0;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (DEC_STAGES + s); };
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    for (int s = 0; s < DEC_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  WaitCtx wc{&abort_sh, p.status, p.limit_ns, 4};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int zkv = b * p.nkv + g;
+      int last_fill[DEC_STAGES];
+      for (int s = 0; s < DEC_STAGES; ++s) last_fill[s] = -1;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % DEC_STAGES;
+        if (!mbar_wait(empty_bar(s), ((c / DEC_STAGES) & 1) ^ 1u, wc, 1)) break;
+        uint8_t* st = smem + s * C::STAGE;
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE);
+        const int key0 = j0 + c * DEC_CHUNK;
+        for (int r = 0; r < C::NREG; ++r) {
+          tma_load_3d(smem_u32(st + r * DEC_REGION), &tmK, full_bar(s), r * 64, key0, zkv);
+          tma_load_3d(smem_u32(st + (C::NREG + r) * DEC_REGION), &tmV, full_bar(s), r * 64, key0, zkv);
+        }
+        last_fill[s] = c;
+      }
+      for (int s = 0; s < DEC_STAGES; ++s)
+        if (last_fill[s] >= 0) mbar_wait(full_bar(s), (last_fill[s] / DEC_STAGES) & 1, wc, 9, false);
+    }
+  } else {
+    const int cw = warp - 1;
+    const int r0 = lane >> 2, qd = lane & 3;   // fragment row (and row + 8), quad position
+    // Q as A fragments: rows = query heads of the group (rows >= G are zero)
+    uint32_t qa[KS][4];
+    {
+      const __nv_bfloat16* qrow0 = p.qkv + (size_t)b * p.ld_qkv + (size_t)(g * G) * HD;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int k0 = ks * 16 + qd * 2;
+        uint32_t lo = 0, hi = 0, lo8 = 0, hi8 = 0;
+        if (r0 < G) {
+          lo = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * HD + k0);
+          lo8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * HD + k0 + 8);
+        }
+        if (r0 + 8 < G) {
+          hi = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * HD + k0);
+          hi8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * HD + k0 + 8);
+        }
+        qa[ks][0] = lo;
+        qa[ks][1] = hi;
+        qa[ks][2] = lo8;
+        qa[ks][3] = hi8;
+      }
+    }
+    float o[NT_O][4];
+#pragma unroll
+    for (int i = 0; i < NT_O; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;   // rows r0, r0 + 8
+    bool ok = true;
+    for (int c = cw; c < n_chunks && ok; c += NW) {
+      const int s = c % DEC_STAGES;
+      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), (c / DEC_STAGES) & 1, wc, 2))) {
+        ok = false;
+        break;
+      }
+      const uint32_t sK = smem_u32(smem + s * C::STAGE);
+      const uint32_t sV = sK + C::NREG * DEC_REGION;
+      // S = Q K^T for 64 keys: 8 n-tiles of 8 keys
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        const int key = nt * 8 + (lane & 7);
+#pragma unroll
+        for (int kp = 0; kp < KS; kp += 2) {   // two k-steps (32 dims) per ldmatrix.x4
+          const int chunk = kp * 2 + (lane >> 3);          // 16-byte chunk within the 256-byte row
+          const uint32_t addr = sK + (chunk >> 3) * DEC_REGION + sw128(key, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(sc[nt], qa[kp], b0, b1);
+          mma_bf16_16816(sc[nt], qa[kp + 1], b2, b3);
+        }
+      }
+      // online softmax (log2 domain); keys outside [j0, j1) are masked
+      const int kbase = j0 + c * DEC_CHUNK;
+      float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool valid = kbase + nt * 8 + qd * 2 + e < j1;
+          sc[nt][e] = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
+          sc[nt][2 + e] = valid ? sc[nt][2 + e] * p.scale_log2 : -INFINITY;
+          mx_a = fmaxf(mx_a, sc[nt][e]);
+          mx_b = fmaxf(mx_b, sc[nt][2 + e]);
+        }
+      }
+      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+      const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+      const float al_a = mn_a == -INFINITY ? 1.f : ex2_approx(m_a - mn_a);
+      const float al_b = mn_b == -INFINITY ? 1.f : ex2_approx(m_b - mn_b);
+      m_a = mn_a;
+      m_b = mn_b;
+      const float ref_a = mn_a == -INFINITY ? 0.f : mn_a, ref_b = mn_b == -INFINITY ? 0.f : mn_b;
+      l_a *= al_a;
+      l_b *= al_b;
+#pragma unroll
+      for (int i = 0; i < NT_O; ++i) {
+        o[i][0] *= al_a;
+        o[i][1] *= al_a;
+        o[i][2] *= al_b;
+        o[i][3] *= al_b;
+      }
+      uint32_t pa[4][4];   // P as A fragments: 4 k-steps of 16 keys
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float p0 = ex2_approx(sc[nt][0] - ref_a), p1 = ex2_approx(sc[nt][1] - ref_a);
+        const float p2 = ex2_approx(sc[nt][2] - ref_b), p3 = ex2_approx(sc[nt][3] - ref_b);
+        l_a += p0 + p1;
+        l_b += p2 + p3;
+        pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+      }
+      // O += P V: V rows are keys; ldmatrix.trans gives the k-major B fragments
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int dt = 0; dt < NT_O; dt += 2) {
+          const int chunk = dt + (lane >> 4);              // 8-dim chunk index within the row
+          const uint32_t addr = sV + (chunk >> 3) * DEC_REGION + sw128(key, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(addr, b0, b1, b2, b3);
+          mma_bf16_16816(o[dt], pa[kk], b0, b1);
+          mma_bf16_16816(o[dt + 1], pa[kk], b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+    }
+    // quad-reduce the sums, then publish this warp's state
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    if (qd == 0) {
+      sm_m[cw][r0] = m_a;
+      sm_l[cw][r0] = l_a;
+      sm_m[cw][r0 + 8] = m_b;
+      sm_l[cw][r0 + 8] = l_b;
+    }
+#pragma unroll
+    for (int dt = 0; dt < NT_O; ++dt) {
+      const int col = dt * 8 + qd * 2;
+      if (r0 < G) {
+        sm_o[cw][r0][col] = o[dt][0];
+        sm_o[cw][r0][col + 1] = o[dt][1];
+      }
+      if (r0 + 8 < G) {
+        sm_o[cw][r0 + 8][col] = o[dt][2];
+        sm_o[cw][r0 + 8][col + 1] = o[dt][3];
+      }
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
+    const int gi = idx / HD, d = idx % HD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][gi]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float cf = exp2f(sm_m[w][gi] - M);
+        Lsum += sm_l[w][gi] * cf;
+        O += sm_o[w][gi][d] * cf;
+      }
+    }
+    const int hq = g * G + gi;
+    if (p.splits == 1) {
+      p.out[(size_t)b * p.nh * HD + (size_t)hq * HD + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+    } else {
+      const size_t r = ((size_t)b * p.nh + hq) * p.splits + split;
+      p.part_o[r * HD + d] = O;
+      if (d == 0) {
+        p.part_ml[2 * r] = M;
+        p.part_ml[2 * r + 1] = Lsum;
+      }
+    }
+  }
+}
+
 // out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
                                            __nv_bfloat16* __restrict__ out, int nh, int hd, int splits) {
