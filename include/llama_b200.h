@@ -75,7 +75,7 @@ typedef enum llama_dtype { LLAMA_F32 = 0, LLAMA_BF16 = 1 } llama_dtype;
  * Supported: head_dim in {64, 96, 128} (and 32 for LLAMA_F32);
  * n_heads % n_kv_heads == 0 (GQA group n_heads/n_kv_heads, query head h
  * reads KV head h / group, [DeepDive] LLaMAAttention); dim, ffn_dim and
- * n_heads*head_dim multiples of 8; eps > 0; rope_theta > 1. */
+ * n_heads*head_dim multiples of 8; dim <= 16384; eps > 0; rope_theta > 1. */
 typedef struct llama_dims {
   int32_t dim;
   int32_t n_heads;

@@ -235,6 +235,7 @@ llama_status check_dims(const llama_dims* d) {
   if (d->rope_style != LLAMA_ROPE_HALF && d->rope_style != LLAMA_ROPE_INTERLEAVED) return LLAMA_ERR_INVALID_ARG;
   if (d->dtype != LLAMA_F32 && d->dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
   if (d->dim % 8 || d->ffn_dim % 8) return LLAMA_ERR_UNSUPPORTED;
+  if (d->dim > 16 * 1024) return LLAMA_ERR_UNSUPPORTED;   // RMSNorm keeps a row in one CTA's registers
   const int hd = d->head_dim;
   if (d->dtype == LLAMA_BF16) {
     if (hd != 64 && hd != 96 && hd != 128) return LLAMA_ERR_UNSUPPORTED;
@@ -696,7 +697,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // a2: RMSNorm-1 -> h (bf16)
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<bf><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
     }
     LAUNCH_CHECK();
     // a3: QKV projection
@@ -735,7 +736,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // a8: RMSNorm-2 + gate_up + SiLU·mul
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<bf><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<bf><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
     }
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
@@ -756,7 +757,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     auto grid_for = [](int M_, int N_) { return dim3(cdiv(N_, 64), cdiv(M_, 64)); };
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
     }
     {
       TRACE(K_GEMM_F32, st);
@@ -801,7 +802,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     LAUNCH_CHECK();
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<cdiv(M, rows_per_block), 256, 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
     }
     {
       TRACE(K_GEMM_F32, st);
@@ -1041,7 +1042,7 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<__nv_bfloat16><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
+      rmsnorm_kernel<__nv_bfloat16><<<batch, rmsnorm_threads(d.dim), 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
                                                                      d.eps);
     }
     LAUNCH_CHECK();
@@ -1052,7 +1053,7 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     float* hl = reinterpret_cast<float*>(ws + lay.hl);
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<cdiv(batch, 8), 256, 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
+      rmsnorm_kernel<float><<<batch, rmsnorm_threads(d.dim), 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
     }
     {
       TRACE(K_GEMM_LM_HEAD, st);

@@ -20,32 +20,56 @@ __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // ------------------------------------------------------------------ RMSNorm (K1)
-// h[m, :] = g * (x[m, :] * rsqrt(mean(x[m, :]^2) + eps)), one warp per row,
-// 16-byte loads, warp-shuffle reduction ([MLX-13B] 4. RMSNorm; [DeepDive]
-// LLaMARMSNorm).  `x_row_stride` lets the final norm read the last row of
-// each sequence only.  dim % 4 == 0.
+// h[m, :] = g * (x[m, :] * rsqrt(mean(x[m, :]^2) + eps)) ([MLX-13B] 4. RMSNorm;
+// [DeepDive] LLaMARMSNorm).  One CTA per row; each thread keeps up to four
+// 16-byte chunks of the row in registers, so the row is read from memory
+// once; warp-shuffle then shared-memory reduction of the sum of squares.
+// `x_row_stride` lets the final norm read the last row of each sequence
+// only.  dim % 4 == 0, dim <= 16 * blockDim.x.
+constexpr int RMS_MAX_V4 = 4;
+
+inline int rmsnorm_threads(int dim) {
+  int t = ((dim / 4 + RMS_MAX_V4 - 1) / RMS_MAX_V4 + 31) / 32 * 32;
+  return t < 32 ? 32 : (t > 1024 ? 1024 : t);
+}
+
 template <typename OutT>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, long long x_row_stride,
-                                                      const float* __restrict__ g, OutT* __restrict__ h, int rows,
-                                                      int dim, float eps) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)warp * x_row_stride);
+__global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__ x, long long x_row_stride,
+                                                       const float* __restrict__ g, OutT* __restrict__ h, int rows,
+                                                       int dim, float eps) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * x_row_stride);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
   const int n4 = dim >> 2;
+  float4 v[RMS_MAX_V4];
   float ss = 0.f;
-  for (int i = lane; i < n4; i += 32) {
-    float4 v = __ldg(xr + i);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+  for (int k = 0; k < RMS_MAX_V4; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    v[k] = i < n4 ? __ldg(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
   }
   ss = warp_sum(ss);
-  const float rstd = rsqrtf(ss / (float)dim + eps);
-  OutT* hr = h + (size_t)warp * dim;
-  const float4* g4 = reinterpret_cast<const float4*>(g);
-  for (int i = lane; i < n4; i += 32) {
-    float4 v = __ldg(xr + i);
-    float4 w = __ldg(g4 + i);
-    float a = w.x * (v.x * rstd), b = w.y * (v.y * rstd), c = w.z * (v.z * rstd), d = w.w * (v.w * rstd);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (warp == 0) {
+    float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_sum(t);
+    if (lane == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float rstd = rsqrtf(red[0] / (float)dim + eps);
+  OutT* hr = h + (size_t)row * dim;
+#pragma unroll
+  for (int k = 0; k < RMS_MAX_V4; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    if (i >= n4) break;
+    const float4 w = __ldg(g4 + i);
+    const float a = w.x * (v[k].x * rstd), b = w.y * (v[k].y * rstd), c = w.z * (v[k].z * rstd),
+                d = w.w * (v[k].w * rstd);
     if constexpr (sizeof(OutT) == 2) {
       uint2 o;
       o.x = pack_bf16x2(a, b);
@@ -58,19 +82,22 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 }
 
 // ------------------------------------------------------------------ RoPE + KV append (K3)
-// One CTA per token.  The token's cos/sin ladder is computed once in fp64
-// (angle p * theta^(-2i/hd), [DeepDive] LLaMARoPE) into shared memory, then
-// every (head, pair) of q and k is rotated; q is rotated in place in the
+// One CTA per token.  The token's cos/sin ladder is computed once into shared
+// memory: the angle p * theta^(-2i/hd) ([DeepDive] LLaMARoPE) is formed and
+// reduced modulo 2*pi in fp64, then sincosf evaluates the reduced angle.
+// Every (head, pair) of q and k is rotated; q is rotated in place in the
 // projection buffer, rotated k and plain v are written to the cache at
 // position p0 + t ([MLX-13B] KV 缓存实现片段: concatenate after the cached
 // entries, RoPE offset = cache length).
 //   qkv   [M, (nh + 2 nkv) hd] row-major (q | k | v), M = batch * L
 //   cache [batch][nkv][cap][hd]
 // style 0: rotate-half pairs (i, i + hd/2); style 1: adjacent pairs (2i, 2i+1).
+// Each thread moves 16 bytes at a time (8 bf16 or 4 fp32 elements).
 template <typename T>
 __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T* __restrict__ kc,
                                                           T* __restrict__ vc, int L, int p0, int nh, int nkv,
                                                           int hd, int cap, float theta, int style) {
+  constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
   __shared__ float cs[64], sn[64];
   const int m = blockIdx.x;
   const int b = m / L;
@@ -79,42 +106,68 @@ __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T
   const int half = hd >> 1;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     const double inv = pow((double)theta, -2.0 * (double)i / (double)hd);
-    double s, c;
-    sincos((double)p * inv, &s, &c);
-    cs[i] = (float)c;
-    sn[i] = (float)s;
+    const double two_pi = 6.283185307179586476925286766559;
+    double a = (double)p * inv;
+    a -= two_pi * floor(a / two_pi);
+    float s, c;
+    sincosf((float)a, &s, &c);
+    cs[i] = c;
+    sn[i] = s;
   }
   __syncthreads();
   const int qkvn = (nh + 2 * nkv) * hd;
   T* row = qkv + (size_t)m * qkvn;
-  // rotate q (heads 0..nh-1) and k (heads nh..nh+nkv-1)
-  const int nrot = (nh + nkv) * half;
-  for (int e = threadIdx.x; e < nrot; e += blockDim.x) {
-    const int head = e / half;
-    const int i = e % half;
-    const int i0 = style == 0 ? i : 2 * i;
-    const int i1 = style == 0 ? i + half : 2 * i + 1;
-    T* hv = row + head * hd;
-    const float x0 = to_f32(hv[i0]), x1 = to_f32(hv[i1]);
-    const float c = cs[i], s = sn[i];
-    const float y0 = x0 * c - x1 * s;
-    const float y1 = x1 * c + x0 * s;
-    if (head < nh) {
-      hv[i0] = from_f32<T>(y0);
-      hv[i1] = from_f32<T>(y1);
-    } else {
-      const int g = head - nh;
-      T* dst = kc + (((size_t)b * nkv + g) * cap + p) * hd;
-      dst[i0] = from_f32<T>(y0);
-      dst[i1] = from_f32<T>(y1);
+  const int heads = nh + nkv;
+  if (style == 0) {
+    // rotate-half: a vector of VE elements at i (first half) pairs with the one at i + half
+    const int vph = half / VE;                        // vectors per half head
+    for (int e = threadIdx.x; e < heads * vph; e += blockDim.x) {
+      const int head = e / vph, i0 = (e % vph) * VE;
+      T* hv = row + head * hd;
+      uint4 ua = *reinterpret_cast<const uint4*>(hv + i0);
+      uint4 ub = *reinterpret_cast<const uint4*>(hv + i0 + half);
+      T* xa = reinterpret_cast<T*>(&ua);
+      T* xb = reinterpret_cast<T*>(&ub);
+#pragma unroll
+      for (int k = 0; k < VE; ++k) {
+        const float x0 = to_f32(xa[k]), x1 = to_f32(xb[k]);
+        const float c = cs[i0 + k], s = sn[i0 + k];
+        xa[k] = from_f32<T>(x0 * c - x1 * s);
+        xb[k] = from_f32<T>(x1 * c + x0 * s);
+      }
+      T* dst = hv;
+      if (head >= nh) dst = kc + (((size_t)b * nkv + (head - nh)) * cap + p) * hd;
+      *reinterpret_cast<uint4*>(dst + i0) = ua;
+      *reinterpret_cast<uint4*>(dst + i0 + half) = ub;
+    }
+  } else {
+    // interleaved: a vector holds VE/2 adjacent pairs
+    const int vpr = hd / VE;                          // vectors per head row
+    for (int e = threadIdx.x; e < heads * vpr; e += blockDim.x) {
+      const int head = e / vpr, i0 = (e % vpr) * VE;
+      T* hv = row + head * hd;
+      uint4 u = *reinterpret_cast<const uint4*>(hv + i0);
+      T* x = reinterpret_cast<T*>(&u);
+#pragma unroll
+      for (int k = 0; k < VE; k += 2) {
+        const float x0 = to_f32(x[k]), x1 = to_f32(x[k + 1]);
+        const int pi = (i0 + k) >> 1;
+        const float c = cs[pi], s = sn[pi];
+        x[k] = from_f32<T>(x0 * c - x1 * s);
+        x[k + 1] = from_f32<T>(x1 * c + x0 * s);
+      }
+      T* dst = hv;
+      if (head >= nh) dst = kc + (((size_t)b * nkv + (head - nh)) * cap + p) * hd;
+      *reinterpret_cast<uint4*>(dst + i0) = u;
     }
   }
   // copy v
-  const int nv = nkv * hd;
+  const int vpr = hd / VE;
   const T* vsrc = row + (nh + nkv) * hd;
-  for (int e = threadIdx.x; e < nv; e += blockDim.x) {
-    const int g = e / hd, d = e % hd;
-    vc[(((size_t)b * nkv + g) * cap + p) * hd + d] = vsrc[e];
+  for (int e = threadIdx.x; e < nkv * vpr; e += blockDim.x) {
+    const int gkv = e / vpr, i0 = (e % vpr) * VE;
+    *reinterpret_cast<uint4*>(vc + (((size_t)b * nkv + gkv) * cap + p) * hd + i0) =
+        *reinterpret_cast<const uint4*>(vsrc + gkv * hd + i0);
   }
 }
 
