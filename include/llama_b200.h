@@ -136,8 +136,9 @@ void llama_kv_cache_destroy(llama_kv_cache* cache);
 
 /* Bytes of device workspace a layer call with `batch` sequences of up to
  * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
- * The workspace is caller-owned scratch; its first 256 bytes hold the
- * device status word and must be zeroed once before first use. */
+ * The workspace is caller-owned scratch.  Zero-fill it once before its first
+ * use (its first 256 bytes hold the device status word, and the GEMMs keep
+ * per-launch flags in it); after that the library keeps it consistent. */
 size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_len);
 
 /* Byte offsets, inside the workspace of a layer call with (batch, seq_len),

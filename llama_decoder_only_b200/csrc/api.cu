@@ -6,11 +6,13 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <unordered_map>
 #include <vector>
 
@@ -223,6 +225,33 @@ int num_sms() {
   return n;
 }
 
+// Launch with programmatic stream serialization (the kernels call pdl_trigger /
+// pdl_wait), so a kernel's prologue overlaps the tail of the one before it.
+// LLAMA_NO_PDL=1 launches them in plain stream order instead.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_NO_PDL");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------------ validation
 
 llama_status check_dims(const llama_dims* d) {
@@ -268,6 +297,7 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 struct WsLayout {
   size_t qkv, h, attn, mbuf, partial, att_ml, att_o;        // layer scratch
+  size_t sk_part, sk_flags;                                 // tile-mode stream-K partials / flags
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
@@ -306,6 +336,10 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   w.partial = take(pf * 4);
   w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
   w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
+  if (d.dtype == LLAMA_BF16) {
+    w.sk_part = take((size_t)kMaxSkGrid * 128 * 256 * 4);
+    w.sk_flags = take((size_t)kMaxSkGrid * 4);
+  }
   if (vocab > 0) {
     w.xa = take(M * (size_t)d.dim * 4);
     w.xb = take(M * (size_t)d.dim * 4);
@@ -337,15 +371,22 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
   }
   {
     TRACE(kind, st);
-    gemm_tc_kernel<BN, SWAP, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(a, w[0], w[1], w[2], p);
+    CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, 192, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
 
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
+struct SkBuffers {
+  float* partial;
+  unsigned* flags;
+};
+std::atomic<unsigned> g_sk_epoch{0};
+
 llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
-                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind) {
+                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind,
+                          SkBuffers sk) {
   constexpr int BN = 256;
   GemmParams p{};
   p.K = K;
@@ -388,7 +429,22 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
     p.n_tiles = t;
   }
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = std::min(tiles, num_sms());
+  int grid = std::min(tiles, num_sms());
+  // Stream-K when the last wave of whole tiles would leave more than 10% of
+  // the SMs idle; every CTA then gets the same number of (tile, k-block) units.
+  const int G = std::min(num_sms(), kMaxSkGrid);
+  const double waves = (double)tiles / G;
+  const double dp_eff = waves / std::ceil(waves);
+  if (sk.partial != nullptr && tiles >= G && dp_eff < 0.9) {
+    grid = G;
+    p.sk_tiles = 1;
+    p.units = (long long)tiles * p.num_kb;
+    p.sk_partial = sk.partial;
+    p.sk_flags = sk.flags;
+    unsigned e = g_sk_epoch.fetch_add(1) + 1;
+    if (e == 0) e = g_sk_epoch.fetch_add(1) + 1;
+    p.sk_epoch = e;
+  }
   switch (epi) {
     case EPI_BF16:
       return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st, kind);
@@ -471,10 +527,10 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   dim3 grid_r(cdiv(n_out, 256), M);
   TRACE(K_SPLITK_REDUCE, st);
   switch (dec_epi) {
-    case DEC_BF16: splitk_reduce_kernel<DEC_BF16><<<grid_r, 256, 0, st>>>(r); break;
-    case DEC_RESID_F32: splitk_reduce_kernel<DEC_RESID_F32><<<grid_r, 256, 0, st>>>(r); break;
-    case DEC_SWIGLU_BF16: splitk_reduce_kernel<DEC_SWIGLU_BF16><<<grid_r, 256, 0, st>>>(r); break;
-    default: splitk_reduce_kernel<DEC_F32><<<grid_r, 256, 0, st>>>(r); break;
+    case DEC_BF16: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_BF16>, grid_r, 256, 0, st, r)); break;
+    case DEC_RESID_F32: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_RESID_F32>, grid_r, 256, 0, st, r)); break;
+    case DEC_SWIGLU_BF16: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_SWIGLU_BF16>, grid_r, 256, 0, st, r)); break;
+    default: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_F32>, grid_r, 256, 0, st, r)); break;
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -483,7 +539,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
                        int epi, void* out, int ldo, const float* resid, int ldr, float* partial,
-                       DevStatus* status, int kind) {
+                       DevStatus* status, int kind, SkBuffers sk = SkBuffers{nullptr, nullptr}) {
   if (decode && M <= kSwapMaxTokens) {
     const int dec = epi == EPI_BF16 ? DEC_BF16 : epi == EPI_RESID_F32 ? DEC_RESID_F32
                   : epi == EPI_SWIGLU_BF16 ? DEC_SWIGLU_BF16 : DEC_F32;
@@ -492,7 +548,7 @@ llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int
     if (epi == EPI_SWIGLU_BF16) s2[1].col0 = segs[0].rows;  // up rows follow the gate rows
     return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status, kind);
   }
-  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
+  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind, sk);
 }
 
 // ------------------------------------------------------------------ attention launchers
@@ -534,14 +590,14 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.limit_ns = g_wait_limit_ns.load();
   dim3 grid(p.n_qblocks, d.n_heads, B);
   TRACE(K_ATTN_PREFILL, st);
-  attn_prefill_kernel<<<grid, ATT_THREADS, ATT_SMEM, st>>>(tq, tk, tv, p);
+  CUDA_TRY(launch_k(attn_prefill_kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
 
 template <int HD, int G>
-void launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st) {
-  attn_decode_kernel<HD, G><<<grid, 128, 0, st>>>(p);
+cudaError_t launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st) {
+  return launch_k(attn_decode_kernel<HD, G>, grid, 128, 0, st, p);
 }
 
 template <int HD, int G>
@@ -554,7 +610,7 @@ llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv
                                   C::SMEM));
     attr_set = true;
   }
-  attn_decode_mma_kernel<HD, G><<<grid, 160, C::SMEM, st>>>(tk, tv, p);
+  CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G>, grid, 160, C::SMEM, st, tk, tv, p));
   return LLAMA_OK;
 }
 
@@ -602,7 +658,7 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   LAUNCH_CHECK();
   if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
-    attn_decode_combine_kernel<<<dim3(d.n_heads, B), 128, 0, st>>>(part_ml, part_o, out, d.n_heads, hd, splits);
+    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -645,7 +701,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   {
   TRACE(K_ATTN_DECODE, st);
 #define DEC_CASE(HD_, G_) \
-  if (hd == HD_ && grp == G_) launch_attn_decode<HD_, G_>(p, grid, st);
+  if (hd == HD_ && grp == G_) CUDA_TRY((launch_attn_decode<HD_, G_>(p, grid, st)));
   DEC_CASE(64, 1) DEC_CASE(64, 2) DEC_CASE(64, 4) DEC_CASE(64, 8)
   DEC_CASE(96, 1) DEC_CASE(96, 2) DEC_CASE(96, 4) DEC_CASE(96, 8)
   DEC_CASE(128, 1) DEC_CASE(128, 2) DEC_CASE(128, 4) DEC_CASE(128, 8)
@@ -654,7 +710,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   LAUNCH_CHECK();
   if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
-    attn_decode_combine_kernel<<<dim3(d.n_heads, B), 128, 0, st>>>(part_ml, part_o, out, d.n_heads, hd, splits);
+    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
     LAUNCH_CHECK();
   }
   return LLAMA_OK;
@@ -694,10 +750,11 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     bf* att = reinterpret_cast<bf*>(ws + lay.attn);
     bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
     float* part = reinterpret_cast<float*>(ws + lay.partial);
+    const SkBuffers sk{reinterpret_cast<float*>(ws + lay.sk_part), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
     // a2: RMSNorm-1 -> h (bf16)
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<bf><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps));
     }
     LAUNCH_CHECK();
     // a3: QKV projection
@@ -713,12 +770,13 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
-    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
+    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV,
+                  sk));
     // a4: RoPE + KV append
     {
       TRACE(K_ROPE_APPEND, st);
-      rope_append_kernel<bf><<<M, 256, 0, st>>>(qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
-                                                 p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+      CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
+                                                 p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style));
     }
     LAUNCH_CHECK();
     // a5 / a6: attention
@@ -732,20 +790,20 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // a7: o_proj + residual -> x_out holds x_mid
     WSeg so{w.wo, d.dim, 0};
     TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status,
-                  K_GEMM_O));
+                  K_GEMM_O, sk));
     // a8: RMSNorm-2 + gate_up + SiLU·mul
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<bf><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps));
     }
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
     TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
-                  K_GEMM_GATE_UP));
+                  K_GEMM_GATE_UP, sk));
     // a9: down + residual (in place on x_out)
     WSeg sd{w.w2, d.dim, 0};
     TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
-                  K_GEMM_DOWN));
+                  K_GEMM_DOWN, sk));
   } else {
     float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
     float* h = reinterpret_cast<float*>(ws + lay.h);
@@ -1014,8 +1072,8 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
   {
   TRACE(K_EMBED, st);
   if (d.dtype == LLAMA_BF16)
-    embed_kernel<__nv_bfloat16><<<cdiv(M, 8), 256, 0, st>>>(
-        tokens, static_cast<const __nv_bfloat16*>(m->embed), xa, M, d.dim, m->vocab, status);
+    CUDA_TRY(launch_k(embed_kernel<__nv_bfloat16>, cdiv(M, 8), 256, 0, st, 
+        tokens, static_cast<const __nv_bfloat16*>(m->embed), xa, M, d.dim, m->vocab, status));
   else
     embed_kernel<float><<<cdiv(M, 8), 256, 0, st>>>(tokens, static_cast<const float*>(m->embed), xa, M, d.dim,
                                                     m->vocab, status);
@@ -1032,7 +1090,7 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     float* g = reinterpret_cast<float*>(ws + lay.xl);
     {
       TRACE(K_GATHER_LAST, st);
-      gather_last_rows_kernel<<<dim3(cdiv(d.dim, 256), batch), 256, 0, st>>>(xa, g, seq_len, d.dim);
+      CUDA_TRY(launch_k(gather_last_rows_kernel, dim3(cdiv(d.dim, 256), batch), 256, 0, st, xa, g, seq_len, d.dim));
     }
     LAUNCH_CHECK();
     xl = g;
@@ -1042,8 +1100,8 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<__nv_bfloat16><<<batch, rmsnorm_threads(d.dim), 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
-                                                                     d.eps);
+      CUDA_TRY(launch_k(rmsnorm_kernel<__nv_bfloat16>, batch, rmsnorm_threads(d.dim), 0, st, xl, d.dim, m->final_norm, hl, batch, d.dim,
+                                                                     d.eps));
     }
     LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};
@@ -1065,7 +1123,7 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
   }
   {
     TRACE(K_ARGMAX, st);
-    argmax_kernel<<<batch, 1024, 0, st>>>(logits, m->vocab, next_ids);
+    CUDA_TRY(launch_k(argmax_kernel, batch, 1024, 0, st, logits, m->vocab, next_ids));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;

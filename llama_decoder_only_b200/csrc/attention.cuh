@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = tmem_base_sh;   // S_t at col 128 t, O_t at col 256 + 128 t
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, 3};
 
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
   }
 
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -361,6 +363,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
   constexpr int KPW = 32 / LPK;                 // keys per warp step
   constexpr int NK = 4;                         // keys per lane group per step
   constexpr int NW = 4;
+  pdl_wait();
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPK, sub = lane % LPK;
@@ -615,6 +618,7 @@ __global__ void __launch_bounds__(160, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, 4};
 
   if (warp == 0) {
@@ -778,6 +782,7 @@ __global__ void __launch_bounds__(160, 1)
     }
   }
   __syncthreads();
+  pdl_trigger();
   for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
     const int gi = idx / HD, d = idx % HD;
     float M = -INFINITY;
@@ -809,6 +814,7 @@ __global__ void __launch_bounds__(160, 1)
 // out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
                                            __nv_bfloat16* __restrict__ out, int nh, int hd, int splits) {
+  pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y;
   const size_t r0 = ((size_t)b * nh + h) * splits;
   float M = -INFINITY;

@@ -267,6 +267,16 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels are launched so that the next kernel in the stream may start once
+// every CTA of this one has called pdl_trigger (done at entry).  pdl_wait
+// blocks until the previous kernel has completed and its writes are visible;
+// every kernel calls it before its first global-memory access, so each kernel
+// completes only after its predecessor (completion stays in stream order).
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ misc
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

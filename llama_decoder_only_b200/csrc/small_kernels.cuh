@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__
                                                        const float* __restrict__ g, OutT* __restrict__ h, int rows,
                                                        int dim, float eps) {
   __shared__ float red[32];
+  pdl_wait();
   const int row = blockIdx.x;
   if (row >= rows) return;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * x_row_stride);
@@ -115,6 +116,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T
     sn[i] = s;
   }
   __syncthreads();
+  pdl_wait();
   const int qkvn = (nh + 2 * nkv) * hd;
   T* row = qkv + (size_t)m * qkvn;
   const int heads = nh + nkv;
@@ -179,6 +181,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) embed_kernel(const int32_t* __restrict__ tok, const T* __restrict__ E,
                                                     float* __restrict__ x, int M, int dim, int vocab,
                                                     DevStatus* st) {
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= M) return;
@@ -214,6 +217,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const int32_t* __restrict__ 
 // One CTA per row; NaN never wins.
 __global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ logits, int vocab,
                                                       int32_t* __restrict__ ids) {
+  pdl_wait();
   const int b = blockIdx.x;
   const float* r = logits + (size_t)b * vocab;
   float best = -INFINITY;
@@ -261,6 +265,7 @@ __global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ 
 
 // Gather the last row of each of `batch` sequences of length L: dst[b] = src[b*L + L-1].
 __global__ void gather_last_rows_kernel(const float* __restrict__ src, float* __restrict__ dst, int L, int dim) {
+  pdl_wait();
   const int b = blockIdx.y;
   const float* s = src + ((size_t)b * L + (L - 1)) * dim;
   float* d = dst + (size_t)b * dim;
