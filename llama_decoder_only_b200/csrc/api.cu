@@ -297,7 +297,6 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 struct WsLayout {
   size_t qkv, h, attn, mbuf, partial, att_ml, att_o;        // layer scratch
-  size_t sk_part, sk_flags;                                 // tile-mode stream-K partials / flags
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
@@ -336,10 +335,6 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   w.partial = take(pf * 4);
   w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
   w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
-  if (d.dtype == LLAMA_BF16) {
-    w.sk_part = take((size_t)kMaxSkGrid * 128 * 256 * 4);
-    w.sk_flags = take((size_t)kMaxSkGrid * 4);
-  }
   if (vocab > 0) {
     w.xa = take(M * (size_t)d.dim * 4);
     w.xb = take(M * (size_t)d.dim * 4);
@@ -378,15 +373,8 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
 }
 
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
-struct SkBuffers {
-  float* partial;
-  unsigned* flags;
-};
-std::atomic<unsigned> g_sk_epoch{0};
-
 llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
-                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind,
-                          SkBuffers sk) {
+                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind) {
   constexpr int BN = 256;
   GemmParams p{};
   p.K = K;
@@ -429,22 +417,7 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
     p.n_tiles = t;
   }
   const int tiles = p.m_tiles * p.n_tiles;
-  int grid = std::min(tiles, num_sms());
-  // Stream-K when the last wave of whole tiles would leave more than 10% of
-  // the SMs idle; every CTA then gets the same number of (tile, k-block) units.
-  const int G = std::min(num_sms(), kMaxSkGrid);
-  const double waves = (double)tiles / G;
-  const double dp_eff = waves / std::ceil(waves);
-  if (sk.partial != nullptr && tiles >= G && dp_eff < 0.9) {
-    grid = G;
-    p.sk_tiles = 1;
-    p.units = (long long)tiles * p.num_kb;
-    p.sk_partial = sk.partial;
-    p.sk_flags = sk.flags;
-    unsigned e = g_sk_epoch.fetch_add(1) + 1;
-    if (e == 0) e = g_sk_epoch.fetch_add(1) + 1;
-    p.sk_epoch = e;
-  }
+  const int grid = std::min(tiles, num_sms());
   switch (epi) {
     case EPI_BF16:
       return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st, kind);
@@ -539,7 +512,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
                        int epi, void* out, int ldo, const float* resid, int ldr, float* partial,
-                       DevStatus* status, int kind, SkBuffers sk = SkBuffers{nullptr, nullptr}) {
+                       DevStatus* status, int kind) {
   if (decode && M <= kSwapMaxTokens) {
     const int dec = epi == EPI_BF16 ? DEC_BF16 : epi == EPI_RESID_F32 ? DEC_RESID_F32
                   : epi == EPI_SWIGLU_BF16 ? DEC_SWIGLU_BF16 : DEC_F32;
@@ -548,7 +521,7 @@ llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int
     if (epi == EPI_SWIGLU_BF16) s2[1].col0 = segs[0].rows;  // up rows follow the gate rows
     return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status, kind);
   }
-  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind, sk);
+  return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
 }
 
 // ------------------------------------------------------------------ attention launchers
@@ -750,7 +723,6 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     bf* att = reinterpret_cast<bf*>(ws + lay.attn);
     bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
     float* part = reinterpret_cast<float*>(ws + lay.partial);
-    const SkBuffers sk{reinterpret_cast<float*>(ws + lay.sk_part), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
     // a2: RMSNorm-1 -> h (bf16)
     {
       TRACE(K_RMSNORM, st);
@@ -770,8 +742,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
-    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV,
-                  sk));
+    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
     // a4: RoPE + KV append
     {
       TRACE(K_ROPE_APPEND, st);
@@ -790,7 +761,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // a7: o_proj + residual -> x_out holds x_mid
     WSeg so{w.wo, d.dim, 0};
     TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status,
-                  K_GEMM_O, sk));
+                  K_GEMM_O));
     // a8: RMSNorm-2 + gate_up + SiLU·mul
     {
       TRACE(K_RMSNORM, st);
@@ -799,11 +770,11 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
     TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
-                  K_GEMM_GATE_UP, sk));
+                  K_GEMM_GATE_UP));
     // a9: down + residual (in place on x_out)
     WSeg sd{w.w2, d.dim, 0};
     TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
-                  K_GEMM_DOWN, sk));
+                  K_GEMM_DOWN));
   } else {
     float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
     float* h = reinterpret_cast<float*>(ws + lay.h);

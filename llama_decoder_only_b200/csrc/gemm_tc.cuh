@@ -53,15 +53,8 @@ struct GemmParams {
   int ldr;
   // stream-K mode
   float* partial;
-  long long units;     // (swap) n_tiles * num_kb; (tile stream-K) m_tiles * n_tiles * num_kb
+  long long units;     // n_tiles * num_kb
   int max_pieces;      // partial slots per CTA
-  // tile mode with stream-K: units split evenly over the CTAs, each CTA walks
-  // its range backwards; a tile split between two CTAs is finished by the one
-  // holding its last k-block, which adds the other's fp32 partial
-  int sk_tiles;
-  float* sk_partial;   // [grid][128][BN]
-  unsigned* sk_flags;  // [grid]: epoch once that CTA's partial is written
-  unsigned sk_epoch;
   DevStatus* status;
   unsigned long long limit_ns;
 };
@@ -89,24 +82,16 @@ struct GemmItem {
 struct GemmIter {
   // tile mode
   int next_tile, tile_count;
-  // stream-K modes
-  long long u, u0, u1;
+  // stream-K mode
+  long long u, u1;
   int first_tile;
   int num_kb;
   bool streamk;
-  bool reverse;   // tile stream-K: walk the unit range backwards
 
   __device__ void init(const GemmParams& p, bool sk) {
     streamk = sk;
-    reverse = false;
     num_kb = p.num_kb;
-    if (!sk && p.sk_tiles) {
-      const long long G = gridDim.x;
-      u0 = p.units * (long long)blockIdx.x / G;
-      u1 = p.units * (long long)(blockIdx.x + 1) / G;
-      u = u1;
-      reverse = true;
-    } else if (!sk) {
+    if (!sk) {
       next_tile = blockIdx.x;
       tile_count = p.m_tiles * p.n_tiles;
     } else {
@@ -117,17 +102,6 @@ struct GemmIter {
     }
   }
   __device__ bool next(GemmItem& it) {
-    if (reverse) {
-      if (u <= u0) return false;
-      it.tile = (int)((u - 1) / num_kb);
-      const long long start = (long long)it.tile * num_kb;
-      const long long lo = u0 > start ? u0 : start;
-      it.kb0 = (int)(lo - start);
-      it.kb1 = (int)(u - start);
-      it.slot = 0;
-      u = lo;
-      return true;
-    }
     if (!streamk) {
       if (next_tile >= tile_count) return false;
       it.tile = next_tile;
@@ -341,58 +315,11 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < 16; ++j)
             if (c + j < p.act_rows) dst[(size_t)(c + j) * 128 + row] = v[j];
         }
-      } else if (p.sk_tiles && item.kb1 < p.num_kb) {
-        // head piece of a split tile: publish the fp32 partial for its finisher
-        float* dst = p.sk_partial + ((size_t)blockIdx.x * 128 + row) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          tmem_ld32(tbase + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            reinterpret_cast<float4*>(dst + c)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 64) {
-          __threadfence();
-          asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.sk_flags + blockIdx.x), "r"(p.sk_epoch)
-                       : "memory");
-        }
       } else {
         const int wtile = item.tile / p.m_tiles;
         const int m = (item.tile % p.m_tiles) * 128 + row;
         const bool row_ok = m < p.act_rows;
-        // tail piece of a split tile: wait for the head's partial (written by the CTA
-        // whose range holds the tile's first unit) and add it below
-        const float* add = nullptr;
-        if (p.sk_tiles && item.kb0 > 0) {
-          const long long x = (long long)item.tile * p.num_kb;
-          const long long G = gridDim.x;
-          long long c = ((x + 1) * G + p.units - 1) / p.units - 1;
-          c = c < 0 ? 0 : (c > G - 1 ? G - 1 : c);
-          const unsigned* flag = p.sk_flags + c;
-          if (threadIdx.x == 64) {
-            const uint64_t t0 = globaltimer_ns();
-            while (true) {
-              unsigned f;
-              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
-              if (f == p.sk_epoch) break;
-              if (globaltimer_ns() - t0 > p.limit_ns) {
-                abort_sh = 1;
-                record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 5, item.tile);
-                break;
-              }
-              __nanosleep(64);
-            }
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          unsigned f;
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
-          (void)f;
-          add = p.sk_partial + ((size_t)c * 128 + row) * BN;
-        }
+
         if (EPI == EPI_SWIGLU_BF16) {
           const int n0 = wtile * (BN / 2);
           const int nlim = p.seg_rows[0];
@@ -403,15 +330,6 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld32(tbase + c, g);
             tmem_ld32(tbase + BN / 2 + c, u);
             tmem_ld_wait();
-            if (add != nullptr) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 a = reinterpret_cast<const float4*>(add + c)[q];
-                const float4 b2 = reinterpret_cast<const float4*>(add + BN / 2 + c)[q];
-                g[4 * q] += a.x; g[4 * q + 1] += a.y; g[4 * q + 2] += a.z; g[4 * q + 3] += a.w;
-                u[4 * q] += b2.x; u[4 * q + 1] += b2.y; u[4 * q + 2] += b2.z; u[4 * q + 3] += b2.w;
-              }
-            }
             if (row_ok) {
               const int n = n0 + c;
               if (n + 32 <= nlim) {
@@ -441,13 +359,6 @@ __global__ void __launch_bounds__(192, 1)
             float v[32];
             tmem_ld32(tbase + c, v);
             tmem_ld_wait();
-            if (add != nullptr) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 a = reinterpret_cast<const float4*>(add + c)[q];
-                v[4 * q] += a.x; v[4 * q + 1] += a.y; v[4 * q + 2] += a.z; v[4 * q + 3] += a.w;
-              }
-            }
             if (!row_ok || nl0 + c >= nlim) continue;
             const bool full = nl0 + c + 32 <= nlim;
             const int n = col0 + c;
