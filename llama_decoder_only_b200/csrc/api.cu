@@ -366,7 +366,7 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
   }
   {
     TRACE(kind, st);
-    CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, 192, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
+    CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -464,6 +464,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.n_tiles = t;
   p.units = (long long)p.n_tiles * p.num_kb;
   const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
+  if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;  // reduce uses 32-bit unit math
   const long long per = (p.units + grid - 1) / grid;
   p.max_pieces = (int)((per + p.num_kb - 1) / p.num_kb) + 1;
   llama_status s = LLAMA_OK;

@@ -236,26 +236,25 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
-      }
+      // all four 32-column loads in flight, one wait
+      float sv[4][32];
+      tmem_ld32(tS + 0, sv[0]);
+      tmem_ld32(tS + 32, sv[1]);
+      tmem_ld32(tS + 64, sv[2]);
+      tmem_ld32(tS + 96, sv[3]);
+      tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_free(t));
+      // raw scores: the scale (> 0) is applied once to the maximum and folded
+      // into the exponent below
       const bool need_mask = j * 128 + 127 > pos_min;
-      float mx = -INFINITY;
+      float mraw = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 128; ++i) {
-        float x = s[i] * p.scale_log2;
-        if (need_mask && (j * 128 + i > pos)) x = -INFINITY;
-        s[i] = x;
-        mx = fmaxf(mx, x);
+        if (need_mask && (j * 128 + i > pos)) sv[i >> 5][i & 31] = -INFINITY;
+        mraw = fmaxf(mraw, sv[i >> 5][i & 31]);
       }
+      const float mx = mraw * p.scale_log2;
       // Move this row's reference maximum only when it grew by more than
       // 2^8; rows that keep theirs use alpha = 1.  The O rescale below is a
       // warp-collective TMEM read-modify-write, so the warp does it when any
@@ -273,34 +272,61 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      if (rescale) {
-        l *= alpha;
-        for (int c = 0; c < hd_pad; c += 32) {
-          float v[32];
-          tmem_ld32(tO + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(tO + c, v);
-        }
-        tmem_st_wait();
-      }
       // P = 2^(s - m_used) as bf16 into the swizzled K-major A tile
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      const float sc = p.scale_log2;
       float psum = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {   // 16-byte chunk c holds keys 8c .. 8c+7
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = ex2_approx(s[8 * c + 2 * e] - mref);
-          const float bb = ex2_approx(s[8 * c + 2 * e + 1] - mref);
+          const int i0 = 8 * c + 2 * e;
+          const float a = ex2_approx(fmaf(sv[i0 >> 5][i0 & 31], sc, -mref));
+          const float bb = ex2_approx(fmaf(sv[(i0 + 1) >> 5][(i0 + 1) & 31], sc, -mref));
           psum += a + bb;
           w[e] = pack_bf16x2(a, bb);
         }
         const int region = c >> 3, cc = c & 7;
         uint8_t* dst = prow0 + region * ATT_REGION + ((cc ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // rescale O after P is written: the scores are dead by now, which keeps
+      // the 128 loaded O columns from competing with them for registers
+      if (rescale) {
+        l *= alpha;
+        if (hd_pad == 128) {
+          float v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(tO + 0, v0);
+          tmem_ld32(tO + 32, v1);
+          tmem_ld32(tO + 64, v2);
+          tmem_ld32(tO + 96, v3);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v0[i] *= alpha;
+            v1[i] *= alpha;
+            v2[i] *= alpha;
+            v3[i] *= alpha;
+          }
+          tmem_st32(tO + 0, v0);
+          tmem_st32(tO + 32, v1);
+          tmem_st32(tO + 64, v2);
+          tmem_st32(tO + 96, v3);
+        } else {
+          float v0[32], v1[32];
+          tmem_ld32(tO + 0, v0);
+          tmem_ld32(tO + 32, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v0[i] *= alpha;
+            v1[i] *= alpha;
+          }
+          tmem_st32(tO + 0, v0);
+          tmem_st32(tO + 32, v1);
+        }
+        tmem_st_wait();
       }
       l += psum;
       fence_proxy_async_smem();

@@ -7,8 +7,10 @@
 //               STAGES shared-memory stages, 128-byte swizzle, no multicast;
 //   warp 1      TMEM allocator and MMA issuer (one lane): 4 x tcgen05.mma
 //               (M=128, N=BN, K=16) per 64-wide k-block, commit frees the stage;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread), fused epilogue, global store.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread; two warps per lane quadrant, each
+//               taking half of the tile's columns), fused epilogue, global
+//               store.
 // The accumulator is double-buffered in TMEM (2 x BN fp32 columns), so the
 // epilogue of one tile overlaps the main loop of the next.
 //
@@ -58,6 +60,9 @@ struct GemmParams {
   DevStatus* status;
   unsigned long long limit_ns;
 };
+
+constexpr int GEMM_EPI_WARPS = 8;
+constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 
 template <int BN>
 struct GemmCfg {
@@ -130,7 +135,7 @@ __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
 }
 
 template <int BN, bool SWAP, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW0,
                    const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                    const GemmParams p) {
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 128);
+      mbar_init(acce_bar(b), 32 * GEMM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
     fence_barrier_init();
@@ -291,8 +296,9 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int quad = warp & 3;
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;          // which half of the tile's columns
     const int row = quad * 32 + lane;  // TMEM lane == accumulator row
     int abuf = 0;
     uint32_t aphase = 0;
@@ -307,7 +313,7 @@ __global__ void __launch_bounds__(192, 1)
         // partial[(cta * max_pieces + slot)][token][128] (fp32); row = weight row in tile
         float* dst = p.partial + ((size_t)blockIdx.x * p.max_pieces + item.slot) * (size_t)BN * 128;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = half * 16; c < BN; c += 32) {
           float v[16];
           tmem_ld16(tbase + c, v);
           tmem_ld_wait();
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(192, 1)
           const int nlim = p.seg_rows[0];
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.ldo;
 #pragma unroll 1
-          for (int c = 0; c < BN / 2; c += 32) {
+          for (int c = half * (BN / 4); c < (half + 1) * (BN / 4); c += 32) {
             float g[32], u[32];
             tmem_ld32(tbase + c, g);
             tmem_ld32(tbase + BN / 2 + c, u);
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(192, 1)
           const int nlim = p.seg_rows[seg];
           const int col0 = p.seg_col0[seg] + nl0;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
             float v[32];
             tmem_ld32(tbase + c, v);
             tmem_ld_wait();
@@ -447,20 +453,22 @@ struct ReduceParams {
 };
 
 // Sum of the stream-K pieces of weight row `wrow` (tile-local `r`) for token `t`.
+// 32-bit arithmetic: the host guarantees units * grid < 2^32.
 __device__ __forceinline__ float sk_sum(const ReduceParams& p, int wtile, int r, int t) {
-  const long long x = (long long)wtile * p.num_kb;
-  // largest CTA c with floor(units*c/G) <= x
-  long long c = ((x + 1) * p.grid + p.units - 1) / p.units - 1;
+  const unsigned U = (unsigned)p.units, G = (unsigned)p.grid, KB = (unsigned)p.num_kb;
+  const unsigned x = (unsigned)wtile * KB;
+  // largest CTA c with floor(U*c/G) <= x
+  int c = (int)(((x + 1) * G + U - 1) / U) - 1;
   if (c < 0) c = 0;
   if (c > p.grid - 1) c = p.grid - 1;
   float s = 0.f;
-  const long long xend = x + p.num_kb;
+  const unsigned xend = x + KB;
   for (; c < p.grid; ++c) {
-    const long long start = p.units * c / p.grid;
+    const unsigned start = U * (unsigned)c / G;
     if (start >= xend) break;
-    const long long stop = p.units * (c + 1) / p.grid;
+    const unsigned stop = U * (unsigned)(c + 1) / G;
     if (stop <= start) continue;
-    const int slot = wtile - (int)(start / p.num_kb);
+    const int slot = wtile - (int)(start / KB);
     s += p.partial[((size_t)c * p.max_pieces + slot) * (size_t)p.BN * 128 + (size_t)t * 128 + r];
   }
   return s;
