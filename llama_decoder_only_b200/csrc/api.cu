@@ -47,12 +47,12 @@ constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K for
 
 enum KernelKind : int {
   K_RMSNORM = 0, K_GEMM_QKV, K_ROPE_APPEND, K_ATTN_PREFILL, K_ATTN_DECODE, K_ATTN_COMBINE, K_GEMM_O,
-  K_GEMM_GATE_UP, K_GEMM_DOWN, K_SPLITK_REDUCE, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
+  K_GEMM_GATE_UP, K_GEMM_DOWN, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
   K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
   "rmsnorm", "gemm_qkv", "rope_kv_append", "attn_prefill", "attn_decode", "attn_decode_combine", "gemm_o_proj",
-  "gemm_gate_up_swiglu", "gemm_down", "splitk_reduce", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
+  "gemm_gate_up_swiglu", "gemm_down", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
   "gemm_f32", "attn_f32", "selftest"};
 
 struct ProfRec {
@@ -296,18 +296,15 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // ------------------------------------------------------------------ workspace layout
 
 struct WsLayout {
-  size_t qkv, h, attn, mbuf, partial, att_ml, att_o;        // layer scratch
+  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o;   // layer scratch
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
 
 int swap_bn(int tokens) { return tokens <= 16 ? 16 : tokens <= 32 ? 32 : tokens <= 64 ? 64 : 128; }
 
-// Bound on the stream-K partial buffer of one decode GEMM (floats).
-size_t sk_partial_floats(int n_rows_total, int tokens) {
-  const long long n_tiles = cdiv(n_rows_total, 128) + 3;  // + segment padding
-  return (size_t)(n_tiles + 3LL * kMaxSkGrid) * swap_bn(tokens) * 128;
-}
+// Stream-K partial buffer of one decode GEMM (floats): one [BN][128] piece per CTA.
+size_t sk_partial_floats(int tokens) { return (size_t)kMaxSkGrid * swap_bn(tokens) * 128; }
 
 WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   WsLayout w{};
@@ -324,15 +321,10 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   w.h = take(M * (size_t)d.dim * es);
   w.attn = take(M * (size_t)d.n_heads * d.head_dim * es);
   w.mbuf = take(M * (size_t)d.ffn_dim * es);
-  size_t pf = 0;
-  if (d.dtype == LLAMA_BF16 && batch <= kSwapMaxTokens) {
-    // decode GEMMs (M = batch) and the lm_head on the last rows (M = batch)
-    pf = sk_partial_floats(qkvn, batch);
-    pf = std::max(pf, sk_partial_floats(d.dim, batch));
-    pf = std::max(pf, sk_partial_floats(2 * d.ffn_dim, batch));
-    if (vocab > 0) pf = std::max(pf, sk_partial_floats(vocab, batch));
-  }
-  w.partial = take(pf * 4);
+  // decode GEMMs (M = batch) and the lm_head on the last rows (M = batch)
+  const bool sk = d.dtype == LLAMA_BF16 && batch <= kSwapMaxTokens;
+  w.partial = take(sk ? sk_partial_floats(batch) * 4 : 0);
+  w.sk_flags = take(sk ? (size_t)kMaxSkGrid * 4 : 0);
   w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
   w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
   if (vocab > 0) {
@@ -370,6 +362,24 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
+}
+
+// Stream-K scratch of the decode GEMMs: one fp32 piece and one flag per CTA.
+struct SkScratch {
+  float* partial;
+  unsigned* flags;
+};
+
+template <int BN>
+llama_status launch_gemm_sk(int epi, const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
+                            cudaStream_t st, int kind) {
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_tc<BN, true, EPI_BF16>(a, w, p, grid, st, kind);
+    case EPI_RESID_F32: return launch_gemm_tc<BN, true, EPI_RESID_F32>(a, w, p, grid, st, kind);
+    case EPI_SWIGLU_BF16: return launch_gemm_tc<BN, true, EPI_SWIGLU_BF16>(a, w, p, grid, st, kind);
+    case EPI_F32: return launch_gemm_tc<BN, true, EPI_F32>(a, w, p, grid, st, kind);
+  }
+  return LLAMA_ERR_INVALID_ARG;
 }
 
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
@@ -431,10 +441,11 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
   return LLAMA_ERR_INVALID_ARG;
 }
 
-// Stream-K (decode) GEMM: partials = act[M, K] · W^T with W as the MMA's A
-// operand, then the reduce kernel applies `dec_epi`.
-llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int dec_epi,
-                         void* out, int ldo, const float* resid, int ldr, float* partial, DevStatus* status,
+// Stream-K (decode) GEMM: out = epilogue(act[M, K] · W^T) with W as the MMA's
+// A operand.  The CTA that ends a weight tile adds the other CTAs' pieces of
+// it (published in `sk.partial` under `sk.flags`) and applies the epilogue.
+llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
+                         void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
                          int kind) {
   const int BN = swap_bn(M);
   GemmParams p{};
@@ -443,85 +454,55 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.act_rows = M;
   p.m_tiles = 1;
   p.nseg = nseg;
+  p.out = out;
+  p.ldo = ldo;
+  p.resid = resid;
+  p.ldr = ldr;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
-  p.partial = partial;
+  p.partial = sk.partial;
+  p.flags = sk.flags;
   CUtensorMap ta, tw[3];
   std::memset(tw, 0, sizeof(tw));
   if (!make_map_2d(&ta, act, K, M, BN)) return LLAMA_ERR_CUDA;
   int t = 0;
-  int n_out = 0;
-  for (int s = 0; s < nseg; ++s) {
-    p.seg_rows[s] = segs[s].rows;
-    p.seg_col0[s] = segs[s].col0;
-    p.seg_tile0[s] = t;
-    t += cdiv(segs[s].rows, 128);
-    n_out = std::max(n_out, segs[s].col0 + segs[s].rows);
-    if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, 128)) return LLAMA_ERR_CUDA;
+  if (epi == EPI_SWIGLU_BF16) {
+    // a weight tile = 64 gate rows + the matching 64 up rows
+    p.seg_rows[0] = segs[0].rows;
+    t = cdiv(segs[0].rows, 64);
+    for (int s = 0; s < 2; ++s)
+      if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, 64)) return LLAMA_ERR_CUDA;
+    tw[2] = tw[0];
+  } else {
+    for (int s = 0; s < nseg; ++s) {
+      p.seg_rows[s] = segs[s].rows;
+      p.seg_col0[s] = segs[s].col0;
+      p.seg_tile0[s] = t;
+      t += cdiv(segs[s].rows, 128);
+      if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, 128)) return LLAMA_ERR_CUDA;
+    }
+    for (int s = nseg; s < 3; ++s) tw[s] = tw[0];
   }
-  for (int s = nseg; s < 3; ++s) tw[s] = tw[0];
-  for (int s = nseg; s < 4; ++s) p.seg_tile0[s] = t;
+  for (int s = (epi == EPI_SWIGLU_BF16 ? 1 : nseg); s < 4; ++s) p.seg_tile0[s] = t;
   p.n_tiles = t;
   p.units = (long long)p.n_tiles * p.num_kb;
+  // no CTA may have an empty unit range: a tile's finisher waits on every CTA between
   const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
-  if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;  // reduce uses 32-bit unit math
-  const long long per = (p.units + grid - 1) / grid;
-  p.max_pieces = (int)((per + p.num_kb - 1) / p.num_kb) + 1;
-  llama_status s = LLAMA_OK;
+  if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;  // 32-bit unit math
   switch (BN) {
-    case 16: s = launch_gemm_tc<16, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
-    case 32: s = launch_gemm_tc<32, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
-    case 64: s = launch_gemm_tc<64, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
-    default: s = launch_gemm_tc<128, true, EPI_PARTIAL>(ta, tw, p, grid, st, kind); break;
+    case 16: return launch_gemm_sk<16>(epi, ta, tw, p, grid, st, kind);
+    case 32: return launch_gemm_sk<32>(epi, ta, tw, p, grid, st, kind);
+    case 64: return launch_gemm_sk<64>(epi, ta, tw, p, grid, st, kind);
+    default: return launch_gemm_sk<128>(epi, ta, tw, p, grid, st, kind);
   }
-  if (s != LLAMA_OK) return s;
-  ReduceParams r{};
-  r.act_rows = M;
-  r.num_kb = p.num_kb;
-  r.units = p.units;
-  r.grid = grid;
-  r.max_pieces = p.max_pieces;
-  r.BN = BN;
-  r.nseg = nseg;
-  for (int i = 0; i < 3; ++i) {
-    r.seg_rows[i] = p.seg_rows[i];
-    r.seg_col0[i] = p.seg_col0[i];
-  }
-  for (int i = 0; i < 4; ++i) r.seg_tile0[i] = p.seg_tile0[i];
-  r.partial = partial;
-  r.out = out;
-  r.ldo = ldo;
-  r.resid = resid;
-  r.ldr = ldr;
-  if (dec_epi == DEC_SWIGLU_BF16) {
-    r.ffn = segs[0].rows;
-    n_out = segs[0].rows;
-  }
-  r.n_out = n_out;
-  dim3 grid_r(cdiv(n_out, 256), M);
-  TRACE(K_SPLITK_REDUCE, st);
-  switch (dec_epi) {
-    case DEC_BF16: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_BF16>, grid_r, 256, 0, st, r)); break;
-    case DEC_RESID_F32: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_RESID_F32>, grid_r, 256, 0, st, r)); break;
-    case DEC_SWIGLU_BF16: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_SWIGLU_BF16>, grid_r, 256, 0, st, r)); break;
-    default: CUDA_TRY(launch_k(splitk_reduce_kernel<DEC_F32>, grid_r, 256, 0, st, r)); break;
-  }
-  LAUNCH_CHECK();
-  return LLAMA_OK;
 }
 
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
-                       int epi, void* out, int ldo, const float* resid, int ldr, float* partial,
+                       int epi, void* out, int ldo, const float* resid, int ldr, SkScratch sk,
                        DevStatus* status, int kind) {
-  if (decode && M <= kSwapMaxTokens) {
-    const int dec = epi == EPI_BF16 ? DEC_BF16 : epi == EPI_RESID_F32 ? DEC_RESID_F32
-                  : epi == EPI_SWIGLU_BF16 ? DEC_SWIGLU_BF16 : DEC_F32;
-    WSeg s2[3];
-    for (int i = 0; i < nseg; ++i) s2[i] = segs[i];
-    if (epi == EPI_SWIGLU_BF16) s2[1].col0 = segs[0].rows;  // up rows follow the gate rows
-    return gemm_decode(st, act, M, K, s2, nseg, dec, out, ldo, resid, ldr, partial, status, kind);
-  }
+  if (decode && M <= kSwapMaxTokens)
+    return gemm_decode(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, kind);
   return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
 }
 
@@ -723,7 +704,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     bf* h = reinterpret_cast<bf*>(ws + lay.h);
     bf* att = reinterpret_cast<bf*>(ws + lay.attn);
     bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
-    float* part = reinterpret_cast<float*>(ws + lay.partial);
+    const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
     // a2: RMSNorm-1 -> h (bf16)
     {
       TRACE(K_RMSNORM, st);
@@ -1078,7 +1059,8 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};
     TRY(gemm_bf16(st, true, hl, batch, d.dim, &s, 1, EPI_F32, logits, m->vocab, nullptr, 0,
-                  reinterpret_cast<float*>(ws + lay.partial), status, K_GEMM_LM_HEAD));
+                  SkScratch{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)},
+                  status, K_GEMM_LM_HEAD));
   } else {
     float* hl = reinterpret_cast<float*>(ws + lay.hl);
     {

@@ -24,9 +24,13 @@
 //  * stream-K mode (decode, SWAP = true): the weight is A (its rows fill the
 //    MMA's M = 128) and the few token rows are B (N = BN >= tokens), so the
 //    weight streams from HBM once.  The (weight tile, k-block) units are split
-//    evenly over the CTAs; each CTA writes one fp32 partial per tile piece and
-//    a separate reduce kernel adds the pieces in CTA order (deterministic)
-//    and applies the epilogue.
+//    evenly over the CTAs and each CTA walks its range backwards: its only
+//    piece that does not end a tile comes first and is published at once as
+//    an fp32 partial plus an epoch flag; the CTA that holds a tile's last
+//    k-block waits (bounded) for the lower CTAs' partials, adds them in CTA
+//    order (deterministic) and applies the epilogue itself.  For gate_up a
+//    weight tile is 64 gate rows followed by the matching 64 up rows, so
+//    SiLU(gate)·up pairs TMEM lane r with lane r + 64 (through shared memory).
 //
 // The weight can be given as up to three row segments with their own tensor
 // maps (q, k, v when the three projections are not contiguous; gate and up).
@@ -36,7 +40,7 @@
 
 namespace llama {
 
-enum GemmEpi : int { EPI_BF16 = 0, EPI_RESID_F32 = 1, EPI_SWIGLU_BF16 = 2, EPI_F32 = 3, EPI_PARTIAL = 4 };
+enum GemmEpi : int { EPI_BF16 = 0, EPI_RESID_F32 = 1, EPI_SWIGLU_BF16 = 2, EPI_F32 = 3 };
 
 struct GemmParams {
   int K;
@@ -54,9 +58,9 @@ struct GemmParams {
   const float* resid;
   int ldr;
   // stream-K mode
-  float* partial;
+  float* partial;      // [grid][128 rows][BN tokens] fp32: each CTA's one non-final piece
+  unsigned* flags;     // [grid]: 1 while that CTA's partial waits for its finisher, else 0
   long long units;     // n_tiles * num_kb
-  int max_pieces;      // partial slots per CTA
   DevStatus* status;
   unsigned long long limit_ns;
 };
@@ -74,22 +78,21 @@ struct GemmCfg {
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                         : (2 * BN <= 256) ? 256 : 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int EXCH_BYTES = 2 * 64 * 16 * 4;   // gate/up pairing exchange (stream-K gate_up)
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + EXCH_BYTES;
 };
 
 // Work item shared by the three roles: one output tile and a k-block range.
 struct GemmItem {
   int tile;   // tile mode: linear (m fastest); stream-K: weight tile
   int kb0, kb1;
-  int slot;   // swap stream-K: partial slot within the CTA
 };
 
 struct GemmIter {
   // tile mode
   int next_tile, tile_count;
-  // stream-K mode
-  long long u, u1;
-  int first_tile;
+  // stream-K mode: this CTA's unit range [u0, u1), walked from the top
+  long long u, u0;
   int num_kb;
   bool streamk;
 
@@ -101,9 +104,8 @@ struct GemmIter {
       tile_count = p.m_tiles * p.n_tiles;
     } else {
       const long long G = gridDim.x;
-      u = p.units * (long long)blockIdx.x / G;
-      u1 = p.units * (long long)(blockIdx.x + 1) / G;
-      first_tile = (int)(u / num_kb);
+      u0 = p.units * (long long)blockIdx.x / G;
+      u = p.units * (long long)(blockIdx.x + 1) / G;
     }
   }
   __device__ bool next(GemmItem& it) {
@@ -112,17 +114,16 @@ struct GemmIter {
       it.tile = next_tile;
       it.kb0 = 0;
       it.kb1 = num_kb;
-      it.slot = 0;
       next_tile += gridDim.x;
       return true;
     }
-    if (u >= u1) return false;
-    it.tile = (int)(u / num_kb);
-    it.kb0 = (int)(u % num_kb);
-    long long rem = u1 - u;
-    it.kb1 = (int)((long long)it.kb0 + rem < num_kb ? it.kb0 + rem : num_kb);
-    it.slot = it.tile - first_tile;
-    u += it.kb1 - it.kb0;
+    if (u <= u0) return false;
+    it.tile = (int)((u - 1) / num_kb);
+    const long long start = (long long)it.tile * num_kb;
+    const long long lo = u0 > start ? u0 : start;
+    it.kb0 = (int)(lo - start);
+    it.kb1 = (int)(u - start);
+    u = lo;
     return true;
   }
 };
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, epilogue group
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
   auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  const uint32_t epi_bar = bar0 + 8u * (2 * STAGES + 5);
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(acce_bar(b), 32 * GEMM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(epi_bar, 32 * GEMM_EPI_WARPS);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -220,7 +223,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sb = sa + C::A_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
           if (SWAP) {
-            tma_load_2d(sa, wm, full_bar(stage), kb * 64, wrow0);
+            if (EPI == EPI_SWIGLU_BF16) {
+              // 64 gate rows into lanes 0..63 of the tile, the same 64 up rows into 64..127
+              tma_load_2d(sa, &tmW0, full_bar(stage), kb * 64, wtile * 64);
+              tma_load_2d(sa + 64 * 128, &tmW1, full_bar(stage), kb * 64, wtile * 64);
+            } else {
+              tma_load_2d(sa, wm, full_bar(stage), kb * 64, wrow0);
+            }
             tma_load_2d(sb, &tmAct, full_bar(stage), kb * 64, 0);
           } else {
             tma_load_2d(sa, &tmAct, full_bar(stage), kb * 64, m0);
@@ -300,6 +309,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may read
     const int half = (warp - 2) >> 2;          // which half of the tile's columns
     const int row = quad * 32 + lane;  // TMEM lane == accumulator row
+    // Barrier of the epilogue warps: an mbarrier with a bounded wait rather than
+    // a named barrier, so a warp that left the loop on an error cannot hang the rest.
+    uint32_t epi_phase = 0;
+    auto epi_sync = [&]() {
+      mbar_arrive(epi_bar);
+      mbar_wait(epi_bar, epi_phase, wc, 7);
+      epi_phase ^= 1u;
+    };
     int abuf = 0;
     uint32_t aphase = 0;
     GemmIter it;
@@ -310,16 +327,135 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(abuf * BN);
       if (SWAP) {
-        // partial[(cta * max_pieces + slot)][token][128] (fp32); row = weight row in tile
-        float* dst = p.partial + ((size_t)blockIdx.x * p.max_pieces + item.slot) * (size_t)BN * 128;
+        // accumulator: TMEM lane `row` = weight row of the tile, column j = token j
+        if (item.kb1 < p.num_kb) {
+          // a piece that does not end its tile: publish it for the tile's finisher
+          float* dst = p.partial + ((size_t)blockIdx.x * 128 + row) * BN;
 #pragma unroll 1
-        for (int c = half * 16; c < BN; c += 32) {
-          float v[16];
-          tmem_ld16(tbase + c, v);
-          tmem_ld_wait();
+          for (int c = half * 16; c < BN; c += 32) {
+            float v[16];
+            tmem_ld16(tbase + c, v);
+            tmem_ld_wait();
+            float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c + j < p.act_rows) dst[(size_t)(c + j) * 128 + row] = v[j];
+            for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+          // the group barrier orders every thread's stores before thread 64's
+          // release, which makes them visible at GPU scope before the flag
+          epi_sync();
+          if (threadIdx.x == 64)
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + blockIdx.x), "r"(1u) : "memory");
+        } else {
+          // this CTA ends the tile: add the partials of the lower CTAs that share it
+          const unsigned U = (unsigned)p.units, G = gridDim.x, KB = (unsigned)p.num_kb;
+          const unsigned x = (unsigned)item.tile * KB;
+          int c_first = (int)(((x + 1) * G + U - 1) / U) - 1;
+          c_first = c_first < 0 ? 0 : c_first;
+          // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count)
+          const int n_contrib = (int)blockIdx.x - c_first;
+          if (n_contrib > 0) {
+            if (threadIdx.x == 64) {
+              for (int c = c_first; c < (int)blockIdx.x; ++c) {
+                const uint64_t t0 = globaltimer_ns();
+                while (true) {
+                  unsigned f;
+                  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.flags + c) : "memory");
+                  if (f == 1u || *reinterpret_cast<volatile int*>(&abort_sh)) break;
+                  if (globaltimer_ns() - t0 > p.limit_ns) {
+                    abort_sh = 1;
+                    record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 6, item.tile);
+                    break;
+                  }
+                  __nanosleep(32);
+                }
+                // this CTA is the only reader of c's piece: re-arm the flag for the next launch
+                asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.flags + c), "r"(0u) : "memory");
+              }
+            }
+            epi_sync();
+          }
+          // weight row -> output column
+          int seg = 0, n = 0;
+          bool n_ok;
+          if (EPI == EPI_SWIGLU_BF16) {
+            n = item.tile * 64 + (row & 63);
+            n_ok = n < p.seg_rows[0];
+          } else {
+            seg = seg_of_tile(p, item.tile);
+            const int r_in_seg = (item.tile - p.seg_tile0[seg]) * 128 + row;
+            n_ok = r_in_seg < p.seg_rows[seg];
+            n = p.seg_col0[seg] + r_in_seg;
+          }
+          float* xch = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16);
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            const int c = c0 + half * 16;   // this warp's 16 token columns (BN is a multiple of 16)
+            const bool active = c < BN;
+            float v[16];
+            if (active) {
+              tmem_ld16(tbase + c, v);
+              tmem_ld_wait();
+              // the contributors' pieces, in CTA order, up to four per round trip to L2
+              const float4* src = reinterpret_cast<const float4*>(p.partial + ((size_t)c_first * 128 + row) * BN + c);
+              constexpr size_t STRIDE4 = (size_t)128 * BN / 4;
+#pragma unroll 1
+              for (int k = 0; k < n_contrib; k += 4) {
+                float4 a[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                  for (int q = 0; q < 4; ++q)
+                    a[i][q] = k + i < n_contrib ? __ldcg(src + (size_t)(k + i) * STRIDE4 + q)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    v[4 * q + 0] += a[i][q].x;
+                    v[4 * q + 1] += a[i][q].y;
+                    v[4 * q + 2] += a[i][q].z;
+                    v[4 * q + 3] += a[i][q].w;
+                  }
+              }
+            }
+            if (EPI == EPI_SWIGLU_BF16) {
+              // up values (lanes 64..127) go through shared memory to the gate lanes
+              if (active && row >= 64) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) xch[j * 64 + row - 64] = v[j];
+              }
+              epi_sync();
+              if (active && row < 64 && n_ok) {
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (c + j < p.act_rows)
+                    o[(size_t)(c + j) * p.ldo + n] = __float2bfloat16_rn(silu_f(v[j]) * xch[j * 64 + row]);
+              }
+              epi_sync();
+            } else if (active && n_ok) {
+              const int nj = p.act_rows - c < 16 ? p.act_rows - c : 16;
+              if (EPI == EPI_RESID_F32) {
+                // all residual loads first (out may alias resid: same element, same thread)
+                float r[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) r[j] = j < nj ? p.resid[(size_t)(c + j) * p.ldr + n] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (j < nj) reinterpret_cast<float*>(p.out)[(size_t)(c + j) * p.ldo + n] = r[j] + v[j];
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  if (j >= nj) break;
+                  const size_t o_idx = (size_t)(c + j) * p.ldo + n;
+                  if (EPI == EPI_BF16)
+                    reinterpret_cast<__nv_bfloat16*>(p.out)[o_idx] = __float2bfloat16_rn(v[j]);
+                  else
+                    reinterpret_cast<float*>(p.out)[o_idx] = v[j];
+                }
+              }
+            }
+          }
         }
       } else {
         const int wtile = item.tile / p.m_tiles;
@@ -426,87 +562,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
-}
-
-// ------------------------------------------------------------------ stream-K reduce + epilogue
-
-enum DecEpi : int { DEC_BF16 = 0, DEC_RESID_F32 = 1, DEC_SWIGLU_BF16 = 2, DEC_F32 = 3 };
-
-struct ReduceParams {
-  int act_rows;         // tokens
-  int n_out;            // output columns
-  int num_kb;
-  long long units;
-  int grid;             // CTAs of the GEMM launch
-  int max_pieces;
-  int BN;               // token columns per partial piece
-  int nseg;
-  int seg_rows[3];
-  int seg_tile0[4];
-  int seg_col0[3];
-  const float* partial;
-  void* out;
-  int ldo;
-  const float* resid;
-  int ldr;
-  int ffn;              // DEC_SWIGLU: gate in segment 0, up in segment 1
-};
-
-// Sum of the stream-K pieces of weight row `wrow` (tile-local `r`) for token `t`.
-// 32-bit arithmetic: the host guarantees units * grid < 2^32.
-__device__ __forceinline__ float sk_sum(const ReduceParams& p, int wtile, int r, int t) {
-  const unsigned U = (unsigned)p.units, G = (unsigned)p.grid, KB = (unsigned)p.num_kb;
-  const unsigned x = (unsigned)wtile * KB;
-  // largest CTA c with floor(U*c/G) <= x
-  int c = (int)(((x + 1) * G + U - 1) / U) - 1;
-  if (c < 0) c = 0;
-  if (c > p.grid - 1) c = p.grid - 1;
-  float s = 0.f;
-  const unsigned xend = x + KB;
-  for (; c < p.grid; ++c) {
-    const unsigned start = U * (unsigned)c / G;
-    if (start >= xend) break;
-    const unsigned stop = U * (unsigned)(c + 1) / G;
-    if (stop <= start) continue;
-    const int slot = wtile - (int)(start / KB);
-    s += p.partial[((size_t)c * p.max_pieces + slot) * (size_t)p.BN * 128 + (size_t)t * 128 + r];
-  }
-  return s;
-}
-
-__device__ __forceinline__ int seg_tile_of_row(const ReduceParams& p, int seg, int row_in_seg, int& r) {
-  r = row_in_seg & 127;
-  return p.seg_tile0[seg] + (row_in_seg >> 7);
-}
-
-template <int EPI>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const ReduceParams p) {
-  pdl_wait();
-  const int t = blockIdx.y;
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= p.act_rows || n >= p.n_out) return;
-  if (EPI == DEC_SWIGLU_BF16) {
-    int rg, ru;
-    const int tg = seg_tile_of_row(p, 0, n, rg);
-    const int tu = seg_tile_of_row(p, 1, n, ru);
-    const float g = sk_sum(p, tg, rg, t);
-    const float u = sk_sum(p, tu, ru, t);
-    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)t * p.ldo + n] = __float2bfloat16_rn(silu_f(g) * u);
-    return;
-  }
-  int seg = 0;
-  if (p.nseg > 1 && n >= p.seg_col0[1]) seg = 1;
-  if (p.nseg > 2 && n >= p.seg_col0[2]) seg = 2;
-  int r;
-  const int wt = seg_tile_of_row(p, seg, n - p.seg_col0[seg], r);
-  const float v = sk_sum(p, wt, r, t);
-  if (EPI == DEC_BF16) {
-    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)t * p.ldo + n] = __float2bfloat16_rn(v);
-  } else if (EPI == DEC_RESID_F32) {
-    reinterpret_cast<float*>(p.out)[(size_t)t * p.ldo + n] = p.resid[(size_t)t * p.ldr + n] + v;
-  } else {
-    reinterpret_cast<float*>(p.out)[(size_t)t * p.ldo + n] = v;
-  }
 }
 
 }  // namespace llama
