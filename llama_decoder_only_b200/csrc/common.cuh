@@ -269,11 +269,15 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 // ------------------------------------------------------------------ programmatic dependent launch
 // Kernels are launched so that the next kernel in the stream may start once
-// every CTA of this one has called pdl_trigger (done at entry).  pdl_wait
+// every CTA of this one has called pdl_trigger: the GEMM and attention
+// kernels call it at the end of their work, the small kernels implicitly at
+// exit.  (An early trigger in the small kernels was measured slower: the
+// multi-wave decode attention grid then crowds onto the SMs that free first.)  pdl_wait
 // blocks until the previous kernel has completed and its writes are visible;
-// every kernel calls it before its first global-memory access, so each kernel
-// completes only after its predecessor (completion stays in stream order).
-// Both are no-ops for a kernel launched without the attribute.
+// every kernel calls it before it touches data an earlier kernel writes, so
+// each kernel completes only after its predecessor (completion stays in
+// stream order).  Only reads of data no kernel writes (the weights) may come
+// before it.  Both are no-ops for a kernel launched without the attribute.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

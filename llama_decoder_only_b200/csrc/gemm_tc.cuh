@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();
+  // stream-K (decode): the producer starts the weight stream before its PDL wait
+  if (!(SWAP && warp == 0)) pdl_wait();
   const uint32_t tmem_base = tmem_base_sh;
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, SWAP ? 2 : 1};
 
@@ -199,6 +200,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int filled_parity[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) filled_parity[s] = -1;
+      // weight tile of k-block kb of weight tile wtile (stream-K mode) into A stage sa
+      auto load_weight_swap = [&](uint32_t sa, uint32_t bar, int wtile, int kb) {
+        if (EPI == EPI_SWIGLU_BF16) {
+          // 64 gate rows into lanes 0..63 of the tile, the same 64 up rows into 64..127
+          tma_load_2d(sa, &tmW0, bar, kb * 64, wtile * 64);
+          tma_load_2d(sa + 64 * 128, &tmW1, bar, kb * 64, wtile * 64);
+        } else {
+          const int seg = seg_of_tile(p, wtile);
+          const CUtensorMap* wm = seg == 0 ? &tmW0 : (seg == 1 ? &tmW1 : &tmW2);
+          tma_load_2d(sa, wm, bar, kb * 64, (wtile - p.seg_tile0[seg]) * 128);
+        }
+      };
+      int skip = 0;   // k-blocks already issued before the PDL wait
+      if (SWAP) {
+        // The weights do not depend on the previous kernel: fill every stage's
+        // weight tile first, wait for the previous kernel, then add the
+        // activation tiles.  Every stage is empty at this point.
+        int pre_kb[STAGES];
+        GemmIter it;
+        it.init(p, true);
+        GemmItem item;
+        while (skip < STAGES && it.next(item)) {
+          for (int kb = item.kb0; kb < item.kb1 && skip < STAGES; ++kb) {
+            mbar_arrive_expect_tx(full_bar(skip), C::STAGE_BYTES);
+            load_weight_swap(smem_u32(smem + skip * C::STAGE_BYTES), full_bar(skip), item.tile, kb);
+            pre_kb[skip++] = kb;
+          }
+        }
+        pdl_wait();
+        for (int s = 0; s < skip; ++s) {
+          tma_load_2d(smem_u32(smem + s * C::STAGE_BYTES) + C::A_BYTES, &tmAct, full_bar(s), pre_kb[s] * 64, 0);
+          filled_parity[s] = 0;
+        }
+        stage = skip % STAGES;
+        phase = skip == STAGES ? 1u : 0u;
+      }
       GemmIter it;
       it.init(p, SWAP);
       GemmItem item;
@@ -215,6 +252,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int wrow0 = (wtile - p.seg_tile0[seg]) * WROWS;
         const CUtensorMap* wm = seg == 0 ? &tmW0 : (seg == 1 ? &tmW1 : &tmW2);
         for (int kb = item.kb0; kb < item.kb1; ++kb) {
+          if (skip > 0) {
+            --skip;
+            continue;
+          }
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc, 1)) {
             ok = false;
             break;
@@ -223,13 +264,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sb = sa + C::A_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
           if (SWAP) {
-            if (EPI == EPI_SWIGLU_BF16) {
-              // 64 gate rows into lanes 0..63 of the tile, the same 64 up rows into 64..127
-              tma_load_2d(sa, &tmW0, full_bar(stage), kb * 64, wtile * 64);
-              tma_load_2d(sa + 64 * 128, &tmW1, full_bar(stage), kb * 64, wtile * 64);
-            } else {
-              tma_load_2d(sa, wm, full_bar(stage), kb * 64, wrow0);
-            }
+            load_weight_swap(sa, full_bar(stage), wtile, kb);
             tma_load_2d(sb, &tmAct, full_bar(stage), kb * 64, 0);
           } else {
             tma_load_2d(sa, &tmAct, full_bar(stage), kb * 64, m0);
