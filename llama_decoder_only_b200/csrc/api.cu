@@ -252,6 +252,27 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same for a kernel whose CTAs run in 2-CTA clusters (tcgen05 CTA pairs); grid.x is even.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------------ validation
 
 llama_status check_dims(const llama_dims* d) {
@@ -349,7 +370,7 @@ struct WSeg {
 template <int BN, bool SWAP, int EPI>
 llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
                             cudaStream_t st, int kind) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, !SWAP>;
   static bool attr_set = false;
   if (!attr_set) {
     CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -358,7 +379,11 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
   }
   {
     TRACE(kind, st);
-    CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
+    if (SWAP)
+      CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
+    else
+      CUDA_TRY(launch_k_pair(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2],
+                             p));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -383,6 +408,8 @@ llama_status launch_gemm_sk(int epi, const CUtensorMap& a, const CUtensorMap* w,
 }
 
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
+// Each 256 x 256 output tile runs on a CTA pair: every CTA loads 128 activation
+// rows and 128 weight rows per k-block.
 llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
                           void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind) {
   constexpr int BN = 256;
@@ -390,7 +417,7 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
   p.K = K;
   p.num_kb = cdiv(K, 64);
   p.act_rows = M;
-  p.m_tiles = cdiv(M, 128);
+  p.m_tiles = cdiv(M, 256);
   p.nseg = nseg;
   p.out = out;
   p.ldo = ldo;
@@ -420,14 +447,14 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
       p.seg_col0[s] = segs[s].col0;
       p.seg_tile0[s] = t;
       t += cdiv(segs[s].rows, BN);
-      if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, BN)) return LLAMA_ERR_CUDA;
+      if (!make_map_2d(&tw[s], segs[s].ptr, K, segs[s].rows, BN / 2)) return LLAMA_ERR_CUDA;
     }
     for (int s = nseg; s < 3; ++s) tw[s] = tw[0];
     for (int s = nseg; s < 4; ++s) p.seg_tile0[s] = t;
     p.n_tiles = t;
   }
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = std::min(tiles, num_sms());
+  const int grid = 2 * std::min(tiles, num_sms() / 2);
   switch (epi) {
     case EPI_BF16:
       return launch_gemm_tc<BN, false, EPI_BF16>(ta, tw, p, grid, st, kind);

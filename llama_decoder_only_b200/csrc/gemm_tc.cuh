@@ -2,7 +2,7 @@
 //
 // C = A · B^T with A [rows, K] and B [n, K] both K-major bf16, fp32
 // accumulation in TMEM ([DeepDive] LLaMAAttention / LLaMAMLP: every Linear is
-// y = x W^T with W [out, in]).  One CTA per SM, 6 warps:
+// y = x W^T with W [out, in]).  One CTA per SM, 10 warps:
 //   warp 0      TMA producer (one elected lane): A and B tiles into a ring of
 //               STAGES shared-memory stages, 128-byte swizzle, no multicast;
 //   warp 1      TMEM allocator and MMA issuer (one lane): 4 x tcgen05.mma
@@ -16,8 +16,13 @@
 //
 // Two schedules:
 //  * tile mode (prefill, SWAP = false): A = activations (tokens x K),
-//    B = weight rows; persistent CTAs walk the (m-tile, n-tile) grid with the
-//    m index fastest so concurrently running CTAs share weight tiles in L2.
+//    B = weight rows.  A 2-CTA cluster (the two SMs of a TPC) computes one
+//    256 x 256 tile with tcgen05 cta_group::2 MMAs (M = 256): each CTA loads
+//    its 128 activation rows and half of the 256 weight rows per k-block and
+//    holds its 128 x 256 half of the accumulator, so a CTA moves 32 KB instead
+//    of 48 KB from L2 per k-block.  Persistent pairs walk the (m-tile, n-tile)
+//    grid with the m index fastest so concurrently running pairs share weight
+//    tiles in L2.
 //    Epilogues: bf16 store (QKV), fp32 residual add (o_proj, down), paired
 //    SiLU(gate)·up with gate rows and up rows loaded into the two halves of
 //    one B tile (gate_up), fp32 store (lm_head).
@@ -68,11 +73,13 @@ struct GemmParams {
 constexpr int GEMM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 
-template <int BN>
+// PAIR: tile mode on a CTA pair (M = 256 per MMA); this CTA holds 128 rows of
+// A and BN / 2 rows of B per stage.
+template <int BN, bool PAIR>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
@@ -89,8 +96,8 @@ struct GemmItem {
 };
 
 struct GemmIter {
-  // tile mode
-  int next_tile, tile_count;
+  // tile mode: one tile per CTA pair (cluster) at a time
+  int next_tile, tile_count, tile_stride;
   // stream-K mode: this CTA's unit range [u0, u1), walked from the top
   long long u, u0;
   int num_kb;
@@ -100,7 +107,8 @@ struct GemmIter {
     streamk = sk;
     num_kb = p.num_kb;
     if (!sk) {
-      next_tile = blockIdx.x;
+      next_tile = blockIdx.x >> 1;
+      tile_stride = gridDim.x >> 1;
       tile_count = p.m_tiles * p.n_tiles;
     } else {
       const long long G = gridDim.x;
@@ -114,7 +122,7 @@ struct GemmIter {
       it.tile = next_tile;
       it.kb0 = 0;
       it.kb1 = num_kb;
-      next_tile += gridDim.x;
+      next_tile += tile_stride;
       return true;
     }
     if (u <= u0) return false;
@@ -140,7 +148,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW0,
                    const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                    const GemmParams p) {
-  using C = GemmCfg<BN>;
+  constexpr bool PAIR = !SWAP;            // tile mode runs 256 x BN tiles on CTA pairs
+  using C = GemmCfg<BN, PAIR>;
   constexpr int STAGES = C::STAGES;
   constexpr int WROWS = SWAP ? 128 : BN;  // weight rows per tile
   extern __shared__ uint8_t smem_raw[];
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0: issues the pair's MMAs
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -168,7 +178,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 32 * GEMM_EPI_WARPS);
+      // pair: one arrival per epilogue warp of both CTAs (on rank 0's barrier)
+      mbar_init(acce_bar(b), PAIR ? 2 * GEMM_EPI_WARPS : 32 * GEMM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
     mbar_init(epi_bar, 32 * GEMM_EPI_WARPS);
@@ -181,11 +192,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (p.nseg > 2) tma_prefetch_desc(&tmW2);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_base_sh), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&tmem_base_sh), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&tmem_base_sh), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // pair: the peer's TMA loads and the leader's commits target barriers of the
+  // other CTA, so both must be initialised before either proceeds
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   // stream-K (decode): the producer starts the weight stream before its PDL wait
   if (!(SWAP && warp == 0)) pdl_wait();
@@ -246,10 +264,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           wtile = item.tile;
         } else {
           wtile = item.tile / p.m_tiles;
-          m0 = (item.tile % p.m_tiles) * 128;
+          m0 = (item.tile % p.m_tiles) * 256 + 128 * (int)rank;
         }
         const int seg = seg_of_tile(p, wtile);
-        const int wrow0 = (wtile - p.seg_tile0[seg]) * WROWS;
+        const int wrow0 = (wtile - p.seg_tile0[seg]) * WROWS + (PAIR ? (BN / 2) * (int)rank : 0);
         const CUtensorMap* wm = seg == 0 ? &tmW0 : (seg == 1 ? &tmW1 : &tmW2);
         for (int kb = item.kb0; kb < item.kb1; ++kb) {
           if (skip > 0) {
@@ -262,19 +280,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
-          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
           if (SWAP) {
+            mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
             load_weight_swap(sa, full_bar(stage), wtile, kb);
             tma_load_2d(sb, &tmAct, full_bar(stage), kb * 64, 0);
           } else {
-            tma_load_2d(sa, &tmAct, full_bar(stage), kb * 64, m0);
+            // both CTAs' bytes land on rank 0's full barrier, which rank 0 arms
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+            const uint32_t lbar = mapa_shared(full_bar(stage), 0);
+            tma_load_2d_pair(sa, &tmAct, lbar, kb * 64, m0);
             if (EPI == EPI_SWIGLU_BF16) {
-              // gate rows into the first half of the B tile, up rows into the second
-              const int r0 = (wtile)*(BN / 2);
-              tma_load_2d(sb, &tmW0, full_bar(stage), kb * 64, r0);
-              tma_load_2d(sb + (BN / 2) * 128, &tmW1, full_bar(stage), kb * 64, r0);
+              // B columns 0..BN/2-1 (rank 0) are gate rows, BN/2..BN-1 (rank 1) the matching up rows
+              tma_load_2d_pair(sb, rank == 0 ? &tmW0 : &tmW1, lbar, kb * 64, wtile * (BN / 2));
             } else {
-              tma_load_2d(sb, wm, full_bar(stage), kb * 64, wrow0);
+              tma_load_2d_pair(sb, wm, lbar, kb * 64, wrow0);
             }
           }
           filled_parity[stage] = (int)phase;
@@ -285,13 +304,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
       // drain: every issued fill must have landed before the CTA may exit
-      for (int s = 0; s < STAGES; ++s)
-        if (filled_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)filled_parity[s], wc, 9, false);
+      // (pair: rank 0's full barriers count both CTAs' loads; rank 1 leaves
+      // only after the closing cluster barrier, which rank 0 reaches after this)
+      if (!PAIR || rank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (filled_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)filled_parity[s], wc, 9, false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, 0, 0);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(PAIR ? 256 : 128, BN, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       int abuf = 0;
@@ -317,23 +339,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = smem_desc_sw128(sa + k * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(sb + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb > item.kb0 || k > 0) ? 1u : 0u);
+            if constexpr (PAIR)
+              umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > item.kb0 || k > 0) ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, ad, bd, IDESC, (kb > item.kb0 || k > 0) ? 1u : 0u);
           }
           issued = true;
-          umma_commit(empty_bar(stage));
+          if constexpr (PAIR) umma_commit_pair(empty_bar(stage), 3); else umma_commit(empty_bar(stage));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(accf_bar(abuf));
+        if constexpr (PAIR) umma_commit_pair(accf_bar(abuf), 3); else umma_commit(accf_bar(abuf));
         if (++abuf == 2) {
           abuf = 0;
           aphase ^= 1u;
         }
       }
-      if (issued) {
+      if constexpr (PAIR) {
+        // always (also with nothing issued): rank 1 waits on its copy before
+        // it releases TMEM and leaves
+        umma_commit_pair(drain_bar, 3);
+        mbar_wait(drain_bar, 0, wc, 8, false);
+      } else if (issued) {
         // all MMAs of this thread complete before TMEM is released
         umma_commit(drain_bar);
         mbar_wait(drain_bar, 0, wc, 8, false);
@@ -494,7 +524,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       } else {
         const int wtile = item.tile / p.m_tiles;
-        const int m = (item.tile % p.m_tiles) * 128 + row;
+        const int m = (item.tile % p.m_tiles) * 256 + 128 * (int)rank + row;
         const bool row_ok = m < p.act_rows;
 
         if (EPI == EPI_SWIGLU_BF16) {
@@ -584,7 +614,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(acce_bar(abuf));
+      if constexpr (PAIR) {
+        __syncwarp();   // every lane's TMEM reads are complete (waited above)
+        if (lane == 0) mbar_arrive_remote(mapa_shared(acce_bar(abuf), 0));
+      } else {
+        mbar_arrive(acce_bar(abuf));
+      }
       if (++abuf == 2) {
         abuf = 0;
         aphase ^= 1u;
@@ -594,9 +629,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   pdl_trigger();   // the next kernel may start its prologue while this CTA tears down
   tc_fence_before();
-  __syncthreads();
+  // pair: neither CTA leaves while the other may still use its shared memory
+  // (rank 0's MMAs read rank 1's stages; rank 1's epilogue arrives on rank 0)
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      // rank 0's MMAs also wrote this CTA's TMEM
+      bool drained = true;
+      if (lane == 0) drained = mbar_wait(drain_bar, 0, wc, 8, false);
+      (void)drained;
+      __syncwarp();
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    } else {
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+  }
 }
 
 }  // namespace llama
