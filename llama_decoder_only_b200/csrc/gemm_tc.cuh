@@ -6,7 +6,8 @@
 //   warp 0      TMA producer (one elected lane): A and B tiles into a ring of
 //               STAGES shared-memory stages, 128-byte swizzle, no multicast;
 //   warp 1      TMEM allocator and MMA issuer (one lane): 4 x tcgen05.mma
-//               (M=128, N=BN, K=16) per 64-wide k-block, commit frees the stage;
+//               (M=128, or 256 on a CTA pair; N=BN, K=16) per 64-wide
+//               k-block, commit frees the stage;
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
 //               output row per thread; two warps per lane quadrant, each
 //               taking half of the tile's columns), fused epilogue, global
@@ -21,8 +22,9 @@
 //    its 128 activation rows and half of the 256 weight rows per k-block and
 //    holds its 128 x 256 half of the accumulator, so a CTA moves 32 KB instead
 //    of 48 KB from L2 per k-block.  Persistent pairs walk the (m-tile, n-tile)
-//    grid with the m index fastest so concurrently running pairs share weight
-//    tiles in L2.
+//    grid with the m index fastest inside groups of 8 m-tiles, so pairs that
+//    run at the same time share weight tiles and at most 2048 activation rows
+//    in L2.
 //    Epilogues: bf16 store (QKV), fp32 residual add (o_proj, down), paired
 //    SiLU(gate)·up with gate rows and up rows loaded into the two halves of
 //    one B tile (gate_up), fp32 store (lm_head).
@@ -135,6 +137,18 @@ struct GemmIter {
     return true;
   }
 };
+
+// Tile mode: tile index -> (m-tile, weight tile); m runs fastest inside
+// groups of up to 8 m-tiles (the last group may be smaller).
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& mt, int& wt) {
+  constexpr int GM = 8;
+  const int per_group = GM * p.n_tiles;
+  const int g = tile / per_group;
+  const int gm = min(GM, p.m_tiles - g * GM);
+  const int r = tile - g * per_group;
+  wt = r / gm;
+  mt = g * GM + r % gm;
+}
 
 __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
   int s = 0;
@@ -263,8 +277,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (SWAP) {
           wtile = item.tile;
         } else {
-          wtile = item.tile / p.m_tiles;
-          m0 = (item.tile % p.m_tiles) * 256 + 128 * (int)rank;
+          int mt;
+          tile_coords(p, item.tile, mt, wtile);
+          m0 = mt * 256 + 128 * (int)rank;
         }
         const int seg = seg_of_tile(p, wtile);
         const int wrow0 = (wtile - p.seg_tile0[seg]) * WROWS + (PAIR ? (BN / 2) * (int)rank : 0);
@@ -388,6 +403,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     it.init(p, SWAP);
     GemmItem item;
     while (it.next(item)) {
+      if constexpr (PAIR && EPI == EPI_RESID_F32) {
+        // While this tile's MMAs run, pull this thread's residual row segment
+        // (half of the tile's columns, 4 x 128 B of fp32) into L2, so that the
+        // epilogue -- exposed for a CTA's last tile -- does not wait on DRAM.
+        int mt, wt;
+        tile_coords(p, item.tile, mt, wt);
+        const int m = mt * 256 + 128 * (int)rank + row;
+        const int sg = seg_of_tile(p, wt);
+        const int nl = (wt - p.seg_tile0[sg]) * BN + half * (BN / 2);
+        if (m < p.act_rows && nl < p.seg_rows[sg]) {
+          const float* r = p.resid + (size_t)m * p.ldr + p.seg_col0[sg] + nl;
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q)
+            if (nl + 32 * q < p.seg_rows[sg]) asm volatile("prefetch.global.L2 [%0];" ::"l"(r + 32 * q));
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(accf_bar(abuf), aphase, wc, 4))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(abuf * BN);
@@ -523,8 +554,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       } else {
-        const int wtile = item.tile / p.m_tiles;
-        const int m = (item.tile % p.m_tiles) * 256 + 128 * (int)rank + row;
+        int mt, wtile;
+        tile_coords(p, item.tile, mt, wtile);
+        const int m = mt * 256 + 128 * (int)rank + row;
         const bool row_ok = m < p.act_rows;
 
         if (EPI == EPI_SWIGLU_BF16) {
