@@ -143,7 +143,11 @@ size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_l
 
 /* Byte offsets, inside the workspace of a layer call with (batch, seq_len),
  * of the intermediate tensors the call leaves behind, for inspection:
- *   out[0] qkv   [tokens, (nh + 2 nkv) hd] dtype: q (after RoPE), k (before RoPE), v
+ *   out[0] qkv   [tokens, (nh + 2 nkv) hd] dtype: its q columns hold q after RoPE.
+ *                The k and v columns are scratch: in bf16 prefill with head_dim
+ *                64 or 128 the projection writes k and v straight into the cache;
+ *                elsewhere they hold k before RoPE and v.  Read the appended k
+ *                and v from the cache.
  *   out[1] h     [tokens, dim] dtype: the second RMSNorm's output
  *   out[2] attn  [tokens, nh hd] dtype: attention output (heads concatenated)
  *   out[3] m     [tokens, ffn_dim] dtype: silu(gate) * up

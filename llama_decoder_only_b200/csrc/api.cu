@@ -317,7 +317,7 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // ------------------------------------------------------------------ workspace layout
 
 struct WsLayout {
-  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o;   // layer scratch
+  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab;   // layer scratch
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
@@ -348,6 +348,9 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   w.sk_flags = take(sk ? (size_t)kMaxSkGrid * 4 : 0);
   w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
   w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
+  // per-token cos/sin for the prefill QKV GEMM with RoPE fused in
+  const bool rope_fused = d.dtype == LLAMA_BF16 && (d.head_dim == 64 || d.head_dim == 128);
+  w.rope_tab = take(rope_fused ? M * (size_t)d.head_dim * 4 : 0);
   if (vocab > 0) {
     w.xa = take(M * (size_t)d.dim * 4);
     w.xb = take(M * (size_t)d.dim * 4);
@@ -407,11 +410,20 @@ llama_status launch_gemm_sk(int epi, const CUtensorMap& a, const CUtensorMap* w,
   return LLAMA_ERR_INVALID_ARG;
 }
 
+// RoPE + KV append fused into the prefill QKV GEMM (EPI_QKV_ROPE_BF16).
+struct RopeArgs {
+  void* kc;
+  void* vc;
+  const float* tab;   // per-token cos/sin, written by the first RMSNorm
+  int L, p0, nh, nkv, hd, cap, style;
+};
+
 // Tile-mode (prefill) GEMM: out = epi(act[M, K] · W^T), W given as segments.
 // Each 256 x 256 output tile runs on a CTA pair: every CTA loads 128 activation
 // rows and 128 weight rows per k-block.
 llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
-                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind) {
+                          void* out, int ldo, const float* resid, int ldr, DevStatus* status, int kind,
+                          const RopeArgs* rope = nullptr) {
   constexpr int BN = 256;
   GemmParams p{};
   p.K = K;
@@ -425,6 +437,19 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
   p.ldr = ldr;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
+  if (epi == EPI_QKV_ROPE_BF16) {
+    if (rope == nullptr || (rope->hd != 64 && rope->hd != 128)) return LLAMA_ERR_INVALID_ARG;
+    p.kc = rope->kc;
+    p.vc = rope->vc;
+    p.rope_tab = rope->tab;
+    p.L = rope->L;
+    p.p0 = rope->p0;
+    p.nh = rope->nh;
+    p.nkv = rope->nkv;
+    p.hd = rope->hd;
+    p.cap = rope->cap;
+    p.rope_style = rope->style;
+  }
   CUtensorMap ta, tw[3];
   std::memset(tw, 0, sizeof(tw));
   if (!make_map_2d(&ta, act, K, M, 128)) return LLAMA_ERR_CUDA;
@@ -464,6 +489,8 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
       return launch_gemm_tc<BN, false, EPI_SWIGLU_BF16>(ta, tw, p, grid, st, kind);
     case EPI_F32:
       return launch_gemm_tc<BN, false, EPI_F32>(ta, tw, p, grid, st, kind);
+    case EPI_QKV_ROPE_BF16:
+      return launch_gemm_tc<BN, false, EPI_QKV_ROPE_BF16>(ta, tw, p, grid, st, kind);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -731,11 +758,17 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     bf* h = reinterpret_cast<bf*>(ws + lay.h);
     bf* att = reinterpret_cast<bf*>(ws + lay.attn);
     bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
+    // prefill with head_dim 64 / 128: RoPE and the cache append run in the QKV GEMM's epilogue
+    const bool fuse_rope = !decode && (hd == 64 || hd == 128);
+    float* rtab = reinterpret_cast<float*>(ws + lay.rope_tab);
     const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
     // a2: RMSNorm-1 -> h (bf16)
     {
       TRACE(K_RMSNORM, st);
-      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps));
+      // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
+      const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta};
+      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
+                        d.eps, rt));
     }
     LAUNCH_CHECK();
     // a3: QKV projection
@@ -751,14 +784,22 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
-    TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
-    // a4: RoPE + KV append
-    {
-      TRACE(K_ROPE_APPEND, st);
-      CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k), reinterpret_cast<bf*>(kv->v), L,
-                                                 p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style));
+    if (fuse_rope) {
+      // a3 + a4 in one kernel: rotated q -> qkv, rotated k and v -> the cache
+      const RopeArgs ra{kv->k, kv->v, rtab, L, p0, nh, nkv, hd, kv->capacity, d.rope_style};
+      TRY(gemm_prefill(st, h, M, d.dim, segs, nseg, EPI_QKV_ROPE_BF16, qkv, qkvn, nullptr, 0, status, K_GEMM_QKV,
+                       &ra));
+    } else {
+      TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
+      // a4: RoPE + KV append
+      {
+        TRACE(K_ROPE_APPEND, st);
+        CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
+                          reinterpret_cast<bf*>(kv->v), L, p0, nh, nkv, hd, kv->capacity, d.rope_theta,
+                          d.rope_style));
+      }
+      LAUNCH_CHECK();
     }
-    LAUNCH_CHECK();
     // a5 / a6: attention
     if (decode) {
       TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
@@ -774,7 +815,8 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // a8: RMSNorm-2 + gate_up + SiLU·mul
     {
       TRACE(K_RMSNORM, st);
-      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps));
+      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim,
+                        d.eps, RopeTab{}));
     }
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
@@ -795,7 +837,8 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     auto grid_for = [](int M_, int N_) { return dim3(cdiv(N_, 64), cdiv(M_, 64)); };
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_in, d.dim, w.attn_norm, h, M, d.dim, d.eps,
+                                                                   RopeTab{});
     }
     {
       TRACE(K_GEMM_F32, st);
@@ -840,7 +883,8 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     LAUNCH_CHECK();
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps);
+      rmsnorm_kernel<float><<<M, rmsnorm_threads(d.dim), 0, st>>>(x_out, d.dim, w.ffn_norm, h, M, d.dim, d.eps,
+                                                                    RopeTab{});
     }
     {
       TRACE(K_GEMM_F32, st);
@@ -1080,8 +1124,8 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
     {
       TRACE(K_RMSNORM, st);
-      CUDA_TRY(launch_k(rmsnorm_kernel<__nv_bfloat16>, batch, rmsnorm_threads(d.dim), 0, st, xl, d.dim, m->final_norm, hl, batch, d.dim,
-                                                                     d.eps));
+      CUDA_TRY(launch_k(rmsnorm_kernel<__nv_bfloat16>, batch, rmsnorm_threads(d.dim), 0, st, xl, d.dim,
+                        m->final_norm, hl, batch, d.dim, d.eps, RopeTab{}));
     }
     LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};
@@ -1092,7 +1136,8 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     float* hl = reinterpret_cast<float*>(ws + lay.hl);
     {
       TRACE(K_RMSNORM, st);
-      rmsnorm_kernel<float><<<batch, rmsnorm_threads(d.dim), 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim, d.eps);
+      rmsnorm_kernel<float><<<batch, rmsnorm_threads(d.dim), 0, st>>>(xl, d.dim, m->final_norm, hl, batch, d.dim,
+                                                                      d.eps, RopeTab{});
     }
     {
       TRACE(K_GEMM_LM_HEAD, st);

@@ -47,7 +47,11 @@
 
 namespace llama {
 
-enum GemmEpi : int { EPI_BF16 = 0, EPI_RESID_F32 = 1, EPI_SWIGLU_BF16 = 2, EPI_F32 = 3 };
+// EPI_QKV_ROPE_BF16 (tile mode, head_dim 64 or 128): the QKV projection with
+// RoPE and the KV-cache append fused in ([DeepDive] apply_rotary_emb; [MLX-13B]
+// RoPE(traditional=True) and the cache concatenation): rotated q -> out,
+// rotated k and v -> the cache at position p0 + t.
+enum GemmEpi : int { EPI_BF16 = 0, EPI_RESID_F32 = 1, EPI_SWIGLU_BF16 = 2, EPI_F32 = 3, EPI_QKV_ROPE_BF16 = 4 };
 
 struct GemmParams {
   int K;
@@ -64,6 +68,11 @@ struct GemmParams {
   int ldo;
   const float* resid;
   int ldr;
+  // EPI_QKV_ROPE_BF16: tokens m = b * L + t sit at position p0 + t
+  void* kc;                // bf16 cache [batch][nkv][cap][hd]
+  void* vc;
+  const float* rope_tab;   // [M][hd]: cos of the token's hd/2 angles, then sin
+  int L, p0, nh, nkv, hd, cap, rope_style;
   // stream-K mode
   float* partial;      // [grid][128 rows][BN tokens] fp32: each CTA's one non-final piece
   unsigned* flags;     // [grid]: 1 while that CTA's partial waits for its finisher, else 0
@@ -559,7 +568,96 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int m = mt * 256 + 128 * (int)rank + row;
         const bool row_ok = m < p.act_rows;
 
-        if (EPI == EPI_SWIGLU_BF16) {
+        if constexpr (EPI == EPI_QKV_ROPE_BF16) {
+          const int seg = seg_of_tile(p, wtile);
+          const int nl0 = (wtile - p.seg_tile0[seg]) * BN + half * (BN / 2);   // this warp's first row in the segment
+          const int nlim = p.seg_rows[seg];
+          const int n0 = p.seg_col0[seg] + nl0;                                // its first qkv column
+          const int hd = p.hd, nq = p.nh * hd, nk = p.nkv * hd;
+          const int bseq = row_ok ? m / p.L : 0;
+          const int pos = p.p0 + (m - bseq * p.L);
+          const bool halfstyle = p.rope_style == 0;
+          // this token's angles, computed once per token by the first RMSNorm
+          const float* cst = p.rope_tab + (size_t)(row_ok ? m : 0) * hd;
+          const float* snt = cst + hd / 2;
+          auto load16 = [](const float* src, float* dst) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 t = __ldg(reinterpret_cast<const float4*>(src) + q);
+              dst[4 * q] = t.x;
+              dst[4 * q + 1] = t.y;
+              dst[4 * q + 2] = t.z;
+              dst[4 * q + 3] = t.w;
+            }
+          };
+          auto rot = [](float c, float s, float& x0, float& x1) {
+            const float y0 = x0 * c - x1 * s, y1 = x1 * c + x0 * s;
+            x0 = y0;
+            x1 = y1;
+          };
+          // destination of the 32 columns starting at qkv column n (inside one head)
+          auto dst = [&](int n) -> __nv_bfloat16* {
+            if (n < nq) return reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.ldo + n;
+            const bool is_k = n < nq + nk;
+            const int r = is_k ? n - nq : n - nq - nk;
+            __nv_bfloat16* c = reinterpret_cast<__nv_bfloat16*>(is_k ? p.kc : p.vc);
+            return c + (((size_t)bseq * p.nkv + r / hd) * p.cap + pos) * hd + r % hd;
+          };
+          auto store32 = [&](__nv_bfloat16* o, const float (&v)[32]) {
+            uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 w;
+              w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+              w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+              w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+              w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+              o4[q] = w;
+            }
+          };
+          // Two passes over two 32-column chunks (a, b) of this warp's 128 columns.
+          // Rotate-half pairs column d with d + hd/2: hd 128 -> (0, 64), (32, 96);
+          // hd 64 -> (0, 32), (64, 96).  Interleaved pairs and v stay in a chunk.
+#pragma unroll 1
+          for (int pass = 0; pass < 2; ++pass) {
+            const int ca = (halfstyle && hd == 128) ? 32 * pass : 64 * pass;
+            const int cb = (halfstyle && hd == 128) ? ca + 64 : ca + 32;
+            float va[32], vb[32];
+            tmem_ld32(tbase + half * (BN / 2) + ca, va);
+            tmem_ld32(tbase + half * (BN / 2) + cb, vb);
+            tmem_ld_wait();
+            if (!row_ok || nl0 + ca >= nlim) continue;   // segments end on 32-column boundaries
+            const int na = n0 + ca, nb = n0 + cb;
+            const bool b_ok = nl0 + cb < nlim;
+            if (na < nq + nk) {   // q or k: rotate
+              const int da = na % hd;
+              float cs[32], sn[32];
+              if (halfstyle) {
+                // pair i = da + j: (va[j], vb[j])
+                load16(cst + da, cs);
+                load16(cst + da + 16, cs + 16);
+                load16(snt + da, sn);
+                load16(snt + da + 16, sn + 16);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) rot(cs[j], sn[j], va[j], vb[j]);
+              } else {
+                // pairs (2i, 2i+1) inside each chunk: i = da/2 + j and db/2 + j
+                const int db = nb % hd;
+                load16(cst + da / 2, cs);
+                load16(cst + db / 2, cs + 16);
+                load16(snt + da / 2, sn);
+                load16(snt + db / 2, sn + 16);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  rot(cs[j], sn[j], va[2 * j], va[2 * j + 1]);
+                  rot(cs[16 + j], sn[16 + j], vb[2 * j], vb[2 * j + 1]);
+                }
+              }
+            }
+            store32(dst(na), va);
+            if (b_ok) store32(dst(nb), vb);
+          }
+        } else if (EPI == EPI_SWIGLU_BF16) {
           const int n0 = wtile * (BN / 2);
           const int nlim = p.seg_rows[0];
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.ldo;

@@ -33,14 +33,39 @@ inline int rmsnorm_threads(int dim) {
   return t < 32 ? 32 : (t > 1024 ? 1024 : t);
 }
 
+// The RoPE angle of pair i at position pos, p * theta^(-2i/hd) ([DeepDive]
+// LLaMARoPE), is formed and reduced modulo 2*pi in fp64; sincosf evaluates the
+// reduced angle.  Shared by the stand-alone RoPE kernel and the per-token
+// table the first RMSNorm writes for the fused QKV + RoPE GEMM epilogue.
+__device__ __forceinline__ void rope_cos_sin(int pos, int i, int hd, float theta, float& c, float& s) {
+  const double inv = pow((double)theta, -2.0 * (double)i / (double)hd);
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = (double)pos * inv;
+  a -= two_pi * floor(a / two_pi);
+  sincosf((float)a, &s, &c);
+}
+
+// Optional second output of an RMSNorm: per token row r (position p0 + r % L),
+// tab[r * hd + i] = cos and tab[r * hd + hd/2 + i] = sin of pair i's angle.
+struct RopeTab {
+  float* tab;   // nullptr: none
+  int hd, L, p0;
+  float theta;
+};
+
 template <typename OutT>
 __global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__ x, long long x_row_stride,
                                                        const float* __restrict__ g, OutT* __restrict__ h, int rows,
-                                                       int dim, float eps) {
+                                                       int dim, float eps, RopeTab rt) {
   __shared__ float red[32];
   pdl_wait();
   const int row = blockIdx.x;
   if (row >= rows) return;
+  if (rt.tab != nullptr) {
+    const int pos = rt.p0 + row % rt.L, hh = rt.hd >> 1;
+    float* tr = rt.tab + (size_t)row * rt.hd;
+    for (int i = threadIdx.x; i < hh; i += blockDim.x) rope_cos_sin(pos, i, rt.hd, rt.theta, tr[i], tr[hh + i]);
+  }
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * x_row_stride);
   const float4* g4 = reinterpret_cast<const float4*>(g);
   const int n4 = dim >> 2;
@@ -105,16 +130,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T
   const int t = m % L;
   const int p = p0 + t;
   const int half = hd >> 1;
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double inv = pow((double)theta, -2.0 * (double)i / (double)hd);
-    const double two_pi = 6.283185307179586476925286766559;
-    double a = (double)p * inv;
-    a -= two_pi * floor(a / two_pi);
-    float s, c;
-    sincosf((float)a, &s, &c);
-    cs[i] = c;
-    sn[i] = s;
-  }
+  for (int i = threadIdx.x; i < half; i += blockDim.x) rope_cos_sin(p, i, hd, theta, cs[i], sn[i]);
   __syncthreads();
   pdl_wait();
   const int qkvn = (nh + 2 * nkv) * hd;

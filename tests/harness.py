@@ -92,7 +92,7 @@ class LayerRun:
         return xo.reshape(B, Lq, D).double().cpu().numpy()
 
     def intermediates(self):
-        """q (rotated), v, attn, h2, m of the last call plus the appended k, as float64 numpy."""
+        """q (rotated), attn, h2, m of the last call plus the appended k and v (from the cache), as float64 numpy."""
         torch = self.torch
         w = self.w
         B, Lq = self.batch, self.last_L
@@ -106,12 +106,13 @@ class LayerRun:
             return self.ws[o:o + M * n * es].view(dt).reshape(M, n).double().cpu().numpy()
 
         qkv = view(off[0], qkvn)
-        nq, nk = w.n_heads * w.head_dim, w.n_kv_heads * w.head_dim
+        nq = w.n_heads * w.head_dim
         p0 = self.p0
         kc = self.cache.k[:, :, p0:p0 + Lq].double().cpu().numpy()          # [B, nkv, L, hd]
+        vc = self.cache.v[:, :, p0:p0 + Lq].double().cpu().numpy()
         return {
             "q": qkv[:, :nq].reshape(B, Lq, w.n_heads, w.head_dim),
-            "v": qkv[:, nq + nk:].reshape(B, Lq, w.n_kv_heads, w.head_dim),
+            "v": np.transpose(vc, (0, 2, 1, 3)),
             "k": np.transpose(kc, (0, 2, 1, 3)),
             "attn": view(off[2], nq).reshape(B, Lq, nq),
             "h2": view(off[1], w.dim).reshape(B, Lq, w.dim),
