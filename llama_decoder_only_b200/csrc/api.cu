@@ -597,7 +597,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.out = out;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
-  dim3 grid(p.n_qblocks, d.n_heads, B);
+  dim3 grid(d.n_heads, B, p.n_qblocks);   // heaviest query blocks dispatched first (see the kernel)
   TRACE(K_ATTN_PREFILL, st);
   CUDA_TRY(launch_k(attn_prefill_kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
   LAUNCH_CHECK();

@@ -73,8 +73,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = p.n_qblocks - 1 - blockIdx.x;   // heavy (late) blocks first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // Causal work grows with the query block.  CTAs are dispatched x-fastest, so
+  // with the block index in z every (head, sequence) starts its heaviest
+  // (latest) block in the first wave and the light ones fill in behind.
+  const int qb = p.n_qblocks - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / (p.nh / p.nkv);
   const int hd = p.hd;
   const int nreg = hd > 64 ? 2 : 1;             // 64-column regions per head row
