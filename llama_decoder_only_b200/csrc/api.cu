@@ -112,17 +112,24 @@ struct LaunchScope {
 };
 #define TRACE(kind, stream) LaunchScope _trace_scope_(stream, kind)
 
-#define CUDA_TRY(x)                           \
-  do {                                        \
-    if ((x) != cudaSuccess) {                 \
-      (void)cudaGetLastError();               \
-      return LLAMA_ERR_CUDA;                  \
-    }                                         \
+// (with LLAMA_SYNC_TRACE=1 the failing call and its error are printed)
+#define CUDA_TRY(x)                                                                  \
+  do {                                                                               \
+    const cudaError_t cuda_try_e = (x);                                              \
+    if (cuda_try_e != cudaSuccess) {                                                 \
+      if (sync_trace()) std::fprintf(stderr, "[llama] %s: %s\n", #x, cudaGetErrorString(cuda_try_e)); \
+      (void)cudaGetLastError();                                                      \
+      return LLAMA_ERR_CUDA;                                                         \
+    }                                                                                \
   } while (0)
 
-#define LAUNCH_CHECK()                        \
-  do {                                        \
-    if (cudaGetLastError() != cudaSuccess) return LLAMA_ERR_CUDA; \
+#define LAUNCH_CHECK()                                                               \
+  do {                                                                               \
+    const cudaError_t launch_check_e = cudaGetLastError();                           \
+    if (launch_check_e != cudaSuccess) {                                             \
+      if (sync_trace()) std::fprintf(stderr, "[llama] launch: %s\n", cudaGetErrorString(launch_check_e)); \
+      return LLAMA_ERR_CUDA;                                                         \
+    }                                                                                \
   } while (0)
 
 #define TRY(x)                                \

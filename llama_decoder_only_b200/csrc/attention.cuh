@@ -60,6 +60,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Two 128-row query tiles (t = 0, 1) of one head share every K/V tile.  The
 // MMA warp interleaves S1_j, P0·V_j, S0_{j+1}, P1·V_j, so while one softmax
 // warpgroup turns S_t into P_t the tensor core works on the other tile.
+// One CTA per SM (shared memory).  __launch_bounds__ lets ptxas pick the
+// register split; an explicit cap of 192 or 200 registers failed to launch
+// ("too many resources") at 320 threads.
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnPrefillParams p) {
@@ -251,12 +254,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // raw scores: the scale (> 0) is applied once to the maximum and folded
       // into the exponent below
       const bool need_mask = j * 128 + 127 > pos_min;
-      float mraw = -INFINITY;
+      if (need_mask) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        if (need_mask && (j * 128 + i > pos)) sv[i >> 5][i & 31] = -INFINITY;
-        mraw = fmaxf(mraw, sv[i >> 5][i & 31]);
+        for (int i = 0; i < 128; ++i)
+          if (j * 128 + i > pos) sv[i >> 5][i & 31] = -INFINITY;
       }
+      // four independent running maxima (exact in any order), then combined
+      float mr[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mr[k] = sv[0][k];
+#pragma unroll
+      for (int i = 4; i < 128; ++i) mr[i & 3] = fmaxf(mr[i & 3], sv[i >> 5][i & 31]);
+      const float mraw = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3]));
       const float mx = mraw * p.scale_log2;
       // Move this row's reference maximum only when it grew by more than
       // 2^8; rows that keep theirs use alpha = 1.  The O rescale below is a
@@ -278,7 +287,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       // P = 2^(s - m_used) as bf16 into the swizzled K-major A tile
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
       const float sc = p.scale_log2;
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
 #pragma unroll
       for (int c = 0; c < 16; ++c) {   // 16-byte chunk c holds keys 8c .. 8c+7
         uint32_t w[4];
@@ -287,7 +296,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           const int i0 = 8 * c + 2 * e;
           const float a = ex2_approx(fmaf(sv[i0 >> 5][i0 & 31], sc, -mref));
           const float bb = ex2_approx(fmaf(sv[(i0 + 1) >> 5][(i0 + 1) & 31], sc, -mref));
-          psum += a + bb;
+          ps[e] += a + bb;
           w[e] = pack_bf16x2(a, bb);
         }
         const int region = c >> 3, cc = c & 7;
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         tmem_st_wait();
       }
-      l += psum;
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full(t));
