@@ -703,10 +703,13 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   p.part_ml = part_ml;
   p.part_o = part_o;
   p.out = out;
-  // split the keys so that about 4 CTAs per SM run, with >= 128 keys per split
+  // One CTA per (sequence, KV head) when that alone fills 4 CTAs per SM;
+  // otherwise split the keys for about 8 CTAs per SM, >= 64 keys per split
+  // (more, shorter splits keep more loads in flight; with a long cache and a
+  // full grid, extra splits only add the combine pass)
   const int base = B * d.n_kv_heads;
-  int splits = cdiv(4 * num_sms(), base);
-  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 128))));
+  int splits = base >= 4 * num_sms() ? 1 : cdiv(8 * num_sms(), base);
+  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 64))));
   splits = std::max(std::min(min_splits, cdiv(T, 32)), std::min(splits, max_splits));
   int kps = cdiv(T, splits);
   kps = cdiv(kps, 32) * 32;
