@@ -137,10 +137,13 @@ void llama_kv_cache_destroy(llama_kv_cache* cache);
 /* Bytes of device workspace a layer call with `batch` sequences of up to
  * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
  * The workspace is caller-owned scratch.  Zero-fill it once before its first
- * use (its first 256 bytes hold the device status word, and the decode GEMMs
- * keep per-CTA flags in it that each launch leaves cleared); after that the
- * library keeps it consistent.  After a call that recorded
- * LLAMA_ERR_DEVICE_TIMEOUT, zero-fill it again before reusing it. */
+ * use: a fixed header at its start (the same for every batch and seq_len,
+ * 66,560 bytes) holds the device status word, the decode GEMMs' per-CTA
+ * flags and the decode attention's per-(sequence, KV head) counters, which
+ * every launch leaves at zero; after that the library keeps it consistent,
+ * also when prefill and decode calls of different shapes share it.  After a
+ * call that recorded LLAMA_ERR_DEVICE_TIMEOUT, zero-fill it again before
+ * reusing it. */
 size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_len);
 
 /* Byte offsets, inside the workspace of a layer call with (batch, seq_len),

@@ -12,11 +12,13 @@
 //    overlaps the other tile's MMAs.  The running max is only moved (and
 //    O rescaled) when it grows by more than 2^8, which is exact because the
 //    final division uses the same stale maximum for numerator and sum.
-//  * attn_decode_kernel + attn_decode_combine_kernel: one new query per
-//    sequence; the cache of each (sequence, KV head) is split along the key
-//    axis over several CTAs; the query heads of a GQA group share every K/V
-//    load; partial (max, sum, output) are merged with the usual log-sum-exp
-//    rule.  CUDA-core FMAs, 16-byte loads; bound by HBM bandwidth.
+//  * attn_decode_kernel (and attn_decode_mma_kernel for GQA groups >= 4):
+//    one new query per sequence; the cache of each (sequence, KV head) is
+//    split along the key axis over several CTAs; the query heads of a GQA
+//    group share every K/V load; partial (max, sum, output) are merged with
+//    the usual log-sum-exp rule by the split that finishes last (or by
+//    attn_decode_combine_kernel when the caller has no counter words).
+//    CUDA-core FMAs, 16-byte loads; bound by HBM bandwidth.
 //
 // Definition followed: softmax(q k^T / sqrt(hd)) v over keys j <= p
 // ([MLX-13B] 2. 注意力机制 and 5. 因果掩码; [DeepDive] LLaMAAttention),
@@ -390,8 +392,48 @@ struct AttnDecodeParams {
   float scale_log2;
   float* part_ml;             // [B*nh][splits][2]   (splits > 1)
   float* part_o;              // [B*nh][splits][hd]
+  unsigned* counters;         // [B][nkv], zero between launches; nullptr: a separate combine kernel merges
   __nv_bfloat16* out;         // [B, nh*hd]
 };
+
+// Log-sum-exp merge of the `splits` partial results of query head hq of
+// sequence b (base-2 maxima): out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// Partials are read through L2: other CTAs of the same launch may have written them.
+__device__ __forceinline__ void combine_head(const float* part_ml, const float* part_o, __nv_bfloat16* out, int nh,
+                                             int hd, int splits, int b, int hq) {
+  const size_t r0 = ((size_t)b * nh + hq) * splits;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(part_ml + 2 * (r0 + s)));
+  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < splits; ++s) {
+        const float c = exp2f(__ldcg(part_ml + 2 * (r0 + s)) - M);
+        Lsum += __ldcg(part_ml + 2 * (r0 + s) + 1) * c;
+        O += __ldcg(part_o + (r0 + s) * hd + d) * c;
+      }
+    }
+    out[(size_t)b * nh * hd + (size_t)hq * hd + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+  }
+}
+
+// Split-KV, after every thread of the CTA has written its partials: the CTA
+// that finishes last among the `splits` CTAs of (sequence b, KV head g)
+// merges them for that head's G query heads and re-arms the counter.  The
+// fence-then-count order makes every split's partials visible to it.
+__device__ __forceinline__ void merge_if_last_split(unsigned* counters, const float* part_ml, const float* part_o,
+                                                    __nv_bfloat16* out, int nh, int nkv, int hd, int splits, int b,
+                                                    int g, int G) {
+  __shared__ int last_sh;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_sh = atomicAdd(counters + (size_t)b * nkv + g, 1u) == (unsigned)splits - 1u;
+  __syncthreads();
+  if (!last_sh) return;
+  __threadfence();
+  for (int gi = 0; gi < G; ++gi) combine_head(part_ml, part_o, out, nh, hd, splits, b, g * G + gi);
+  if (threadIdx.x == 0) counters[(size_t)b * nkv + g] = 0u;
+}
 
 template <int HD, int G>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams p) {
@@ -565,6 +607,8 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
       }
     }
   }
+  if (p.splits > 1 && p.counters != nullptr)
+    merge_if_last_split(p.counters, p.part_ml, p.part_o, p.out, p.nh, p.nkv, HD, p.splits, b, g, G);
 }
 
 // ---------------------------------------------------------------------- decode, GQA groups >= 4
@@ -619,6 +663,7 @@ struct AttnDecodeMmaParams {
   float scale_log2;
   float* part_ml;
   float* part_o;
+  unsigned* counters;   // as in AttnDecodeParams
   __nv_bfloat16* out;
   DevStatus* status;
   unsigned long long limit_ns;
@@ -847,27 +892,15 @@ __global__ void __launch_bounds__(160, 1)
       }
     }
   }
+  if (p.splits > 1 && p.counters != nullptr)
+    merge_if_last_split(p.counters, p.part_ml, p.part_o, p.out, p.nh, p.nkv, HD, p.splits, b, g, G);
 }
 
 // out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
                                            __nv_bfloat16* __restrict__ out, int nh, int hd, int splits) {
   pdl_wait();
-  const int h = blockIdx.x, b = blockIdx.y;
-  const size_t r0 = ((size_t)b * nh + h) * splits;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[2 * (r0 + s)]);
-  for (int d = threadIdx.x; d < hd; d += blockDim.x) {
-    float Lsum = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float c = exp2f(part_ml[2 * (r0 + s)] - M);
-        Lsum += part_ml[2 * (r0 + s) + 1] * c;
-        O += part_o[(r0 + s) * hd + d] * c;
-      }
-    }
-    out[(size_t)b * nh * hd + (size_t)h * hd + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
-  }
+  combine_head(part_ml, part_o, out, nh, hd, splits, blockIdx.y, blockIdx.x);
 }
 
 }  // namespace llama
