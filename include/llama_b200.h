@@ -137,10 +137,9 @@ void llama_kv_cache_destroy(llama_kv_cache* cache);
 /* Bytes of device workspace a layer call with `batch` sequences of up to
  * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
  * The workspace is caller-owned scratch.  Zero-fill it once before its first
- * use: a fixed header at its start (the same for every batch and seq_len,
- * 66,560 bytes) holds the device status word, the decode GEMMs' per-CTA
- * flags and the decode attention's per-(sequence, KV head) counters, which
- * every launch leaves at zero; after that the library keeps it consistent,
+ * use: a fixed 1024-byte header at its start (the same for every batch and
+ * seq_len) holds the device status word and the decode GEMMs' per-CTA flags,
+ * which every launch leaves at zero; after that the library keeps it consistent,
  * also when prefill and decode calls of different shapes share it.  After a
  * call that recorded LLAMA_ERR_DEVICE_TIMEOUT, zero-fill it again before
  * reusing it. */

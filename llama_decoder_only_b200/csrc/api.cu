@@ -38,12 +38,10 @@ namespace {
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 constexpr int kMaxSkGrid = 192;     // upper bound on stream-K CTAs (workspace sizing)
 constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
-// workspace header (see plan_ws): status word, GEMM flags, attention counters
+// workspace header (see plan_ws): status word, then the decode GEMMs' flags
 constexpr size_t kWsFlagsOffset = 256;
-constexpr size_t kWsCountersOffset = 1024;
-constexpr int kMaxAttnCounters = 16384;   // (sequence, KV head) pairs merged in-kernel; beyond: combine kernel
-constexpr size_t kWsHeaderBytes = kWsCountersOffset + (size_t)kMaxAttnCounters * 4;
-static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsCountersOffset, "GEMM flags overlap the counters");
+constexpr size_t kWsHeaderBytes = 1024;
+static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsHeaderBytes, "GEMM flags overflow the header");
 constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K form up to here
 
 // ------------------------------------------------------------------ tracing
@@ -330,7 +328,7 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // ------------------------------------------------------------------ workspace layout
 
 struct WsLayout {
-  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, att_cnt, rope_tab;   // layer scratch
+  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab;   // layer scratch
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
@@ -346,12 +344,11 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   const size_t M = (size_t)batch * seq_len;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
   // Fixed header, the same for every (batch, seq_len): the words that must
-  // read zero when a launch starts -- the status word, the decode GEMMs'
-  // per-CTA flags, the decode attention's per-(sequence, KV head) counters.
-  // Every launch leaves them zero; the tensors after the header move with the
-  // call's shape, so one call's data never lands on another call's flags.
+  // read zero when a launch starts -- the status word and the decode GEMMs'
+  // per-CTA flags.  Every launch leaves them zero; the tensors after the
+  // header move with the call's shape, so one call's data never lands on
+  // another call's flags.
   w.sk_flags = kWsFlagsOffset;
-  w.att_cnt = kWsCountersOffset;
   size_t off = kWsHeaderBytes;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -646,8 +643,7 @@ llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv
 // Decode attention for GQA groups of 4 or 8 on the tensor cores.
 llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                              int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
-                             float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits,
-                             unsigned* counters) {
+                             float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   CUtensorMap tk, tv;
   const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)T, (uint64_t)B * d.n_kv_heads};
@@ -664,7 +660,6 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.part_ml = part_ml;
   p.part_o = part_o;
-  p.counters = counters;
   p.out = out;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
@@ -687,7 +682,7 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   }
   if (r != LLAMA_OK) return r;
   LAUNCH_CHECK();
-  if (splits > 1 && counters == nullptr) {   // else the last split of each head merged them
+  if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
     CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
   }
@@ -697,16 +692,14 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
 
 // Decode attention of one new token per sequence over keys [0, T).  Splits of
 // the key range are chosen by a heuristic, clamped to [min_splits, max_splits].
-// With `counters` ([B][nkv] words, zero between launches) the split that
-// finishes last merges each head; without, a combine kernel follows.
 llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                               int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
                               float* part_ml, float* part_o, DevStatus* status, int min_splits = 1,
-                              int max_splits = kMaxAttnSplits, unsigned* counters = nullptr) {
+                              int max_splits = kMaxAttnSplits) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   if (grp >= 4 && (hd == 64 || hd == 128))
     return attn_decode_mma(st, d, kc, vc, capacity, B, T, qkv, ld_qkv, out, part_ml, part_o, status, min_splits,
-                           max_splits, counters);
+                           max_splits);
   AttnDecodeParams p{};
   p.qkv = qkv;
   p.ld_qkv = ld_qkv;
@@ -719,7 +712,6 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.part_ml = part_ml;
   p.part_o = part_o;
-  p.counters = counters;
   p.out = out;
   // One CTA per (sequence, KV head) when that alone fills 4 CTAs per SM;
   // otherwise split the keys for about 8 CTAs per SM, >= 64 keys per split
@@ -745,7 +737,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
 #undef DEC_CASE
   }
   LAUNCH_CHECK();
-  if (splits > 1 && counters == nullptr) {   // else the last split of each head merged them
+  if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
     CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
     LAUNCH_CHECK();
@@ -832,8 +824,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     if (decode) {
       TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
                            reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o),
-                           status, 1, kMaxAttnSplits,
-                           B * nkv <= kMaxAttnCounters ? reinterpret_cast<unsigned*>(ws + lay.att_cnt) : nullptr));
+                           status));
     } else {
       TRY(attn_prefill_bf16(st, d, kv, B, L, p0, qkv, att, status));
     }

@@ -16,8 +16,7 @@
 //    one new query per sequence; the cache of each (sequence, KV head) is
 //    split along the key axis over several CTAs; the query heads of a GQA
 //    group share every K/V load; partial (max, sum, output) are merged with
-//    the usual log-sum-exp rule by the split that finishes last (or by
-//    attn_decode_combine_kernel when the caller has no counter words).
+//    the usual log-sum-exp rule by attn_decode_combine_kernel.
 //    CUDA-core FMAs, 16-byte loads; bound by HBM bandwidth.
 //
 // Definition followed: softmax(q k^T / sqrt(hd)) v over keys j <= p
@@ -392,7 +391,6 @@ struct AttnDecodeParams {
   float scale_log2;
   float* part_ml;             // [B*nh][splits][2]   (splits > 1)
   float* part_o;              // [B*nh][splits][hd]
-  unsigned* counters;         // [B][nkv], zero between launches; nullptr: a separate combine kernel merges
   __nv_bfloat16* out;         // [B, nh*hd]
 };
 
@@ -417,23 +415,6 @@ __device__ __forceinline__ void combine_head(const float* part_ml, const float* 
   }
 }
 
-// Split-KV, after every thread of the CTA has written its partials: the CTA
-// that finishes last among the `splits` CTAs of (sequence b, KV head g)
-// merges them for that head's G query heads and re-arms the counter.  The
-// fence-then-count order makes every split's partials visible to it.
-__device__ __forceinline__ void merge_if_last_split(unsigned* counters, const float* part_ml, const float* part_o,
-                                                    __nv_bfloat16* out, int nh, int nkv, int hd, int splits, int b,
-                                                    int g, int G) {
-  __shared__ int last_sh;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last_sh = atomicAdd(counters + (size_t)b * nkv + g, 1u) == (unsigned)splits - 1u;
-  __syncthreads();
-  if (!last_sh) return;
-  __threadfence();
-  for (int gi = 0; gi < G; ++gi) combine_head(part_ml, part_o, out, nh, hd, splits, b, g * G + gi);
-  if (threadIdx.x == 0) counters[(size_t)b * nkv + g] = 0u;
-}
 
 template <int HD, int G>
 __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams p) {
@@ -607,8 +588,6 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
       }
     }
   }
-  if (p.splits > 1 && p.counters != nullptr)
-    merge_if_last_split(p.counters, p.part_ml, p.part_o, p.out, p.nh, p.nkv, HD, p.splits, b, g, G);
 }
 
 // ---------------------------------------------------------------------- decode, GQA groups >= 4
@@ -663,7 +642,6 @@ struct AttnDecodeMmaParams {
   float scale_log2;
   float* part_ml;
   float* part_o;
-  unsigned* counters;   // as in AttnDecodeParams
   __nv_bfloat16* out;
   DevStatus* status;
   unsigned long long limit_ns;
@@ -892,8 +870,6 @@ __global__ void __launch_bounds__(160, 1)
       }
     }
   }
-  if (p.splits > 1 && p.counters != nullptr)
-    merge_if_last_split(p.counters, p.part_ml, p.part_o, p.out, p.nh, p.nkv, HD, p.splits, b, g, G);
 }
 
 // out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
