@@ -161,6 +161,22 @@ def test_workspace_grows_with_tokens():
     assert all(a < b for a, b in zip(sizes, sizes[1:]))
 
 
+def test_workspace_tensors_start_past_the_fixed_header():
+    """The first 1024 bytes of every workspace (status word, decode-GEMM flags)
+    sit at the same place for every call shape and are never part of a tensor:
+    a prefill call's data must not land on the words a later decode call
+    expects to read zero, whatever the two calls' shapes."""
+    header = 1024
+    for dims in [L.make_dims(4096, 32, 32, 128, 11008, 1e-6, 1e4, "half", "bf16"),
+                 L.make_dims(3072, 32, 32, 96, 8192, 1e-5, 1e4, "half", "bf16"),
+                 L.make_dims(256, 8, 2, 32, 688, 1e-5, 1e4, "half", "f32")]:
+        for batch, seq_len in [(1, 1), (16, 1), (64, 1), (1, 2048), (2, 4096), (8, 512)]:
+            offs = L.workspace_offsets(dims, batch, seq_len)
+            assert min(offs) >= header, (batch, seq_len, offs)
+            assert all(o % 256 == 0 for o in offs)
+            assert L.workspace_size(dims, batch, seq_len) > max(offs)
+
+
 def test_model_call_validation():
     d = dims()
     lib = L.lib()
