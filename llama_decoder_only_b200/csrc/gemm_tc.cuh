@@ -25,15 +25,17 @@
 //    grid with the m index fastest inside groups of 8 m-tiles, so pairs that
 //    run at the same time share weight tiles and at most 2048 activation rows
 //    in L2.
-//    Epilogues: bf16 store (QKV), fp32 residual add (o_proj, down), paired
-//    SiLU(gate)·up with gate rows and up rows loaded into the two halves of
-//    one B tile (gate_up), fp32 store (lm_head).
+//    Epilogues: bf16 store (QKV), QKV with RoPE and the KV-cache append
+//    fused in (head_dim 64/128), fp32 residual add (o_proj, down; the
+//    residual rows are prefetched into L2 during the tile's MMAs), paired
+//    SiLU(gate)·up with the pair's B halves holding gate rows (rank 0) and the
+//    matching up rows (rank 1) (gate_up), fp32 store (lm_head).
 //  * stream-K mode (decode, SWAP = true): the weight is A (its rows fill the
 //    MMA's M = 128) and the few token rows are B (N = BN >= tokens), so the
 //    weight streams from HBM once.  The (weight tile, k-block) units are split
 //    evenly over the CTAs and each CTA walks its range backwards: its only
 //    piece that does not end a tile comes first and is published at once as
-//    an fp32 partial plus an epoch flag; the CTA that holds a tile's last
+//    an fp32 partial plus a flag word; the CTA that holds a tile's last
 //    k-block waits (bounded) for the lower CTAs' partials, adds them in CTA
 //    order (deterministic) and applies the epilogue itself.  For gate_up a
 //    weight tile is 64 gate rows followed by the matching 64 up rows, so
