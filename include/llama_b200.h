@@ -25,7 +25,11 @@
  *   Projection weights, the embedding and lm_head are `dims.dtype`.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream).  All work is enqueued on it; no call synchronises, except
- *   llama_device_status.
+ *   llama_device_status.  Layer and model calls may be captured into a CUDA
+ *   graph (stream capture): they enqueue kernels only.  Positions (the cache
+ *   length when the call is enqueued) are fixed in the captured work, so a
+ *   replay recomputes the step at the captured position; the caller restores
+ *   the cache length (and contents, if it needs them) before replaying.
  * Errors.  Calls return a llama_status and never throw.  Argument checks run
  *   before anything is enqueued; on failure nothing is enqueued and the cache
  *   length is unchanged.  Device-side failures (a bounded wait that ran out)
