@@ -13,6 +13,9 @@ block  -- NumPy float64 definition of every step (norm, projections, RoPE in
           wiring, embedding, final norm, lm_head, greedy argmax).
 brute  -- pure-Python (``math`` only) triple-loop restatement of the same
           block, used to cross-check ``block`` on tiny shapes.
+quant  -- the 4-bit group-64 quantised Linear the pages name (group-wise
+          affine codes, packing, dequantised product), the oracle of the next
+          row of the build; pinned by ``tests/test_oracle_quant.py``.
 
 Parity status: every function in ``block`` is pinned by the CPU tests in
 ``tests/test_oracle_*.py`` (closed forms, invariants, library special cases,
