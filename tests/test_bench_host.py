@@ -65,3 +65,23 @@ def test_reference_arm_prints_one_json_line():
 def test_reference_arm_other_ranks_do_no_work():
     r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "1"], {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_work_accounting_matches_the_hand_counts():
+    """The flop and byte counts behind every roofline figure, against counts
+    made by hand from the layer shapes: 7B-shaped prefill 828.9 GFLOP of
+    GEMMs + 34.4 GFLOP of causal attention per layer; weights per layer
+    634.4 MB (13B shape), 1711.3 MB (70B shape), and 7247.8 MB for the 32
+    Phi-3-shaped layers."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    W = synth.WORKLOADS
+    w7 = W["llama7b_prefill"]
+    assert bench.gemm_flops_per_token(w7) * 2048 == pytest.approx(828.9e9, rel=1e-4)
+    assert bench.attn_prefill_flops(w7, 1, 2048) == pytest.approx(34.37e9, rel=1e-3)
+    # causal pairs: with p0 = 0 the count is L(L+1)/2 per head
+    assert bench.attn_prefill_flops(w7, 1, 4) == 4 * 128 * 32 * 10
+    assert bench.layer_weight_bytes(W["llama13b_decode"]) == pytest.approx(634.4e6, rel=1e-4)
+    assert bench.layer_weight_bytes(W["gqa70b"]) == pytest.approx(1711.3e6, rel=1e-4)
+    assert 32 * bench.layer_weight_bytes(W["phi3mini_model"]) == pytest.approx(7247.8e6, rel=1e-4)
