@@ -203,6 +203,27 @@ def test_selftest_rejects_bad_args():
     assert lib.llama_selftest_wait_timeout(FAKE, 10 ** 10, None) == 1
 
 
+def test_noalloc_attention_validates_before_any_launch():
+    """Every rejection of the allocation-free decode attention happens on the
+    host, before the library touches the device: too large for its fixed
+    scratch (SCRATCH_LIMIT), fp32 dims (UNSUPPORTED), bad sizes (INVALID_ARG),
+    misaligned pointers or ld_q (ALIGNMENT)."""
+    lib = L.lib()
+    d = L.make_dims(8192, 64, 8, 128, 28672, 1e-5, 1e4, "half", "bf16")
+    q, k, v, o = FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30)
+    call = lambda dd, b, qq, ld, kk, vv, cap, n, oo: lib.llama_attention_decode_noalloc(  # noqa: E731
+        ctypes.byref(dd), b, qq, ld, kk, vv, cap, n, oo, None)
+    # 1024 sequences x 64 heads x 130 floats x 2 splits x 4 bytes = 68 MB > 8 MiB
+    assert call(d, 1024, q, 64 * 128, k, v, 4096, 100, o) == 8
+    f32 = L.make_dims(8192, 64, 8, 128, 28672, 1e-5, 1e4, "half", "f32")
+    assert call(f32, 1, q, 64 * 128, k, v, 4096, 100, o) == 2
+    assert call(d, 1, q, 64 * 128, k, v, 100, 101, o) == 1          # length > capacity
+    assert call(d, 1, q, 64 * 128 - 8, k, v, 4096, 100, o) == 1     # ld_q < n_heads * head_dim
+    assert call(d, 1, None, 64 * 128, k, v, 4096, 100, o) == 1
+    assert call(d, 1, q + 8, 64 * 128, k, v, 4096, 100, o) == 4     # misaligned q
+    assert call(d, 1, q, 64 * 128 + 4, k, v, 4096, 100, o) == 4     # ld_q not a multiple of 8
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(L, "_lib", None)
