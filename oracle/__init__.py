@@ -16,6 +16,8 @@ brute  -- pure-Python (``math`` only) triple-loop restatement of the same
 quant  -- the 4-bit group-64 quantised Linear the pages name (group-wise
           affine codes, packing, dequantised product), the oracle of the next
           row of the build; pinned by ``tests/test_oracle_quant.py``.
+sampling -- temperature / top-p (nucleus) sampling after the lm_head, with
+          the uniform draw as an input; pinned by ``tests/test_oracle_sampling.py``.
 
 Parity status: every function in ``block`` is pinned by the CPU tests in
 ``tests/test_oracle_*.py`` (closed forms, invariants, library special cases,
