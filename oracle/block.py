@@ -290,6 +290,20 @@ def final_logits(x_last, g_final, W_lm, eps, rounding=None):
     return h @ np.asarray(W_lm, np.float64).T
 
 
+def layer_forward_ragged(d: Dims, W, xs, caches, rounding=None):
+    """A ragged batch: sequence ``b`` brings ``xs[b]`` of shape ``[L_b, dim]`` at
+    positions ``caches[b].length .. + L_b - 1`` of its own single-sequence cache
+    (decode rows, L_b = 1, and prefill chunks may be mixed).
+
+    The block never mixes sequences: attention runs within one sequence
+    ([DeepDive] LLaMAAttention, per batch row; [MLX-13B] KV 缓存实现片段, one
+    cache per sequence) and the norms, projections and FFN act per token.  So a
+    ragged batch is ``layer_forward`` applied to each sequence with its own
+    offset.  Returns the list of ``[L_b, dim]`` outputs.
+    """
+    return [layer_forward(d, W, np.asarray(x)[None], c, rounding)[0][0] for x, c in zip(xs, caches)]
+
+
 def greedy_argmax(logits):
     """Greedy decoding: index of the largest logit, lowest index on ties.
 

@@ -414,3 +414,31 @@ def test_pin_catches_off_by_one_causal_mask(monkeypatch):
     _planted(monkeypatch, "causal_gqa_attention", wrong)
     with pytest.raises(AssertionError):
         test_block_matches_pure_python_brute_force("half")
+
+
+def test_ragged_batch_matches_batched_and_full_prefill():
+    """Ragged batches (per-sequence offsets and chunk lengths): with equal
+    lengths they equal the batched block; with different ones each
+    sequence's rows equal the matching rows of a one-shot prefill of its
+    whole prefix (a different code path: one call, no chunking)."""
+    d = tiny_dims()
+    W = rand_weights(d, RNG)
+    # equal lengths: per-sequence caches vs one batched cache
+    x = RNG.standard_normal((3, 5, d.dim))
+    batched, _ = ob.layer_forward(d, W, x, ob.KVCache(3, d.n_kv_heads, d.head_dim, 16))
+    rag = ob.layer_forward_ragged(d, W, list(x), [ob.KVCache(1, d.n_kv_heads, d.head_dim, 16) for _ in range(3)])
+    assert np.allclose(np.stack(rag), batched, rtol=0, atol=1e-12)
+    # mixed: sequence 0 decodes its 8th token, sequence 1 prefills 4 tokens after 3 cached, sequence 2 starts fresh
+    prefixes = [RNG.standard_normal((8, d.dim)), RNG.standard_normal((7, d.dim)), RNG.standard_normal((2, d.dim))]
+    cached = [7, 3, 0]
+    caches = []
+    for pre, n in zip(prefixes, cached):
+        c = ob.KVCache(1, d.n_kv_heads, d.head_dim, 16)
+        if n:
+            ob.layer_forward(d, W, pre[None, :n], c)
+        caches.append(c)
+    outs = ob.layer_forward_ragged(d, W, [pre[n:] for pre, n in zip(prefixes, cached)], caches)
+    for pre, n, out in zip(prefixes, cached, outs):
+        full, _ = ob.layer_forward(d, W, pre[None], ob.KVCache(1, d.n_kv_heads, d.head_dim, 16))
+        assert out.shape == (len(pre) - n, d.dim)
+        assert np.allclose(out, full[0, n:], rtol=0, atol=1e-12)
