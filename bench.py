@@ -44,9 +44,10 @@ HEADLINE = "llama7b_prefill"
 METRIC = "prefill & decode tokens/s per layer at 1 B200; % of TC / HBM roofline"
 UNIT = "tokens/s/layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# dram__bytes_read.sum + dram__bytes_write.sum of one gate_up launch of the headline
-# layer, from an ncu capture of the current kernel (None once the kernel changes)
-GATE_UP_TRAFFIC_BYTES = 235.64e6
+# ncu summary of the roofline kernel: its `traffic_bytes_per_launch` line is used
+# only while `source_sha256` matches the kernel sources it was captured from
+ROOFLINE_PROFILE = os.path.join(ROOT, "profiles", "gemm_gate_up_swiglu_llama7b_prefill.md")
+KERNEL_SOURCES = ("llama_decoder_only_b200/csrc/gemm_tc.cuh", "llama_decoder_only_b200/csrc/common.cuh")
 
 
 # ------------------------------------------------------------------ peaks, clocks
@@ -59,6 +60,32 @@ def load_peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha256():
+    """sha256 over the sources of the tensor-core GEMM kernel (gemm_tc.cuh, common.cuh)."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def roofline_traffic():
+    """(bytes per launch or None, note) from the committed ncu summary of the roofline kernel."""
+    try:
+        fields = {}
+        with open(ROOFLINE_PROFILE) as f:
+            for line in f:
+                if ":" in line and line.split(":", 1)[0].strip() in ("traffic_bytes_per_launch", "source_sha256"):
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_sha256") != kernel_source_sha256():
+            return None, "null: the kernel sources changed since the ncu capture"
+        return float(fields["traffic_bytes_per_launch"]), f"ncu capture in {os.path.relpath(ROOFLINE_PROFILE, ROOT)}"
+    except Exception as e:  # missing or unreadable summary
+        return None, f"null: {type(e).__name__}"
 
 
 class ClockSampler:
@@ -112,7 +139,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ distributed plumbing
 
-def dist_init(n_gpus):
+def spawn_ranks(n_gpus, argv):
+    """Re-run this script as ``n_gpus`` ranks (one process per GPU) under
+    torch.distributed.run on this node; returns the launcher's exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    try:
+        return subprocess.run(cmd, timeout=3600).returncode
+    except subprocess.TimeoutExpired:
+        return 124
+
+
+def dist_init(n_gpus, backend="nccl"):
+    """(rank, world, local rank) from the torchrun environment; one GPU per rank."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -121,10 +164,13 @@ def dist_init(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -207,6 +253,13 @@ def attn_prefill_flops(w, B, L, p0=0):
 def layer_weight_bytes(w):
     qkv = (w.n_heads + 2 * w.n_kv_heads) * w.head_dim
     return 2 * w.dim * (qkv + w.n_heads * w.head_dim + 3 * w.ffn_dim)
+
+
+def layer_weight_bytes_q4(w):
+    """Bytes of a layer's seven projections in the 4-bit group-64 form: half a byte
+    per weight plus a bf16 scale and offset per 64 weights."""
+    params = layer_weight_bytes(w) // 2
+    return params // 2 + (params // 64) * 4
 
 
 def bench_prefill_layer(L, torch, w, steps, warmup, world, seed, with_e2e):
@@ -312,12 +365,18 @@ def pipelined_e2e(torch, L, dims, lw, cache, B, S, dim, ws, steps, warmup, world
     return e0.elapsed_time(e1) / 1e3 / steps
 
 
-def bench_decode_layer(L, torch, w, steps, warmup, world, seed):
+def bench_decode_layer(L, torch, w, steps, warmup, world, seed, q4=False):
     from synth import device as sd
     dims = L.make_dims(w.dim, w.n_heads, w.n_kv_heads, w.head_dim, w.ffn_dim, w.eps, w.rope_theta,
                        w.rope_style, w.dtype)
-    dev = sd.random_layer_on_device(w, seed)
-    lw = L.layer_weights(dev)
+    if q4:
+        dev = sd.random_q4_layer_on_device(w, seed)
+        lw = L.layer_weights_q4(dev)
+        layer_call = L.layer_decode_q4
+    else:
+        dev = sd.random_layer_on_device(w, seed)
+        lw = L.layer_weights(dev)
+        layer_call = L.layer_decode
     B, T0, nsteps = w.decode_batch, w.cache_len, w.decode_steps
     cap = T0 + nsteps
     g = torch.Generator(device="cuda")
@@ -334,7 +393,7 @@ def bench_decode_layer(L, torch, w, steps, warmup, world, seed):
         cache.set_length(T0 + (i % nsteps))
 
     def step(i):
-        L.layer_decode(dims, lw, cache, B, xs[i % nsteps], y, ws)
+        layer_call(dims, lw, cache, B, xs[i % nsteps], y, ws)
 
     n0 = L.launch_count()
     t = timed(torch, step, steps, warmup, world, between=pos)
@@ -346,11 +405,11 @@ def bench_decode_layer(L, torch, w, steps, warmup, world, seed):
     kv_bytes = 2 * B * w.n_kv_heads * mean_T * w.head_dim * 2
     return {"tokens_per_step": B, "t_step_s": t / steps, "launches_per_step": launches,
             "kernels": {kk: {"avg_us": 1e3 * ms / n, "launches": n // steps} for kk, (ms, n) in kern.items()},
-            "weight_bytes": layer_weight_bytes(w), "kv_bytes": kv_bytes,
+            "weight_bytes": layer_weight_bytes_q4(w) if q4 else layer_weight_bytes(w), "kv_bytes": kv_bytes,
             "append_bytes": 2 * B * w.n_kv_heads * w.head_dim * 2}
 
 
-def bench_model(L, torch, w, steps, warmup, world, seed):
+def bench_model(L, torch, w, steps, warmup, world, seed, prefill_steps=None):
     from synth import device as sd
     dims = L.make_dims(w.dim, w.n_heads, w.n_kv_heads, w.head_dim, w.ffn_dim, w.eps, w.rope_theta,
                        w.rope_style, w.dtype)
@@ -377,7 +436,8 @@ def bench_model(L, torch, w, steps, warmup, world, seed):
     def prefill(_):
         L.model_forward(model, caches, prompt, B, S, None, ids, ws)
 
-    tp = timed(torch, prefill, max(1, steps // 4), max(1, warmup // 2), world, between=reset_all)
+    n_pre = prefill_steps or max(1, steps // 4)
+    tp = timed(torch, prefill, n_pre, max(3, warmup // 2), world, between=reset_all)
     kp = traced(L, torch, prefill, 1, between=reset_all)
 
     def pos(i):
@@ -391,7 +451,6 @@ def bench_model(L, torch, w, steps, warmup, world, seed):
     kd = traced(L, torch, decode, steps, between=pos)
     if L.device_status(ws) != 0:
         raise RuntimeError("device status error during the model bench")
-    n_pre = max(1, steps // 4)
     mean_T = sum(S + (i % nsteps) + 1 for i in range(steps)) / steps
     kv_bytes = w.n_layers * 2 * B * w.n_kv_heads * mean_T * w.head_dim * 2
     return {
@@ -431,6 +490,83 @@ def oracle_sample(tokens=256, repeats=None, budget_s=12.0):
     return tokens, times
 
 
+def _fp64_layer(w, seed):
+    """fp64 weights of workload ``w``'s layer shape for the CPU oracle's timing
+    (the seeded recipe; values do not change the oracle's time)."""
+    import numpy as np
+    return {k: np.asarray(v, np.float64) for k, v in synth.layer_weights(w, np.random.default_rng(seed)).items()}
+
+
+def _time_repeats(fn, budget_s):
+    """Median wall time of ``fn()`` over repeats within ``budget_s`` (at least one)."""
+    times = []
+    t_start = time.perf_counter()
+    while not times or time.perf_counter() - t_start < budget_s:
+        t0 = time.perf_counter()
+        fn()
+        times.append(time.perf_counter() - t0)
+    return statistics.median(times), len(times)
+
+
+def oracle_workload_baselines(budget_s=3.0):
+    """The fp64 oracle timed on a bounded sample of each non-headline workload
+    (host cores; weights converted to fp64 outside the timed region).  Returns
+    {workload key: cpu_baseline object} in the units of that workload's line."""
+    import numpy as np
+
+    from oracle import block as ob
+    out = {}
+    cores, model = cpu_threads(), cpu_model()
+
+    def dims(w):
+        return ob.Dims(w.dim, w.n_heads, w.n_kv_heads, w.head_dim, w.ffn_dim, w.eps, w.rope_theta, w.rope_style)
+
+    def decode_sample(w, T0):
+        W = _fp64_layer(w, w.seed)
+        rng = np.random.default_rng(w.seed + 1)
+        k0 = rng.standard_normal((1, w.n_kv_heads, T0, w.head_dim))
+        v0 = rng.standard_normal((1, w.n_kv_heads, T0, w.head_dim))
+        x = rng.standard_normal((1, 1, w.dim))
+
+        def one():
+            ob.layer_forward(dims(w), W, x, ob.KVCache(1, w.n_kv_heads, w.head_dim, T0 + 1, k0, v0))
+        return one
+
+    def prefill_sample(w, tokens):
+        W = _fp64_layer(w, w.seed)
+        x = np.random.default_rng(w.seed + 1).standard_normal((1, tokens, w.dim))
+
+        def one():
+            ob.layer_forward(dims(w), W, x, ob.KVCache(1, w.n_kv_heads, w.head_dim, tokens))
+        return one
+
+    W = synth.WORKLOADS
+    t, n = _time_repeats(decode_sample(W["llama13b_decode"], 4096), budget_s)
+    out["llama13b_decode/decode"] = {
+        "value": 1.0 / t, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle decode step of 1 of 16 sequences at cache length 4097, median of {n} ({model})"}
+    t, n = _time_repeats(prefill_sample(W["gqa70b"], 256), budget_s)
+    out["gqa70b/prefill"] = {
+        "value": 256 / t, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle prefill of the first 256 of 2 x 4096 tokens, median of {n} ({model})"}
+    t, n = _time_repeats(decode_sample(W["gqa70b"], 4096), budget_s)
+    out["gqa70b/decode"] = {
+        "value": 1.0 / t, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle decode step of 1 of 64 sequences at cache length 4097, median of {n} ({model})"}
+    w = W["phi3mini_model"]
+    t, n = _time_repeats(prefill_sample(w, 128), budget_s)
+    out["phi3mini_model/prefill"] = {
+        "value": 128 / (t * w.n_layers), "unit": "tokens/s (model)", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle prefill of 128 of 8 x 512 tokens through ONE of the 32 layers, median of {n}, "
+                  f"scaled by 32 layers (embedding and lm_head not timed) ({model})"}
+    t, n = _time_repeats(decode_sample(w, 512), budget_s)
+    out["phi3mini_model/decode"] = {
+        "value": 1.0 / (t * w.n_layers), "unit": "tokens/s (model)", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle decode step of 1 of 8 sequences at cache length 513 through ONE of the 32 layers, "
+                  f"median of {n}, scaled by 32 layers ({model})"}
+    return out
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -465,6 +601,7 @@ def headline_config(w):
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     w = synth.WORKLOADS[HEADLINE]
@@ -472,7 +609,7 @@ def run_reference(args):
     _, times = oracle_sample(tokens, repeats=args.warmup + args.steps)
     timed_s = sum(times[args.warmup:])
     value = tokens * args.steps / timed_s
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * timed_s / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights)", "config": headline_config(w),
@@ -481,6 +618,31 @@ def run_reference(args):
                                        f"per step ({cpu_model()})"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+    return 0
+
+
+def run_fake(args):
+    """Host-logic self-test of the multi-rank plumbing (no GPU, gloo): every rank
+    'processes' 1000 units per step in (1 + rank) ms of sleep, timed on the host
+    clock; the line carries the same aggregation as a real run."""
+    rank, world, _ = dist_init(args.gpus, backend="gloo")
+    for _ in range(args.warmup):
+        time.sleep(0.001 * (1 + rank))
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.001 * (1 + rank))
+    elapsed = time.perf_counter() - t0
+    barrier(world)
+    value, slowest = aggregate_throughput(1000 * args.steps, elapsed, world, device="cpu")
+    if rank == 0:
+        print(json.dumps({"metric": "fake units/s", "value": value, "unit": "units/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * slowest / args.steps,
+                          "higher_is_better": True, "scaling": "weak", "data": "fake (host-logic self-test)",
+                          "slowest_rank_s": slowest}))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
     return 0
 
 
@@ -494,8 +656,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=None, choices=sorted(WORKLOAD_RUNNERS),
                     help="run one workload alone and print its own line (for profiling)")
+    ap.add_argument("--fake-workload", action="store_true",
+                    help="host-logic self-test of the multi-rank plumbing: no GPU, gloo, sleeps")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: re-run this command as N ranks on this node
+        return spawn_ranks(args.gpus, sys.argv[1:])
+    if args.fake_workload:
+        return run_fake(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.workload:
@@ -525,10 +694,12 @@ def main():
     peak_key = "bf16_tflops_sustained" if timed_region_s > 2.0 else "bf16_tflops"
     gu_flops = 2.0 * w.batch * w.prefill_len * 2 * w.ffn_dim * w.dim
     achieved = gu_flops / (kg["avg_us"] * 1e-6) / 1e12 if kg else None
+    traffic, traffic_note = roofline_traffic()
     roofline = {"kernel": "gemm_gate_up_swiglu", "bound": "tensor", "achieved": achieved,
                 "peak": peaks[peak_key], "unit": "TFLOP/s",
                 "frac": achieved / peaks[peak_key] if achieved else None,
-                "traffic": GATE_UP_TRAFFIC_BYTES, "peak_source": f"{peak_key} ({'of measured' if peak_src == 'measured' else 'of fallback'})",
+                "traffic": traffic, "traffic_source": traffic_note,
+                "peak_source": f"{peak_key} ({'of measured' if peak_src == 'measured' else 'of fallback'})",
                 "algorithmic_flops_per_launch": gu_flops}
     layer_flops = r["gemm_flops"] + r["attn_flops"]
     layer_tflops = layer_flops / r["t_step_s"] / 1e12
@@ -539,6 +710,10 @@ def main():
         cpu = {"value": tokens / statistics.median(times), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"fp64 oracle prefill of the first {tokens} of {w.prefill_len} tokens of the headline layer, "
                          f"median of {len(times)} runs ({cpu_model()})"}
+        if workloads:
+            for name, cb in oracle_workload_baselines().items():
+                if name in workloads:
+                    workloads[name]["cpu_baseline"] = cb
 
     if rank == 0:
         line = {
@@ -557,6 +732,12 @@ def main():
             "kernels_us": {k: round(v["avg_us"], 2) for k, v in r["kernels"].items()},
             "clocks": clocks, "workloads": workloads,
         }
+        dec = workloads.get("llama13b_decode/decode")
+        if dec:
+            line["decode"] = {"workload": "llama13b_decode: LLaMA-2-13B-shaped layer, bf16, batch 16, cache "
+                                          "4096 -> 4224 over 128 steps, interleaved RoPE",
+                              "value": dec["tokens_per_s_per_layer"], "unit": UNIT,
+                              "frac_of_hbm_peak": dec["frac_of_hbm_peak"]}
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
@@ -564,8 +745,8 @@ def main():
     return 0
 
 
-def _single_decode(L, torch, name, args):
-    r = bench_decode_layer(L, torch, synth.WORKLOADS[name], args.steps, args.warmup, 1, seed=11)
+def _single_decode(L, torch, name, args, q4=False):
+    r = bench_decode_layer(L, torch, synth.WORKLOADS[name], args.steps, args.warmup, 1, seed=11, q4=q4)
     by = r["weight_bytes"] + r["kv_bytes"] + r["append_bytes"]
     return {"metric": "decode tokens/s per layer", "unit": UNIT, "value": r["tokens_per_step"] / r["t_step_s"],
             "ms_per_step": 1e3 * r["t_step_s"], "gbs": by / r["t_step_s"] / 1e9,
@@ -592,6 +773,7 @@ WORKLOAD_RUNNERS = {
     "llama13b_decode": lambda L, t, a: _single_decode(L, t, "llama13b_decode", a),
     "gqa70b_prefill": lambda L, t, a: _single_prefill(L, t, "gqa70b", a),
     "gqa70b_decode": lambda L, t, a: _single_decode(L, t, "gqa70b", a),
+    "llama13b_decode_q4": lambda L, t, a: _single_decode(L, t, "llama13b_decode", a, q4=True),
     "phi3_prefill": lambda L, t, a: _single_model(L, t, "prefill", a),
     "phi3_decode": lambda L, t, a: _single_model(L, t, "decode", a),
 }
@@ -621,21 +803,34 @@ def run_other_workloads(L, torch, args, peaks):
                 "tokens_per_s_per_layer": r["tokens_per_step"] / r["t_step_s"], "ms_per_step": 1e3 * r["t_step_s"],
                 "tflops": fl / r["t_step_s"] / 1e12, "frac_of_tensor_peak": fl / r["t_step_s"] / tc,
                 "kernels_us": {k: round(v["avg_us"], 1) for k, v in r["kernels"].items()}}
-        r = bench_decode_layer(L, torch, w, args.steps, args.warmup, 1, seed=11)
+        r = bench_decode_layer(L, torch, w, w.decode_steps, args.warmup, 1, seed=11)
         by = r["weight_bytes"] + r["kv_bytes"] + r["append_bytes"]
         out[f"{name}/decode"] = {
+            "steps": w.decode_steps, "cache_lengths": [w.cache_len + 1, w.cache_len + w.decode_steps],
             "tokens_per_s_per_layer": r["tokens_per_step"] / r["t_step_s"], "ms_per_step": 1e3 * r["t_step_s"],
             "gbs": by / r["t_step_s"] / 1e9, "frac_of_hbm_peak": by / r["t_step_s"] / hbm,
             "kernels_us": {k: round(v["avg_us"], 1) for k, v in r["kernels"].items()}}
         torch.cuda.empty_cache()
+    w = synth.WORKLOADS["llama13b_decode"]
+    r = bench_decode_layer(L, torch, w, w.decode_steps, args.warmup, 1, seed=13, q4=True)
+    by = r["weight_bytes"] + r["kv_bytes"] + r["append_bytes"]
+    out["llama13b_decode_q4/decode"] = {
+        "weights": "4-bit group-64 (codes + bf16 scale/offset per 64 weights)",
+        "steps": w.decode_steps, "cache_lengths": [w.cache_len + 1, w.cache_len + w.decode_steps],
+        "weight_bytes": r["weight_bytes"], "tokens_per_s_per_layer": r["tokens_per_step"] / r["t_step_s"],
+        "ms_per_step": 1e3 * r["t_step_s"], "gbs": by / r["t_step_s"] / 1e9, "frac_of_hbm_peak": by / r["t_step_s"] / hbm,
+        "kernels_us": {k: round(v["avg_us"], 1) for k, v in r["kernels"].items()}}
+    torch.cuda.empty_cache()
     w = synth.WORKLOADS["phi3mini_model"]
-    r = bench_model(L, torch, w, args.steps, args.warmup, 1, seed=21)
+    r = bench_model(L, torch, w, w.decode_steps, args.warmup, 1, seed=21, prefill_steps=max(3, args.steps // 4))
     p, d = r["prefill"], r["decode"]
     out["phi3mini_model/prefill"] = {"tokens_per_s_model": p["tokens_per_step"] / p["t_step_s"],
                                      "ms_per_step": 1e3 * p["t_step_s"],
                                      "tflops": p["flops"] / p["t_step_s"] / 1e12,
                                      "frac_of_tensor_peak": p["flops"] / p["t_step_s"] / tc}
-    out["phi3mini_model/decode"] = {"tokens_per_s_model": d["tokens_per_step"] / d["t_step_s"],
+    out["phi3mini_model/decode"] = {"steps": w.decode_steps,
+                                    "cache_lengths": [w.prefill_len + 1, w.prefill_len + w.decode_steps],
+                                    "tokens_per_s_model": d["tokens_per_step"] / d["t_step_s"],
                                     "ms_per_step": 1e3 * d["t_step_s"],
                                     "gbs": d["bytes"] / d["t_step_s"] / 1e9,
                                     "frac_of_hbm_peak": d["bytes"] / d["t_step_s"] / hbm,

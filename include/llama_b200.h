@@ -197,6 +197,48 @@ llama_status llama_layer_decode(const llama_dims* dims, const llama_layer_weight
                                 int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/* ------------------------------------------------------------------ 4-bit group-64 weights (decode) */
+
+/* One projection [out_features, in_features] with 4-bit group-wise weights
+ * ([MLX-13B] "LLaMA 2 的结构分析": every projection of the 13B block is a
+ * QuantizedLinear; "模型配置": "quantization": {"group_size": 64, "bits": 4}).
+ * The pages name the scheme without defining it; reading taken: each row is
+ * cut into groups of 64 consecutive inputs, a group keeps a scale s and an
+ * offset b, and each weight an unsigned code q in 0..15, so that the Linear
+ * uses w = s * q + b (y = x W^T, no bias).
+ *   codes    device uint32 [out][in / 8]: code of input 8j + k of a row in
+ *            bits 4k .. 4k+3 of word j (low nibble first)
+ *   scales   device bf16 [in / 64][out]: s of (row o, group g) at [g][o]
+ *   offsets  device bf16 [in / 64][out]: b, same layout
+ * (the scales and offsets are stored group-major so that one group's values
+ * for 64 consecutive rows are one contiguous 128-byte block).  The kernel
+ * forms bf16 w = fma(q, s, b) with one rounding and multiplies on the tensor
+ * cores with fp32 accumulation. */
+typedef struct llama_q4_weight {
+  const uint32_t* codes;
+  const void* scales;
+  const void* offsets;
+} llama_q4_weight;
+
+/* One block's weights with every projection in the 4-bit form; norm weights
+ * float32 [dim].  wq/wk/wv rows as in llama_layer_weights (three separate
+ * projections); w1 gate, w3 up, w2 down. */
+typedef struct llama_layer_weights_q4 {
+  const float* attn_norm;
+  llama_q4_weight wq, wk, wv, wo;
+  const float* ffn_norm;
+  llama_q4_weight w1, w3, w2;
+} llama_layer_weights_q4;
+
+/* llama_layer_decode with 4-bit group-64 weights: the same block, the same
+ * cache (dims->dtype must be LLAMA_BF16: bf16 activations and KV cache) and
+ * the same workspace (llama_workspace_size(dims, batch, 1)).  Requires dim,
+ * ffn_dim and n_heads*head_dim multiples of 64 and batch <= 128.
+ * Errors: as llama_layer_decode; UNSUPPORTED for the shapes above. */
+llama_status llama_layer_decode_q4(const llama_dims* dims, const llama_layer_weights_q4* w, llama_kv_cache* cache,
+                                   int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
 /* ------------------------------------------------------------------ whole model */
 
 /* A whole model ([DeepDive] class LLaMA; [HandsOn] Phi3ForCausalLM tree).
@@ -226,6 +268,36 @@ size_t llama_model_workspace_size(const llama_model* model, int32_t batch, int32
 llama_status llama_model_forward(const llama_model* model, llama_kv_cache* const* caches, const int32_t* tokens,
                                  int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ sampling */
+
+/* Temperature / top-p (nucleus) sampling of the next token ([DeepDive] class
+ * LLaMA, generate: logits / temperature, sorted descending, cumulative
+ * softmax; a token is dropped once the probability of the tokens sorted
+ * before it exceeds top_p, so the token that crosses top_p is kept; the kept
+ * tokens are renormalised and one is drawn.  [MLX-13B] 生成过程: temperature 0
+ * is greedy argmax).
+ *   logits   device float32 [batch, vocab]
+ *   u        device float32 [batch], one uniform in [0, 1) per sequence: the
+ *            draw is an input; the token picked is the kept token whose
+ *            interval of the cumulative renormalised distribution, in sorted
+ *            order, holds u (inverse CDF)
+ *   ids      device int32 [batch]
+ * Sorted order is descending logit / temperature, equal values by ascending
+ * index.  Probabilities are exp(z - max z) in fp32, accumulated as integers
+ * in units of 2^-40 (exact, order-independent sums).  temperature 0 takes
+ * the argmax (u unused, may be NULL); otherwise temperature > 0 and
+ * 0 < top_p <= 1.  Allocates nothing; no workspace.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+llama_status llama_sample_top_p(const float* logits, int32_t batch, int32_t vocab, float temperature, float top_p,
+                                const float* u, int32_t* ids, void* stream);
+
+/* llama_model_forward with the next token chosen by llama_sample_top_p's rule
+ * on the last row's logits instead of argmax (temperature 0: argmax). */
+llama_status llama_model_forward_sample(const llama_model* model, llama_kv_cache* const* caches,
+                                        const int32_t* tokens, int32_t batch, int32_t seq_len, float temperature,
+                                        float top_p, const float* u, float* logits_or_null, int32_t* next_ids,
+                                        void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ allocation-free decode attention */
 

@@ -25,6 +25,7 @@ __all__ = [
     "workspace_size", "model_workspace_size", "layer_prefill", "layer_decode",
     "model_forward", "device_status", "workspace_offsets", "set_wait_limit_ns", "selftest_wait_timeout",
     "launch_count", "profile_enable", "profile_read", "profile_inflight", "attention_decode_noalloc",
+    "sample_top_p", "model_forward_sample", "Q4Weight", "LayerWeightsQ4", "layer_weights_q4", "layer_decode_q4",
 ]
 
 F32, BF16 = 0, 1
@@ -60,6 +61,16 @@ class Model(ctypes.Structure):
                 ("layers", ctypes.POINTER(LayerWeights))]
 
 
+class Q4Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("offsets", ctypes.c_void_p)]
+
+
+class LayerWeightsQ4(ctypes.Structure):
+    _fields_ = [("attn_norm", ctypes.c_void_p), ("wq", Q4Weight), ("wk", Q4Weight), ("wv", Q4Weight),
+                ("wo", Q4Weight), ("ffn_norm", ctypes.c_void_p), ("w1", Q4Weight), ("w3", Q4Weight),
+                ("w2", Q4Weight)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
 _S = ctypes.c_size_t
@@ -83,9 +94,13 @@ EXPORTS = {
     "llama_workspace_offsets": (_I, [_DP, _I, _I, ctypes.POINTER(_S), _I]),
     "llama_layer_prefill": (_I, [_DP, _WP, _P, _I, _I, _P, _P, _P, _S, _P]),
     "llama_layer_decode": (_I, [_DP, _WP, _P, _I, _P, _P, _P, _S, _P]),
+    "llama_layer_decode_q4": (_I, [_DP, ctypes.POINTER(LayerWeightsQ4), _P, _I, _P, _P, _P, _S, _P]),
     "llama_model_workspace_size": (_S, [_MP, _I, _I]),
     "llama_model_forward": (_I, [_MP, ctypes.POINTER(_P), _P, _I, _I, _P, _P, _P, _S, _P]),
     "llama_selftest_wait_timeout": (_I, [_P, _U64, _P]),
+    "llama_sample_top_p": (_I, [_P, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P]),
+    "llama_model_forward_sample": (_I, [_MP, ctypes.POINTER(_P), _P, _I, _I, ctypes.c_float, ctypes.c_float, _P,
+                                        _P, _P, _P, _S, _P]),
     "llama_attention_decode_noalloc": (_I, [_DP, _I, _P, _I, _P, _P, _I, _I, _P, _P]),
     "llama_launch_count": (_U64, []),
     "llama_profile_enable": (_I, [_I]),
@@ -143,6 +158,16 @@ def layer_weights(t):
     """``LayerWeights`` from a dict of device tensors (keys attn_norm, wq, ... w2)."""
     return LayerWeights(*[_ptr(t[k]) for k in
                           ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w1", "w3", "w2")])
+
+
+def layer_weights_q4(t):
+    """``LayerWeightsQ4`` from a dict: attn_norm, ffn_norm (device float32) and, for each of
+    wq wk wv wo w1 w3 w2, a (codes, scales, offsets) triple of device tensors."""
+    def q(k):
+        c, sc, of = t[k]
+        return Q4Weight(_ptr(c), _ptr(sc), _ptr(of))
+    return LayerWeightsQ4(_ptr(t["attn_norm"]), q("wq"), q("wk"), q("wv"), q("wo"), _ptr(t["ffn_norm"]),
+                          q("w1"), q("w3"), q("w2"))
 
 
 def model_struct(dims, embed, final_norm, lm_head, layers):
@@ -204,11 +229,33 @@ def layer_decode(dims, w, cache, batch, x_in, x_out, ws, stream=None):
            "llama_layer_decode")
 
 
+def layer_decode_q4(dims, w, cache, batch, x_in, x_out, ws, stream=None):
+    _check(lib().llama_layer_decode_q4(ctypes.byref(dims), ctypes.byref(w), cache.handle, batch, _ptr(x_in),
+                                       _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "llama_layer_decode_q4")
+
+
 def model_forward(model, caches, tokens, batch, seq_len, logits, next_ids, ws, stream=None):
     arr = (ctypes.c_void_p * len(caches))(*[c.handle.value for c in caches])
     _check(lib().llama_model_forward(ctypes.byref(model), arr, _ptr(tokens), batch, seq_len, _ptr(logits),
                                      _ptr(next_ids), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "llama_model_forward")
+
+
+def model_forward_sample(model, caches, tokens, batch, seq_len, temperature, top_p, u, logits, next_ids, ws,
+                         stream=None):
+    arr = (ctypes.c_void_p * len(caches))(*[c.handle.value for c in caches])
+    _check(lib().llama_model_forward_sample(ctypes.byref(model), arr, _ptr(tokens), batch, seq_len,
+                                            float(temperature), float(top_p), _ptr(u), _ptr(logits),
+                                            _ptr(next_ids), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)), "llama_model_forward_sample")
+
+
+def sample_top_p(logits, temperature, top_p, u, ids, stream=None):
+    """ids [B] from logits [B, V] (device float32) and uniforms u [B] (device float32)."""
+    B, V = logits.shape
+    _check(lib().llama_sample_top_p(_ptr(logits), B, V, float(temperature), float(top_p), _ptr(u), _ptr(ids),
+                                    _stream(stream)), "llama_sample_top_p")
 
 
 def workspace_offsets(dims, batch, seq_len):

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <set>
 #include <utility>
 #include <unordered_map>
 #include <vector>
@@ -19,7 +20,9 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "f32_path.cuh"
+#include "gemm_q4.cuh"
 #include "gemm_tc.cuh"
+#include "sampling.cuh"
 #include "small_kernels.cuh"
 
 using namespace llama;
@@ -52,12 +55,12 @@ constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K for
 enum KernelKind : int {
   K_RMSNORM = 0, K_GEMM_QKV, K_ROPE_APPEND, K_ATTN_PREFILL, K_ATTN_DECODE, K_ATTN_COMBINE, K_GEMM_O,
   K_GEMM_GATE_UP, K_GEMM_DOWN, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
-  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_COUNT
+  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_SAMPLE, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
   "rmsnorm", "gemm_qkv", "rope_kv_append", "attn_prefill", "attn_decode", "attn_decode_combine", "gemm_o_proj",
   "gemm_gate_up_swiglu", "gemm_down", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
-  "gemm_f32", "attn_f32", "selftest"};
+  "gemm_f32", "attn_f32", "selftest", "sample_top_p"};
 
 struct ProfRec {
   cudaEvent_t a, b;
@@ -163,8 +166,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
 // dims[0] is the contiguous dimension; strides are in bytes for dims 1..rank-1.
-bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box) {
+bool make_map_ex(CUtensorMap* m, const void* base, CUtensorMapDataType dt, CUtensorMapSwizzle sw, int rank,
+                 const uint64_t* dims, const uint64_t* strides, const uint32_t* box) {
   auto enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t d[5], s[4];
@@ -175,10 +178,14 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides[i];
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s, bx, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, dt, (cuuint32_t)rank, const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  return make_map_ex(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, rank, dims, strides, box);
 }
 
 // Encoded 2-D maps are cached by (base, inner, rows, box rows): weights and
@@ -282,6 +289,20 @@ cudaError_t launch_k_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// cudaFuncSetAttribute acts on the current device only, so a kernel's dynamic
+// shared-memory limit is raised once per (kernel, device) pair.
+llama_status ensure_smem_attr(const void* kernel, int bytes) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> g(mu);
+  if (done.count({kernel, dev}) != 0) return LLAMA_OK;
+  CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.insert({kernel, dev});
+  return LLAMA_OK;
 }
 
 // ------------------------------------------------------------------ validation
@@ -391,12 +412,7 @@ template <int BN, bool SWAP, int EPI>
 llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
                             cudaStream_t st, int kind) {
   using C = GemmCfg<BN, !SWAP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, SWAP, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  C::SMEM_BYTES));
-    attr_set = true;
-  }
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, SWAP, EPI>), C::SMEM_BYTES));
   {
     TRACE(kind, st);
     if (SWAP)
@@ -577,15 +593,113 @@ llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int
   return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
 }
 
+// ------------------------------------------------------------------ 4-bit group-64 decode GEMMs
+
+struct Q4Seg {
+  llama_q4_weight w;
+  int rows;
+  int col0;
+};
+
+template <int BN, int EPI>
+llama_status launch_gemm_q4(const CUtensorMap& a, const Q4Maps& maps, const GemmParams& p, int grid, cudaStream_t st,
+                            int kind) {
+  using C = Q4Cfg<BN>;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_q4_kernel<BN, EPI>), C::SMEM_BYTES));
+  {
+    TRACE(kind, st);
+    CUDA_TRY(launch_k(gemm_q4_kernel<BN, EPI>, grid, Q4_THREADS, C::SMEM_BYTES, st, a, maps, p));
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+template <int BN>
+llama_status launch_gemm_q4_epi(int epi, const CUtensorMap& a, const Q4Maps& maps, const GemmParams& p, int grid,
+                                cudaStream_t st, int kind) {
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_q4<BN, EPI_BF16>(a, maps, p, grid, st, kind);
+    case EPI_RESID_F32: return launch_gemm_q4<BN, EPI_RESID_F32>(a, maps, p, grid, st, kind);
+    case EPI_SWIGLU_BF16: return launch_gemm_q4<BN, EPI_SWIGLU_BF16>(a, maps, p, grid, st, kind);
+  }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+// Decode GEMM with 4-bit weights: out = epilogue(act[M, K] . W^T), W given as
+// up to three segments (or, for EPI_SWIGLU_BF16, gate = segs[0], up = segs[1]).
+llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, const Q4Seg* segs, int nseg, int epi,
+                            void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
+                            int kind) {
+  if (M > kSwapMaxTokens || K % 64 != 0) return LLAMA_ERR_UNSUPPORTED;
+  const int BN = swap_bn(M);
+  GemmParams p{};
+  p.K = K;
+  p.num_kb = K / 64;
+  p.act_rows = M;
+  p.m_tiles = 1;
+  p.nseg = nseg;
+  p.out = out;
+  p.ldo = ldo;
+  p.resid = resid;
+  p.ldr = ldr;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  p.partial = sk.partial;
+  p.flags = sk.flags;
+  CUtensorMap ta;
+  Q4Maps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!make_map_2d(&ta, act, K, M, BN)) return LLAMA_ERR_CUDA;
+  for (int s = 0; s < nseg; ++s) {
+    const uint64_t rows = (uint64_t)segs[s].rows, groups = (uint64_t)K / 64;
+    {
+      const uint64_t dims[2] = {(uint64_t)K / 8, rows};
+      const uint64_t strides[1] = {(uint64_t)K / 8 * 4};
+      const uint32_t box[2] = {8, 64};
+      if (!make_map_ex(&maps.codes[s], segs[s].w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       2, dims, strides, box))
+        return LLAMA_ERR_CUDA;
+    }
+    const uint64_t dims[2] = {rows, groups};
+    const uint64_t strides[1] = {rows * 2};
+    const uint32_t box[2] = {64, 1};
+    if (!make_map_ex(&maps.scales[s], segs[s].w.scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     2, dims, strides, box) ||
+        !make_map_ex(&maps.offsets[s], segs[s].w.offsets, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, 2, dims, strides, box))
+      return LLAMA_ERR_CUDA;
+  }
+  int t = 0;
+  if (epi == EPI_SWIGLU_BF16) {
+    p.seg_rows[0] = segs[0].rows;
+    t = cdiv(segs[0].rows, 64);
+    for (int s = 1; s < 4; ++s) p.seg_tile0[s] = t;
+  } else {
+    for (int s = 0; s < nseg; ++s) {
+      p.seg_rows[s] = segs[s].rows;
+      p.seg_col0[s] = segs[s].col0;
+      p.seg_tile0[s] = t;
+      t += cdiv(segs[s].rows, 128);
+    }
+    for (int s = nseg; s < 4; ++s) p.seg_tile0[s] = t;
+  }
+  p.n_tiles = t;
+  p.units = (long long)p.n_tiles * p.num_kb;
+  const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
+  if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;
+  switch (BN) {
+    case 16: return launch_gemm_q4_epi<16>(epi, ta, maps, p, grid, st, kind);
+    case 32: return launch_gemm_q4_epi<32>(epi, ta, maps, p, grid, st, kind);
+    case 64: return launch_gemm_q4_epi<64>(epi, ta, maps, p, grid, st, kind);
+    default: return launch_gemm_q4_epi<128>(epi, ta, maps, p, grid, st, kind);
+  }
+}
+
 // ------------------------------------------------------------------ attention launchers
 
 llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int L, int p0,
                                const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM));
-    attr_set = true;
-  }
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_prefill_kernel), ATT_SMEM));
   const int hd = d.head_dim;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
   const int T = p0 + L;
@@ -630,12 +744,7 @@ template <int HD, int G>
 llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
                                     dim3 grid, cudaStream_t st) {
   using C = DecMmaCfg<HD>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_decode_mma_kernel<HD, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  C::SMEM));
-    attr_set = true;
-  }
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_mma_kernel<HD, G>), C::SMEM));
   CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G>, grid, 160, C::SMEM, st, tk, tv, p));
   return LLAMA_OK;
 }
@@ -885,8 +994,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     const int Tmax = p0 + L;
     const size_t smem = (size_t)Tmax * 4;
     if (smem > 200 * 1024) return LLAMA_ERR_UNSUPPORTED;
-    if (smem > 48 * 1024)
-      CUDA_TRY(cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    if (smem > 48 * 1024) TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_f32_kernel), 200 * 1024));
     {
       TRACE(K_ATTN_F32, st);
       attn_f32_kernel<<<dim3(L, nh, B), 128, smem, st>>>(qkv, qkvn, static_cast<const float*>(kv->k),
@@ -921,6 +1029,75 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     LAUNCH_CHECK();
   }
   kv->length = p0 + L;
+  return LLAMA_OK;
+}
+
+// ------------------------------------------------------------------ one block, 4-bit weights (decode)
+
+llama_status check_q4(const llama_q4_weight& w) {
+  if (w.codes == nullptr || w.scales == nullptr || w.offsets == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(w.codes) || !aligned16(w.scales) || !aligned16(w.offsets)) return LLAMA_ERR_ALIGNMENT;
+  return LLAMA_OK;
+}
+
+llama_status check_layer_q4(const llama_dims* d, const llama_layer_weights_q4* w) {
+  TRY(check_dims(d));
+  if (w == nullptr || w->attn_norm == nullptr || w->ffn_norm == nullptr) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(w->attn_norm) || !aligned16(w->ffn_norm)) return LLAMA_ERR_ALIGNMENT;
+  for (const llama_q4_weight* q : {&w->wq, &w->wk, &w->wv, &w->wo, &w->w1, &w->w3, &w->w2}) TRY(check_q4(*q));
+  if (d->dtype != LLAMA_BF16) return LLAMA_ERR_UNSUPPORTED;
+  // every input dimension is cut into whole groups of 64
+  if (d->dim % 64 || d->ffn_dim % 64 || (d->n_heads * d->head_dim) % 64) return LLAMA_ERR_UNSUPPORTED;
+  return LLAMA_OK;
+}
+
+// Decode step of one block whose seven projections hold 4-bit group-64
+// weights: the same sequence as run_layer's bf16 decode path, each
+// projection on gemm_q4_kernel.
+llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_q4& w, llama_kv_cache* kv, int B,
+                                 const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay,
+                                 cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+  const int qkvn = (nh + 2 * nkv) * hd;
+  const int p0 = kv->length;
+  bf* qkv = reinterpret_cast<bf*>(ws + lay.qkv);
+  bf* h = reinterpret_cast<bf*>(ws + lay.h);
+  bf* att = reinterpret_cast<bf*>(ws + lay.attn);
+  bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
+  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
+  {
+    TRACE(K_RMSNORM, st);
+    CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, B, d.dim,
+                      d.eps, RopeTab{}));
+  }
+  LAUNCH_CHECK();
+  const Q4Seg sq[3] = {{w.wq, nh * hd, 0}, {w.wk, nkv * hd, nh * hd}, {w.wv, nkv * hd, (nh + nkv) * hd}};
+  TRY(gemm_decode_q4(st, h, B, d.dim, sq, 3, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
+  {
+    TRACE(K_ROPE_APPEND, st);
+    CUDA_TRY(launch_k(rope_append_kernel<bf>, B, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
+                      reinterpret_cast<bf*>(kv->v), 1, p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style));
+  }
+  LAUNCH_CHECK();
+  TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
+                       reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o), status));
+  const Q4Seg so{w.wo, d.dim, 0};
+  TRY(gemm_decode_q4(st, att, B, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status, K_GEMM_O));
+  {
+    TRACE(K_RMSNORM, st);
+    CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, B, d.dim,
+                      d.eps, RopeTab{}));
+  }
+  LAUNCH_CHECK();
+  const Q4Seg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
+  TRY(gemm_decode_q4(st, h, B, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
+                     K_GEMM_GATE_UP));
+  const Q4Seg sd{w.w2, d.dim, 0};
+  TRY(gemm_decode_q4(st, mb, B, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
+                     K_GEMM_DOWN));
+  kv->length = p0 + 1;
   return LLAMA_OK;
 }
 
@@ -1077,14 +1254,68 @@ llama_status llama_layer_decode(const llama_dims* dims, const llama_layer_weight
                    static_cast<cudaStream_t>(stream));
 }
 
+llama_status llama_layer_decode_q4(const llama_dims* dims, const llama_layer_weights_q4* w, llama_kv_cache* cache,
+                                   int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  TRY(check_layer_q4(dims, w));
+  if (cache == nullptr || x_in == nullptr || x_out == nullptr || workspace == nullptr || batch <= 0)
+    return LLAMA_ERR_INVALID_ARG;
+  if (batch > kSwapMaxTokens) return LLAMA_ERR_UNSUPPORTED;
+  if (!same_dims(*dims, cache->dims) || batch != cache->batch) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(workspace)) return LLAMA_ERR_ALIGNMENT;
+  const size_t xb = (size_t)batch * dims->dim * 4;
+  if (overlap(x_in, xb, x_out, xb)) return LLAMA_ERR_INVALID_ARG;
+  if ((long long)cache->length + 1 > cache->capacity) return LLAMA_ERR_CACHE_FULL;
+  const WsLayout lay = plan_ws(*dims, batch, 1, 0);
+  if (ws_bytes < lay.total) return LLAMA_ERR_WORKSPACE_TOO_SMALL;
+  return run_layer_decode_q4(*dims, *w, cache, batch, x_in, x_out, static_cast<uint8_t*>(workspace), lay,
+                             static_cast<cudaStream_t>(stream));
+}
+
 size_t llama_model_workspace_size(const llama_model* m, int32_t batch, int32_t seq_len) {
   if (m == nullptr || check_dims(&m->dims) != LLAMA_OK || batch <= 0 || seq_len <= 0 || m->vocab <= 0) return 0;
   return plan_ws(m->dims, batch, seq_len, m->vocab).total;
 }
 
-llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* caches, const int32_t* tokens,
-                                 int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
-                                 void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Next-token choice after the lm_head: greedy argmax, or temperature / top-p
+// sampling with one uniform per sequence.
+struct TokenPick {
+  float temperature;   // 0: argmax
+  float top_p;
+  const float* u;      // device [batch]
+};
+
+llama_status check_pick(const TokenPick& pk, int batch) {
+  if (!(pk.temperature >= 0.f) || !(pk.temperature < 1e30f)) return LLAMA_ERR_INVALID_ARG;
+  if (pk.temperature > 0.f) {
+    if (!(pk.top_p > 0.f) || !(pk.top_p <= 1.f) || pk.u == nullptr) return LLAMA_ERR_INVALID_ARG;
+    if (!aligned16(pk.u)) return LLAMA_ERR_ALIGNMENT;
+  }
+  (void)batch;
+  return LLAMA_OK;
+}
+
+llama_status enqueue_pick(const TokenPick& pk, const float* logits, int batch, int vocab, int32_t* ids,
+                          cudaStream_t st) {
+  if (pk.temperature == 0.f) {
+    TRACE(K_ARGMAX, st);
+    CUDA_TRY(launch_k(argmax_kernel, batch, 1024, 0, st, logits, vocab, ids));
+  } else {
+    TRACE(K_SAMPLE, st);
+    CUDA_TRY(launch_k(sample_top_p_kernel, batch, SAMPLE_THREADS, 0, st, logits, vocab, pk.temperature, pk.top_p,
+                      pk.u, ids));
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, const int32_t* tokens,
+                           int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
+                           void* workspace, size_t ws_bytes, void* stream, const TokenPick& pick) {
   if (m == nullptr || caches == nullptr || tokens == nullptr || next_ids == nullptr || workspace == nullptr)
     return LLAMA_ERR_INVALID_ARG;
   TRY(check_dims(&m->dims));
@@ -1167,12 +1398,37 @@ llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* ca
     }
     LAUNCH_CHECK();
   }
-  {
-    TRACE(K_ARGMAX, st);
-    CUDA_TRY(launch_k(argmax_kernel, batch, 1024, 0, st, logits, m->vocab, next_ids));
-  }
-  LAUNCH_CHECK();
-  return LLAMA_OK;
+  return enqueue_pick(pick, logits, batch, m->vocab, next_ids, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+llama_status llama_model_forward(const llama_model* m, llama_kv_cache* const* caches, const int32_t* tokens,
+                                 int32_t batch, int32_t seq_len, float* logits_or_null, int32_t* next_ids,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  return model_forward(m, caches, tokens, batch, seq_len, logits_or_null, next_ids, workspace, ws_bytes, stream,
+                       TokenPick{0.f, 1.f, nullptr});
+}
+
+llama_status llama_model_forward_sample(const llama_model* m, llama_kv_cache* const* caches, const int32_t* tokens,
+                                        int32_t batch, int32_t seq_len, float temperature, float top_p,
+                                        const float* u, float* logits_or_null, int32_t* next_ids, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  const TokenPick pk{temperature, top_p, u};
+  TRY(check_pick(pk, batch));
+  return model_forward(m, caches, tokens, batch, seq_len, logits_or_null, next_ids, workspace, ws_bytes, stream,
+                       pk);
+}
+
+llama_status llama_sample_top_p(const float* logits, int32_t batch, int32_t vocab, float temperature, float top_p,
+                                const float* u, int32_t* ids, void* stream) {
+  if (logits == nullptr || ids == nullptr || batch <= 0 || vocab <= 0) return LLAMA_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(ids)) return LLAMA_ERR_ALIGNMENT;
+  const TokenPick pk{temperature, top_p, u};
+  TRY(check_pick(pk, batch));
+  return enqueue_pick(pk, logits, batch, vocab, ids, static_cast<cudaStream_t>(stream));
 }
 
 llama_status llama_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {

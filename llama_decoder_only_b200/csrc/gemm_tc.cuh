@@ -168,6 +168,147 @@ __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
   return s;
 }
 
+// Stream-K epilogue of one work item (decode form): the accumulator holds
+// TMEM lane `row` = weight row of the tile, column j = token j.  A piece that
+// does not end its tile is published for the tile's finisher; the CTA that
+// ends the tile adds the pieces of the lower CTAs that share it, in CTA order,
+// and applies the epilogue.  Called by every epilogue thread; `leader` is one
+// of them (it handles the flag words), `xch` this thread's half of the
+// gate/up exchange buffer in shared memory.
+template <int BN, int EPI, typename Sync>
+__device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const GemmItem& item, uint32_t tbase, int row,
+                                                 int half, float* xch, bool leader, int* abort_sh, Sync& epi_sync) {
+  // accumulator: TMEM lane `row` = weight row of the tile, column j = token j
+  if (item.kb1 < p.num_kb) {
+    // a piece that does not end its tile: publish it for the tile's finisher
+    float* dst = p.partial + ((size_t)blockIdx.x * 128 + row) * BN;
+#pragma unroll 1
+    for (int c = half * 16; c < BN; c += 32) {
+      float v[16];
+      tmem_ld16(tbase + c, v);
+      tmem_ld_wait();
+      float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    // the group barrier orders every thread's stores before thread 64's
+    // release, which makes them visible at GPU scope before the flag
+    epi_sync();
+    if (leader)
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + blockIdx.x), "r"(1u) : "memory");
+  } else {
+    // this CTA ends the tile: add the partials of the lower CTAs that share it
+    const unsigned U = (unsigned)p.units, G = gridDim.x, KB = (unsigned)p.num_kb;
+    const unsigned x = (unsigned)item.tile * KB;
+    int c_first = (int)(((x + 1) * G + U - 1) / U) - 1;
+    c_first = c_first < 0 ? 0 : c_first;
+    // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count)
+    const int n_contrib = (int)blockIdx.x - c_first;
+    if (n_contrib > 0) {
+      if (leader) {
+        for (int c = c_first; c < (int)blockIdx.x; ++c) {
+          const uint64_t t0 = globaltimer_ns();
+          while (true) {
+            unsigned f;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.flags + c) : "memory");
+            if (f == 1u || *reinterpret_cast<volatile int*>(abort_sh)) break;
+            if (globaltimer_ns() - t0 > p.limit_ns) {
+              *abort_sh = 1;
+              record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 6, item.tile);
+              break;
+            }
+            __nanosleep(32);
+          }
+          // this CTA is the only reader of c's piece: re-arm the flag for the next launch
+          asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.flags + c), "r"(0u) : "memory");
+        }
+      }
+      epi_sync();
+    }
+    // weight row -> output column
+    int seg = 0, n = 0;
+    bool n_ok;
+    if (EPI == EPI_SWIGLU_BF16) {
+      n = item.tile * 64 + (row & 63);
+      n_ok = n < p.seg_rows[0];
+    } else {
+      seg = seg_of_tile(p, item.tile);
+      const int r_in_seg = (item.tile - p.seg_tile0[seg]) * 128 + row;
+      n_ok = r_in_seg < p.seg_rows[seg];
+      n = p.seg_col0[seg] + r_in_seg;
+    }
+  #pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      const int c = c0 + half * 16;   // this warp's 16 token columns (BN is a multiple of 16)
+      const bool active = c < BN;
+      float v[16];
+      if (active) {
+        tmem_ld16(tbase + c, v);
+        tmem_ld_wait();
+        // the contributors' pieces, in CTA order, up to four per round trip to L2
+        const float4* src = reinterpret_cast<const float4*>(p.partial + ((size_t)c_first * 128 + row) * BN + c);
+        constexpr size_t STRIDE4 = (size_t)128 * BN / 4;
+#pragma unroll 1
+        for (int k = 0; k < n_contrib; k += 4) {
+          float4 a[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              a[i][q] = k + i < n_contrib ? __ldcg(src + (size_t)(k + i) * STRIDE4 + q)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              v[4 * q + 0] += a[i][q].x;
+              v[4 * q + 1] += a[i][q].y;
+              v[4 * q + 2] += a[i][q].z;
+              v[4 * q + 3] += a[i][q].w;
+            }
+        }
+      }
+      if (EPI == EPI_SWIGLU_BF16) {
+        // up values (lanes 64..127) go through shared memory to the gate lanes
+        if (active && row >= 64) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) xch[j * 64 + row - 64] = v[j];
+        }
+        epi_sync();
+        if (active && row < 64 && n_ok) {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c + j < p.act_rows)
+              o[(size_t)(c + j) * p.ldo + n] = __float2bfloat16_rn(silu_f(v[j]) * xch[j * 64 + row]);
+        }
+        epi_sync();
+      } else if (active && n_ok) {
+        const int nj = p.act_rows - c < 16 ? p.act_rows - c : 16;
+        if (EPI == EPI_RESID_F32) {
+          // all residual loads first (out may alias resid: same element, same thread)
+          float r[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) r[j] = j < nj ? p.resid[(size_t)(c + j) * p.ldr + n] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < nj) reinterpret_cast<float*>(p.out)[(size_t)(c + j) * p.ldo + n] = r[j] + v[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (j >= nj) break;
+            const size_t o_idx = (size_t)(c + j) * p.ldo + n;
+            if (EPI == EPI_BF16)
+              reinterpret_cast<__nv_bfloat16*>(p.out)[o_idx] = __float2bfloat16_rn(v[j]);
+            else
+              reinterpret_cast<float*>(p.out)[o_idx] = v[j];
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int BN, bool SWAP, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW0,
@@ -433,137 +574,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(accf_bar(abuf), aphase, wc, 4))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(abuf * BN);
-      if (SWAP) {
-        // accumulator: TMEM lane `row` = weight row of the tile, column j = token j
-        if (item.kb1 < p.num_kb) {
-          // a piece that does not end its tile: publish it for the tile's finisher
-          float* dst = p.partial + ((size_t)blockIdx.x * 128 + row) * BN;
-#pragma unroll 1
-          for (int c = half * 16; c < BN; c += 32) {
-            float v[16];
-            tmem_ld16(tbase + c, v);
-            tmem_ld_wait();
-            float4* d4 = reinterpret_cast<float4*>(dst + c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-          // the group barrier orders every thread's stores before thread 64's
-          // release, which makes them visible at GPU scope before the flag
-          epi_sync();
-          if (threadIdx.x == 64)
-            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + blockIdx.x), "r"(1u) : "memory");
-        } else {
-          // this CTA ends the tile: add the partials of the lower CTAs that share it
-          const unsigned U = (unsigned)p.units, G = gridDim.x, KB = (unsigned)p.num_kb;
-          const unsigned x = (unsigned)item.tile * KB;
-          int c_first = (int)(((x + 1) * G + U - 1) / U) - 1;
-          c_first = c_first < 0 ? 0 : c_first;
-          // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count)
-          const int n_contrib = (int)blockIdx.x - c_first;
-          if (n_contrib > 0) {
-            if (threadIdx.x == 64) {
-              for (int c = c_first; c < (int)blockIdx.x; ++c) {
-                const uint64_t t0 = globaltimer_ns();
-                while (true) {
-                  unsigned f;
-                  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.flags + c) : "memory");
-                  if (f == 1u || *reinterpret_cast<volatile int*>(&abort_sh)) break;
-                  if (globaltimer_ns() - t0 > p.limit_ns) {
-                    abort_sh = 1;
-                    record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 6, item.tile);
-                    break;
-                  }
-                  __nanosleep(32);
-                }
-                // this CTA is the only reader of c's piece: re-arm the flag for the next launch
-                asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.flags + c), "r"(0u) : "memory");
-              }
-            }
-            epi_sync();
-          }
-          // weight row -> output column
-          int seg = 0, n = 0;
-          bool n_ok;
-          if (EPI == EPI_SWIGLU_BF16) {
-            n = item.tile * 64 + (row & 63);
-            n_ok = n < p.seg_rows[0];
-          } else {
-            seg = seg_of_tile(p, item.tile);
-            const int r_in_seg = (item.tile - p.seg_tile0[seg]) * 128 + row;
-            n_ok = r_in_seg < p.seg_rows[seg];
-            n = p.seg_col0[seg] + r_in_seg;
-          }
-          float* xch = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16);
-#pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 32) {
-            const int c = c0 + half * 16;   // this warp's 16 token columns (BN is a multiple of 16)
-            const bool active = c < BN;
-            float v[16];
-            if (active) {
-              tmem_ld16(tbase + c, v);
-              tmem_ld_wait();
-              // the contributors' pieces, in CTA order, up to four per round trip to L2
-              const float4* src = reinterpret_cast<const float4*>(p.partial + ((size_t)c_first * 128 + row) * BN + c);
-              constexpr size_t STRIDE4 = (size_t)128 * BN / 4;
-#pragma unroll 1
-              for (int k = 0; k < n_contrib; k += 4) {
-                float4 a[4][4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                  for (int q = 0; q < 4; ++q)
-                    a[i][q] = k + i < n_contrib ? __ldcg(src + (size_t)(k + i) * STRIDE4 + q)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    v[4 * q + 0] += a[i][q].x;
-                    v[4 * q + 1] += a[i][q].y;
-                    v[4 * q + 2] += a[i][q].z;
-                    v[4 * q + 3] += a[i][q].w;
-                  }
-              }
-            }
-            if (EPI == EPI_SWIGLU_BF16) {
-              // up values (lanes 64..127) go through shared memory to the gate lanes
-              if (active && row >= 64) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) xch[j * 64 + row - 64] = v[j];
-              }
-              epi_sync();
-              if (active && row < 64 && n_ok) {
-                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                  if (c + j < p.act_rows)
-                    o[(size_t)(c + j) * p.ldo + n] = __float2bfloat16_rn(silu_f(v[j]) * xch[j * 64 + row]);
-              }
-              epi_sync();
-            } else if (active && n_ok) {
-              const int nj = p.act_rows - c < 16 ? p.act_rows - c : 16;
-              if (EPI == EPI_RESID_F32) {
-                // all residual loads first (out may alias resid: same element, same thread)
-                float r[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) r[j] = j < nj ? p.resid[(size_t)(c + j) * p.ldr + n] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                  if (j < nj) reinterpret_cast<float*>(p.out)[(size_t)(c + j) * p.ldo + n] = r[j] + v[j];
-              } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  if (j >= nj) break;
-                  const size_t o_idx = (size_t)(c + j) * p.ldo + n;
-                  if (EPI == EPI_BF16)
-                    reinterpret_cast<__nv_bfloat16*>(p.out)[o_idx] = __float2bfloat16_rn(v[j]);
-                  else
-                    reinterpret_cast<float*>(p.out)[o_idx] = v[j];
-                }
-              }
-            }
-          }
-        }
+      if constexpr (SWAP) {
+        streamk_epilogue<BN, EPI>(p, item, tbase, row, half,
+                                  reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16),
+                                  threadIdx.x == 64, &abort_sh, epi_sync);
       } else {
         int mt, wtile;
         tile_coords(p, item.tile, mt, wtile);

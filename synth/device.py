@@ -73,3 +73,28 @@ def random_layer_on_device(w, seed, device="cuda"):
         "wo": n(d, nh * hd), "gate_up": gu, "w1": gu[:f], "w3": gu[f:], "w2": n(d, f),
     }
     return out
+
+
+def random_q4_layer_on_device(w, seed, device="cuda"):
+    """A 4-bit group-64 layer of workload ``w``'s shape drawn on the device, for timing
+    runs: uniform codes (eight per int32 word), scales ~ U(0.3, 0.4) x w_std and
+    offsets = -7.5 x scale (a group of N(0, w_std) weights spans about 15 steps),
+    both bf16 and group-major ``[in / 64][out]``; unit norm weights.  Returns the
+    dict ``layer_weights_q4`` takes: (codes, scales, offsets) per projection."""
+    torch = _torch()
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    d, nh, nkv, hd, f = w.dim, w.n_heads, w.n_kv_heads, w.head_dim, w.ffn_dim
+
+    def q(out_f, in_f):
+        codes = torch.randint(-2 ** 31, 2 ** 31 - 1, (out_f, in_f // 8), generator=g, device=device,
+                              dtype=torch.int64).to(torch.int32)
+        s = (0.3 + 0.1 * torch.rand(in_f // 64, out_f, generator=g, device=device)) * w.w_std
+        return codes, s.to(torch.bfloat16), (-7.5 * s).to(torch.bfloat16)
+
+    return {
+        "attn_norm": torch.ones(d, device=device, dtype=torch.float32),
+        "ffn_norm": torch.ones(d, device=device, dtype=torch.float32),
+        "wq": q(nh * hd, d), "wk": q(nkv * hd, d), "wv": q(nkv * hd, d), "wo": q(d, nh * hd),
+        "w1": q(f, d), "w3": q(f, d), "w2": q(d, f),
+    }

@@ -85,3 +85,22 @@ def test_work_accounting_matches_the_hand_counts():
     assert bench.layer_weight_bytes(W["llama13b_decode"]) == pytest.approx(634.4e6, rel=1e-4)
     assert bench.layer_weight_bytes(W["gqa70b"]) == pytest.approx(1711.3e6, rel=1e-4)
     assert 32 * bench.layer_weight_bytes(W["phi3mini_model"]) == pytest.approx(7247.8e6, rel=1e-4)
+
+
+def test_gpus_n_starts_n_ranks_itself():
+    """``bench.py --gpus 2`` run as a plain command (no torchrun environment)
+    starts two ranks itself; with the host-logic fake workload (gloo, no GPU)
+    rank r spends (1 + r) ms per step, and the line aggregates both ranks'
+    units over the slowest rank's time."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "20",
+                        "--warmup", "3", "--fake-workload"], capture_output=True, text=True, env=env,
+                       timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["steps"] == 20
+    # both ranks' units over the slowest rank's time: rank 1 sleeps 2 ms per step
+    assert d["value"] == pytest.approx(2 * 1000 * 20 / d["slowest_rank_s"])
+    assert d["slowest_rank_s"] >= 20 * 0.002

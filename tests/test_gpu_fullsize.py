@@ -1,16 +1,20 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
 benchmark times, checked on outputs the fp64 oracle can compute row by row.
 
-* 7B-shaped prefill (1 x 2048): sampled query rows (the oracle computes K/V
-  for every row and the rest of the block for the sampled rows only).
+* 7B-shaped prefill (1 x 2048): 64 sampled query rows, four in every
+  128-row tile (the oracle computes K/V for every row and the rest of the
+  block for the sampled rows only).
 * 13B-shaped decode (batch 16, 4096-position cache, interleaved RoPE): three
   decode steps, sampled sequences (sequences are independent).
-* 70B-shaped GQA layer: prefill 2 x 4096 on sampled rows; decode at batch 64
-  on a 4096-position cache, sampled sequences.
-* Phi-3-mini-shaped model: 2 full-width layers against the oracle (logits and
-  argmax ids), and the full 32-layer model against properties that hold at
-  any size: decode with the cache reproduces the prefill's last-row logits,
-  and the ids are the argmax of the logits.
+* 70B-shaped GQA layer: prefill 2 x 4096 on 64 sampled rows of each
+  sequence, two in every 128-row tile; decode at batch 64 on a 4096-position
+  cache, sampled sequences.
+* Phi-3-mini-shaped model at its stated size (32 layers, vocab 32064, batch
+  8, 512-token prompt, 128 teacher-forced decode steps): logits and argmax
+  ids of sequences 0 and 7 against the oracle at all 129 generated
+  positions; also 2 full-width layers against the oracle at a small batch,
+  and properties that hold at any size (decode with the cache reproduces the
+  prefill's last-row logits; the ids are the argmax of the logits).
 
 Tolerances.  At these widths the FFN branch dominates the block output, and
 rounding the GEMM operands to bf16 -- which any bf16 tensor-core block must
@@ -53,12 +57,19 @@ def _check(label, y, yb, ye, absolute_rms=True):
     assert r_rms <= FLOOR_RMS and r_max <= FLOOR_MAX, label
 
 
+def _tile_rows(L, offsets):
+    """Rows at the given offsets inside every 128-row tile of a length-L sequence."""
+    rows = [t * 128 + o for t in range((L + 127) // 128) for o in offsets if t * 128 + o < L]
+    assert len(rows) >= 64
+    return rows
+
+
 def test_llama7b_prefill_full_size_sampled_rows():
     w = synth.WORKLOADS["llama7b_prefill"]
     inp = synth.prefill_inputs(w, with_steps=False)
     run = LayerRun(w, inp.weights, w.batch, w.prefill_len, w.prefill_len)
     y = run.step(inp.x)
-    rows = [0, 1, 127, 128, 129, 1000, 2046, 2047]
+    rows = _tile_rows(w.prefill_len, (0, 37, 90, 127))
     d = oracle_dims(w)
     yb, _ = ob.layer_forward(d, inp.weights, inp.x, ob.KVCache(1, w.n_kv_heads, w.head_dim, w.prefill_len),
                              rounding="bf16", rows=rows)
@@ -97,7 +108,7 @@ def test_gqa70b_prefill_full_size_sampled_rows():
     inp = synth.prefill_inputs(w, with_steps=False)
     run = LayerRun(w, inp.weights, w.batch, w.prefill_len, w.prefill_len)
     y = run.step(inp.x)
-    rows = [0, 129, 4095]
+    rows = _tile_rows(w.prefill_len, (5, 127))
     d = oracle_dims(w)
     yb, _ = ob.layer_forward(d, inp.weights, inp.x, ob.KVCache(2, w.n_kv_heads, w.head_dim, w.prefill_len),
                              rounding="bf16", rows=rows)
@@ -199,3 +210,72 @@ def test_phi3_full_model_properties():
     delta = float(np.max(np.abs(dec_logits - full_logits)))
     ok, n = _ids_agree(dec_ids, full_logits, 2 * delta)
     assert ok
+
+
+def _host_layer(dev):
+    """One device layer's weights as the float32 host arrays the oracle reads (bf16 values, exact)."""
+    return {k: dev[k].float().cpu().numpy() for k in
+            ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w1", "w3", "w2")}
+
+
+def test_phi3_full_model_vs_oracle_sampled_sequences():
+    """The Phi-3-mini-shaped model at its stated size against the fp64 oracle.
+
+    GPU: 32 layers, vocab 32064, batch 8, prefill of a 512-token prompt, then
+    128 teacher-forced decode steps ([HandsOn] 第三章: the module tree, and the
+    next token is the argmax of the last position's scores; [DeepDive] class
+    LLaMA forward), through llama_model_forward, one call per step.
+    Oracle: sequences 0 and 7 only (sequences never mix: pinned by the
+    oracle's batch-permutation test).  With teacher forcing the whole token
+    sequence is known, so the oracle runs each layer once over the 640
+    tokens; its rows 511 ... 639 are the prefill's last row and the 128 decode
+    steps (pinned: decode with the cache reproduces the prefill's rows).
+    Logits at all 129 positions are held to the bf16 floor; ids must agree
+    wherever the oracle's top-2 gap is decisive.
+    """
+    w = synth.WORKLOADS["phi3mini_model"]
+    B, S, n = w.batch, w.prefill_len, w.decode_steps
+    seqs = [0, 7]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed)
+    layers = [sd.random_layer_on_device(w, w.seed + 1 + i) for i in range(w.n_layers)]
+    emb = (torch.randn(w.vocab, w.dim, generator=g, device="cuda") * w.w_std).to(torch.bfloat16)
+    lm = (torch.randn(w.vocab, w.dim, generator=g, device="cuda") * w.w_std).to(torch.bfloat16)
+    fn = torch.ones(w.dim, device="cuda", dtype=torch.float32)
+    prompt, forced = synth.model_tokens(w)
+    run = ModelRun(w, None, B, S + n, S, device_weights=(layers, emb, fn, lm))
+    gl, gi = [], []
+    logits, ids = run.forward(prompt)
+    gl.append(logits[seqs])
+    gi.append(ids[seqs])
+    for t in range(n):
+        logits, ids = run.forward(forced[t][:, None])
+        gl.append(logits[seqs])
+        gi.append(ids[seqs])
+    del run
+    gpu_logits = np.stack(gl, axis=1)                       # [2, 129, vocab]
+    gpu_ids = np.stack(gi, axis=1)                          # [2, 129]
+
+    # oracle over the full teacher-forced sequence of each checked sequence
+    toks = np.concatenate([prompt[seqs], np.stack([f[seqs] for f in forced], axis=1)], axis=1)   # [2, 640]
+    d = oracle_dims(w)
+    E = emb.float().cpu().numpy()
+    xe = ob.embed(E, toks)
+    xb = xe.copy()
+    del E
+    T = S + n
+    for dev in layers:
+        W = _host_layer(dev)
+        xe, _ = ob.layer_forward(d, W, xe, ob.KVCache(2, w.n_kv_heads, w.head_dim, T))
+        xb, _ = ob.layer_forward(d, W, xb, ob.KVCache(2, w.n_kv_heads, w.head_dim, T), rounding="bf16")
+    Wlm = lm.float().cpu().numpy()
+    g_f = fn.cpu().numpy()
+    le = ob.final_logits(xe[:, S - 1:], g_f, Wlm, w.eps)                     # [2, 129, vocab]
+    lb = ob.final_logits(xb[:, S - 1:], g_f, Wlm, w.eps, rounding="bf16")
+    _check("phi3 32-layer logits, seqs 0 and 7, prefill + 128 steps", gpu_logits, lb, le, absolute_rms=False)
+    floor = float(np.max(np.abs(lb - le)))
+    tol = 1e-2 * float(np.sqrt(np.mean(le * le))) + 2 * floor
+    ok, nd = _ids_agree(gpu_ids.reshape(-1), le.reshape(-1, w.vocab), tol)
+    print(f"[fullsize] phi3 32-layer: ids agree on {nd} decisive positions of {gpu_ids.size}")
+    assert ok, "argmax disagreement on decisive positions"
+    assert np.array_equal(gpu_ids, np.argmax(gpu_logits, axis=-1))
