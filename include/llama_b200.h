@@ -131,8 +131,19 @@ llama_status llama_kv_cache_create(const llama_dims* dims, int32_t batch, int32_
  * (rotated) keys and values -- e.g. a synthetic pre-filled cache.
  * Errors: INVALID_ARG (len < 0), CACHE_FULL (len > capacity). */
 llama_status llama_kv_cache_set_length(llama_kv_cache* cache, int32_t len);
-/* Current length (positions filled), or -1 for a null handle. */
+/* Current length (positions filled) when every sequence has the same length;
+ * -2 while the sequences' lengths differ (see llama_kv_cache_lengths); -1 for a
+ * null handle. */
 int32_t llama_kv_cache_length(const llama_kv_cache* cache);
+/* Per-sequence lengths (ragged batch; [MLX-13B] KV 缓存实现片段 keeps one
+ * offset for the whole batch, here each sequence keeps its own): declare
+ * that positions [0, lens[b]) of sequence b hold valid keys and values.
+ *   lens   HOST int32 [batch]
+ * Calls other than llama_layer_forward_ragged need equal lengths and return
+ * INVALID_ARG while they differ.  Errors: INVALID_ARG, CACHE_FULL. */
+llama_status llama_kv_cache_set_lengths(llama_kv_cache* cache, const int32_t* lens);
+/* Copy the per-sequence lengths into lens (HOST int32 [batch]). */
+llama_status llama_kv_cache_lengths(const llama_kv_cache* cache, int32_t* lens);
 int32_t llama_kv_cache_capacity(const llama_kv_cache* cache);
 void llama_kv_cache_destroy(llama_kv_cache* cache);
 
@@ -141,9 +152,9 @@ void llama_kv_cache_destroy(llama_kv_cache* cache);
 /* Bytes of device workspace a layer call with `batch` sequences of up to
  * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
  * The workspace is caller-owned scratch.  Zero-fill it once before its first
- * use: a fixed 1024-byte header at its start (the same for every batch and
+ * use: a fixed 4096-byte header at its start (the same for every batch and
  * seq_len) holds the device status word and the decode GEMMs' per-CTA flags,
- * which every launch leaves at zero; after that the library keeps it consistent,
+ * chunk counters and per-tile counters, which every launch leaves at zero; after that the library keeps it consistent,
  * also when prefill and decode calls of different shapes share it.  After a
  * call that recorded LLAMA_ERR_DEVICE_TIMEOUT, zero-fill it again before
  * reusing it. */
@@ -196,6 +207,30 @@ llama_status llama_layer_prefill(const llama_dims* dims, const llama_layer_weigh
 llama_status llama_layer_decode(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
                                 int32_t batch, const float* x_in, float* x_out, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/* ------------------------------------------------------------------ ragged batches */
+
+/* Workspace bytes of a ragged layer call: `batch` sequences, `total_tokens`
+ * new tokens in all.  0 on invalid arguments (batch > 128 included). */
+size_t llama_workspace_size_ragged(const llama_dims* dims, int32_t batch, int32_t total_tokens);
+
+/* One decoder block over a ragged batch: sequence b brings n_new[b] >= 1 new
+ * tokens at positions lens[b] .. lens[b] + n_new[b] - 1, lens[b] being its own
+ * cache length (llama_kv_cache_set_lengths).  Decode rows (n_new = 1) and
+ * prefill chunks (n_new > 1) may be mixed in one call ([HandsOn] 第三章: the
+ * prefill of a prompt and the token-by-token decode are the same block); the
+ * block never mixes sequences, so each sequence gets exactly what a call on it
+ * alone computes ([DeepDive] LLaMAAttention attends within a batch row).
+ *   n_new   HOST int32 [batch]
+ *   x_in, x_out  device float32 [sum n_new, dim], the rows of sequence 0,
+ *           then of sequence 1, ... (packed, no padding); must not overlap
+ * Each sequence's length advances by n_new[b] when the call is enqueued.
+ * dims->dtype must be LLAMA_BF16; batch <= 128.  Workspace:
+ * llama_workspace_size_ragged(dims, batch, sum n_new).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CACHE_FULL, WORKSPACE_TOO_SMALL, CUDA. */
+llama_status llama_layer_forward_ragged(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                        int32_t batch, const int32_t* n_new, const float* x_in, float* x_out,
+                                        void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ 4-bit group-64 weights (decode) */
 

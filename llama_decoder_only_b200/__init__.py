@@ -26,6 +26,7 @@ __all__ = [
     "model_forward", "device_status", "workspace_offsets", "set_wait_limit_ns", "selftest_wait_timeout",
     "launch_count", "profile_enable", "profile_read", "profile_inflight", "attention_decode_noalloc",
     "sample_top_p", "model_forward_sample", "Q4Weight", "LayerWeightsQ4", "layer_weights_q4", "layer_decode_q4",
+    "workspace_size_ragged", "layer_forward_ragged",
 ]
 
 F32, BF16 = 0, 1
@@ -88,6 +89,10 @@ EXPORTS = {
     "llama_kv_cache_set_length": (_I, [_P, _I]),
     "llama_kv_cache_length": (_I, [_P]),
     "llama_kv_cache_capacity": (_I, [_P]),
+    "llama_kv_cache_set_lengths": (_I, [_P, ctypes.POINTER(_I)]),
+    "llama_kv_cache_lengths": (_I, [_P, ctypes.POINTER(_I)]),
+    "llama_workspace_size_ragged": (_S, [_DP, _I, _I]),
+    "llama_layer_forward_ragged": (_I, [_DP, _WP, _P, _I, ctypes.POINTER(_I), _P, _P, _P, _S, _P]),
     "llama_kv_cache_destroy": (None, [_P]),
     "llama_workspace_size": (_S, [_DP, _I, _I]),
     "llama_device_status": (_I, [_P, _I]),
@@ -200,6 +205,16 @@ class KVCache:
     def set_length(self, n):
         _check(lib().llama_kv_cache_set_length(self.handle, n), "llama_kv_cache_set_length")
 
+    def set_lengths(self, lens):
+        arr = (ctypes.c_int32 * self.batch)(*[int(x) for x in lens])
+        _check(lib().llama_kv_cache_set_lengths(self.handle, arr), "llama_kv_cache_set_lengths")
+
+    @property
+    def lengths(self):
+        arr = (ctypes.c_int32 * self.batch)()
+        _check(lib().llama_kv_cache_lengths(self.handle, arr), "llama_kv_cache_lengths")
+        return list(arr)
+
     def __del__(self):
         h = getattr(self, "handle", None)
         if h is not None and _lib is not None:
@@ -227,6 +242,18 @@ def layer_decode(dims, w, cache, batch, x_in, x_out, ws, stream=None):
     _check(lib().llama_layer_decode(ctypes.byref(dims), ctypes.byref(w), cache.handle, batch, _ptr(x_in),
                                     _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "llama_layer_decode")
+
+
+def workspace_size_ragged(dims, batch, total_tokens):
+    return lib().llama_workspace_size_ragged(ctypes.byref(dims), batch, total_tokens)
+
+
+def layer_forward_ragged(dims, w, cache, n_new, x_in, x_out, ws, stream=None):
+    """One block over a ragged batch: ``n_new[b]`` new tokens of sequence b, packed rows."""
+    arr = (ctypes.c_int32 * len(n_new))(*[int(x) for x in n_new])
+    _check(lib().llama_layer_forward_ragged(ctypes.byref(dims), ctypes.byref(w), cache.handle, len(n_new), arr,
+                                            _ptr(x_in), _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)), "llama_layer_forward_ragged")
 
 
 def layer_decode_q4(dims, w, cache, batch, x_in, x_out, ws, stream=None):

@@ -20,6 +20,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "f32_path.cuh"
+#include "gemm_decode.cuh"
 #include "gemm_q4.cuh"
 #include "gemm_tc.cuh"
 #include "sampling.cuh"
@@ -31,7 +32,8 @@ struct llama_kv_cache {
   llama_dims dims;
   int32_t batch;
   int32_t capacity;
-  int32_t length;
+  int32_t length;              // common length of every sequence; -2 while the lengths differ
+  std::vector<int32_t> lens;   // per-sequence lengths while they differ (empty: all are `length`)
   void* k;
   void* v;
 };
@@ -41,10 +43,17 @@ namespace {
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 constexpr int kMaxSkGrid = 192;     // upper bound on stream-K CTAs (workspace sizing)
 constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
-// workspace header (see plan_ws): status word, then the decode GEMMs' flags
+// workspace header (see plan_ws): status word, the static decode GEMMs' flags,
+// the dynamic decode GEMMs' chunk counters and tile counters
 constexpr size_t kWsFlagsOffset = 256;
-constexpr size_t kWsHeaderBytes = 1024;
-static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsHeaderBytes, "GEMM flags overflow the header");
+constexpr size_t kWsDynCtrOffset = 1024;
+constexpr size_t kWsTileCtrOffset = 2048;
+constexpr size_t kWsHeaderBytes = 4096;
+static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsDynCtrOffset, "GEMM flags overflow their area");
+static_assert(kWsTileCtrOffset + DYN_MAX_TILES * 4 <= kWsHeaderBytes, "tile counters overflow the header");
+// chunks per CTA of the dynamic decode GEMM (more chunks balance better, each
+// partial slot costs 128 x BN fp32 of L2 traffic)
+inline int dyn_chunks_per_cta(int bn) { return bn <= 32 ? 3 : 2; }
 constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K form up to here
 
 // ------------------------------------------------------------------ tracing
@@ -55,12 +64,12 @@ constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K for
 enum KernelKind : int {
   K_RMSNORM = 0, K_GEMM_QKV, K_ROPE_APPEND, K_ATTN_PREFILL, K_ATTN_DECODE, K_ATTN_COMBINE, K_GEMM_O,
   K_GEMM_GATE_UP, K_GEMM_DOWN, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
-  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_SAMPLE, K_COUNT
+  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_SAMPLE, K_SEQTAB, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
   "rmsnorm", "gemm_qkv", "rope_kv_append", "attn_prefill", "attn_decode", "attn_decode_combine", "gemm_o_proj",
   "gemm_gate_up_swiglu", "gemm_down", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
-  "gemm_f32", "attn_f32", "selftest", "sample_top_p"};
+  "gemm_f32", "attn_f32", "selftest", "sample_top_p", "seq_table"};
 
 struct ProfRec {
   cudaEvent_t a, b;
@@ -254,6 +263,40 @@ bool pdl_enabled() {
   return on;
 }
 
+// LLAMA_DECODE_SPLITS=n (n >= 1): use n key splits in the decode attention
+// instead of the heuristic's count (clamped to the kernel's limits).
+int forced_decode_splits() {
+  static const int n = [] {
+    const char* e = std::getenv("LLAMA_DECODE_SPLITS");
+    return e != nullptr ? std::atoi(e) : 0;
+  }();
+  return n;
+}
+
+// Which decode-attention kernel serves (head_dim, GQA group): the TMA-fed
+// tensor-core kernel for groups >= 4 (its 16-row tile fills), the CUDA-core one
+// below that.  LLAMA_DECODE_ATTN=mma | simt forces one of them.
+bool use_decode_mma(int hd, int grp) {
+  static const int forced = [] {
+    const char* e = std::getenv("LLAMA_DECODE_ATTN");
+    if (e == nullptr) return 0;
+    return std::strcmp(e, "mma") == 0 ? 1 : (std::strcmp(e, "simt") == 0 ? 2 : 0);
+  }();
+  if (forced == 1) return true;
+  if (forced == 2) return false;
+  return grp >= 4 && (hd == 64 || hd == 128);
+}
+
+// LLAMA_EARLY_TRIGGER=1: the decode GEMMs, RMSNorm and the split combine signal
+// their dependents at entry instead of at the end of their work.
+int early_trigger() {
+  static const int on = [] {
+    const char* e = std::getenv("LLAMA_EARLY_TRIGGER");
+    return (e != nullptr && e[0] == '1') ? 1 : 0;
+  }();
+  return on;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                      Args&&... args) {
@@ -349,20 +392,30 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // ------------------------------------------------------------------ workspace layout
 
 struct WsLayout {
-  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab;   // layer scratch
+  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab, seqtab;   // layer scratch
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
 
 int swap_bn(int tokens) { return tokens <= 16 ? 16 : tokens <= 32 ? 32 : tokens <= 64 ? 64 : 128; }
 
-// Stream-K partial buffer of one decode GEMM (floats): one [BN][128] piece per CTA.
-size_t sk_partial_floats(int tokens) { return (size_t)kMaxSkGrid * swap_bn(tokens) * 128; }
+// Partial buffer of one decode GEMM (floats): the static form keeps one
+// [128][BN] piece per CTA, the dynamic form two per chunk.
+size_t sk_partial_floats(int tokens) {
+  const int bn = swap_bn(tokens);
+  const size_t stat = (size_t)kMaxSkGrid * bn * 128;
+  const size_t dyn = (size_t)2 * (dyn_chunks_per_cta(bn) * kMaxSkGrid + 1) * bn * 128;
+  return std::max(stat, dyn);
+}
 
-WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
+// ragged_tokens >= 0: a ragged batch of `batch` sequences with that many new
+// tokens in all (seq_len unused); it adds the sequence table at the end.
+WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab, int ragged_tokens = -1) {
   WsLayout w{};
   const size_t es = d.dtype == LLAMA_BF16 ? 2 : 4;
-  const size_t M = (size_t)batch * seq_len;
+  const bool ragged = ragged_tokens >= 0;
+  const size_t M = ragged ? (size_t)ragged_tokens : (size_t)batch * seq_len;
+  const int sk_tokens = ragged ? ragged_tokens : batch;   // token rows of the swapped decode GEMMs
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
   // Fixed header, the same for every (batch, seq_len): the words that must
   // read zero when a launch starts -- the status word and the decode GEMMs'
@@ -381,8 +434,8 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
   w.attn = take(M * (size_t)d.n_heads * d.head_dim * es);
   w.mbuf = take(M * (size_t)d.ffn_dim * es);
   // decode GEMMs (M = batch) and the lm_head on the last rows (M = batch)
-  const bool sk = d.dtype == LLAMA_BF16 && batch <= kSwapMaxTokens;
-  w.partial = take(sk ? sk_partial_floats(batch) * 4 : 0);
+  const bool sk = d.dtype == LLAMA_BF16 && sk_tokens <= kSwapMaxTokens;
+  w.partial = take(sk ? sk_partial_floats(sk_tokens) * 4 : 0);
 
   w.att_ml = take((size_t)batch * d.n_heads * kMaxAttnSplits * 2 * 4);
   w.att_o = take((size_t)batch * d.n_heads * kMaxAttnSplits * d.head_dim * 4);
@@ -396,6 +449,7 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab) {
     w.hl = take((size_t)batch * d.dim * es);
     w.logits = take((size_t)batch * vocab * 4);
   }
+  w.seqtab = take(ragged ? sizeof(SeqTab) : 0);
   w.total = off;
   return w;
 }
@@ -408,37 +462,85 @@ struct WSeg {
   int col0;
 };
 
-template <int BN, bool SWAP, int EPI>
+template <int BN, bool SWAP, int EPI, int KS = 1>
 llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
                             cudaStream_t st, int kind) {
-  using C = GemmCfg<BN, !SWAP>;
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, SWAP, EPI>), C::SMEM_BYTES));
+  using C = GemmCfg<BN, !SWAP, KS>;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, SWAP, EPI, KS>), C::SMEM_BYTES));
   {
     TRACE(kind, st);
     if (SWAP)
-      CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
+      CUDA_TRY(launch_k(gemm_tc_kernel<BN, SWAP, EPI, KS>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2],
+                        p));
     else
-      CUDA_TRY(launch_k_pair(gemm_tc_kernel<BN, SWAP, EPI>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2],
-                             p));
+      CUDA_TRY(launch_k_pair(gemm_tc_kernel<BN, SWAP, EPI, KS>, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1],
+                             w[2], p));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
 
+// LLAMA_DECODE_DYN=0: the decode GEMMs use the static stream-K split instead
+// of dynamically assigned chunks.
+bool decode_dyn() {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_DECODE_DYN");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+template <int BN, int EPI, int KS>
+llama_status launch_gemm_dyn(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
+                             cudaStream_t st, int kind) {
+  using C = GemmCfg<BN, false, KS>;
+  constexpr int SMEM = 1024 + C::STAGES * C::STAGE_BYTES + 512 + C::EXCH_BYTES;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_dyn_kernel<BN, EPI, KS>), SMEM));
+  {
+    TRACE(kind, st);
+    CUDA_TRY(launch_k(gemm_dyn_kernel<BN, EPI, KS>, grid, GEMM_THREADS, SMEM, st, a, w[0], w[1], w[2], p));
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+template <int BN, int KS>
+llama_status launch_gemm_dyn_epi(int epi, const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
+                                 cudaStream_t st, int kind) {
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_dyn<BN, EPI_BF16, KS>(a, w, p, grid, st, kind);
+    case EPI_RESID_F32: return launch_gemm_dyn<BN, EPI_RESID_F32, KS>(a, w, p, grid, st, kind);
+    case EPI_SWIGLU_BF16: return launch_gemm_dyn<BN, EPI_SWIGLU_BF16, KS>(a, w, p, grid, st, kind);
+    case EPI_F32: return launch_gemm_dyn<BN, EPI_F32, KS>(a, w, p, grid, st, kind);
+  }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+// k sub-blocks of 64 per decode GEMM unit (LLAMA_DECODE_KSUB=1 or 2, default 2):
+// 2 makes every stage read 256 contiguous bytes of each weight row.
+int decode_ksub() {
+  static const int ks = [] {
+    const char* e = std::getenv("LLAMA_DECODE_KSUB");
+    return (e != nullptr && e[0] == '1') ? 1 : 2;
+  }();
+  return ks;
+}
+
 // Stream-K scratch of the decode GEMMs: one fp32 piece and one flag per CTA.
 struct SkScratch {
   float* partial;
-  unsigned* flags;
+  unsigned* flags;   // the workspace header's flag area (chunk and tile counters follow it)
 };
 
-template <int BN>
+template <int BN, int KS>
 llama_status launch_gemm_sk(int epi, const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
                             cudaStream_t st, int kind) {
   switch (epi) {
-    case EPI_BF16: return launch_gemm_tc<BN, true, EPI_BF16>(a, w, p, grid, st, kind);
-    case EPI_RESID_F32: return launch_gemm_tc<BN, true, EPI_RESID_F32>(a, w, p, grid, st, kind);
-    case EPI_SWIGLU_BF16: return launch_gemm_tc<BN, true, EPI_SWIGLU_BF16>(a, w, p, grid, st, kind);
-    case EPI_F32: return launch_gemm_tc<BN, true, EPI_F32>(a, w, p, grid, st, kind);
+    case EPI_BF16: return launch_gemm_tc<BN, true, EPI_BF16, KS>(a, w, p, grid, st, kind);
+    case EPI_RESID_F32: return launch_gemm_tc<BN, true, EPI_RESID_F32, KS>(a, w, p, grid, st, kind);
+    case EPI_SWIGLU_BF16: return launch_gemm_tc<BN, true, EPI_SWIGLU_BF16, KS>(a, w, p, grid, st, kind);
+    case EPI_F32: return launch_gemm_tc<BN, true, EPI_F32, KS>(a, w, p, grid, st, kind);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -535,9 +637,10 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
                          void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
                          int kind) {
   const int BN = swap_bn(M);
+  const int KS = decode_ksub();
   GemmParams p{};
   p.K = K;
-  p.num_kb = cdiv(K, 64);
+  p.num_kb = cdiv(K, 64 * KS);
   p.act_rows = M;
   p.m_tiles = 1;
   p.nseg = nseg;
@@ -549,6 +652,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.limit_ns = g_wait_limit_ns.load();
   p.partial = sk.partial;
   p.flags = sk.flags;
+  p.early_trigger = early_trigger();
   CUtensorMap ta, tw[3];
   std::memset(tw, 0, sizeof(tw));
   if (!make_map_2d(&ta, act, K, M, BN)) return LLAMA_ERR_CUDA;
@@ -574,13 +678,44 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.n_tiles = t;
   p.units = (long long)p.n_tiles * p.num_kb;
   // no CTA may have an empty unit range: a tile's finisher waits on every CTA between
-  const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
+  int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
   if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;  // 32-bit unit math
+  if (decode_dyn() && p.n_tiles <= DYN_MAX_TILES) {
+    // chunks of equal units, at most one tile long; the first `grid` are the CTAs' own
+    const long long want = (long long)dyn_chunks_per_cta(BN) * grid;
+    p.chunk_units = (int)std::max<long long>(1, std::min<long long>(p.num_kb, (p.units + want - 1) / want));
+    p.n_chunks = (int)((p.units + p.chunk_units - 1) / p.chunk_units);
+    grid = std::min(grid, p.n_chunks);
+    p.dyn_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsDynCtrOffset);
+    p.tile_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsTileCtrOffset);
+    if (KS == 2) {
+      switch (BN) {
+        case 16: return launch_gemm_dyn_epi<16, 2>(epi, ta, tw, p, grid, st, kind);
+        case 32: return launch_gemm_dyn_epi<32, 2>(epi, ta, tw, p, grid, st, kind);
+        case 64: return launch_gemm_dyn_epi<64, 2>(epi, ta, tw, p, grid, st, kind);
+        default: return launch_gemm_dyn_epi<128, 2>(epi, ta, tw, p, grid, st, kind);
+      }
+    }
+    switch (BN) {
+      case 16: return launch_gemm_dyn_epi<16, 1>(epi, ta, tw, p, grid, st, kind);
+      case 32: return launch_gemm_dyn_epi<32, 1>(epi, ta, tw, p, grid, st, kind);
+      case 64: return launch_gemm_dyn_epi<64, 1>(epi, ta, tw, p, grid, st, kind);
+      default: return launch_gemm_dyn_epi<128, 1>(epi, ta, tw, p, grid, st, kind);
+    }
+  }
+  if (KS == 2) {
+    switch (BN) {
+      case 16: return launch_gemm_sk<16, 2>(epi, ta, tw, p, grid, st, kind);
+      case 32: return launch_gemm_sk<32, 2>(epi, ta, tw, p, grid, st, kind);
+      case 64: return launch_gemm_sk<64, 2>(epi, ta, tw, p, grid, st, kind);
+      default: return launch_gemm_sk<128, 2>(epi, ta, tw, p, grid, st, kind);
+    }
+  }
   switch (BN) {
-    case 16: return launch_gemm_sk<16>(epi, ta, tw, p, grid, st, kind);
-    case 32: return launch_gemm_sk<32>(epi, ta, tw, p, grid, st, kind);
-    case 64: return launch_gemm_sk<64>(epi, ta, tw, p, grid, st, kind);
-    default: return launch_gemm_sk<128>(epi, ta, tw, p, grid, st, kind);
+    case 16: return launch_gemm_sk<16, 1>(epi, ta, tw, p, grid, st, kind);
+    case 32: return launch_gemm_sk<32, 1>(epi, ta, tw, p, grid, st, kind);
+    case 64: return launch_gemm_sk<64, 1>(epi, ta, tw, p, grid, st, kind);
+    default: return launch_gemm_sk<128, 1>(epi, ta, tw, p, grid, st, kind);
   }
 }
 
@@ -634,7 +769,7 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
   const int BN = swap_bn(M);
   GemmParams p{};
   p.K = K;
-  p.num_kb = K / 64;
+  p.num_kb = cdiv(K, 64 * Q4_KG);   // units of four groups; groups past K read as zeros
   p.act_rows = M;
   p.m_tiles = 1;
   p.nseg = nseg;
@@ -646,6 +781,7 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
   p.limit_ns = g_wait_limit_ns.load();
   p.partial = sk.partial;
   p.flags = sk.flags;
+  p.early_trigger = early_trigger();
   CUtensorMap ta;
   Q4Maps maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -655,14 +791,14 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
     {
       const uint64_t dims[2] = {(uint64_t)K / 8, rows};
       const uint64_t strides[1] = {(uint64_t)K / 8 * 4};
-      const uint32_t box[2] = {8, 64};
+      const uint32_t box[2] = {8 * Q4_KG, 64};
       if (!make_map_ex(&maps.codes[s], segs[s].w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, CU_TENSOR_MAP_SWIZZLE_NONE,
                        2, dims, strides, box))
         return LLAMA_ERR_CUDA;
     }
     const uint64_t dims[2] = {rows, groups};
     const uint64_t strides[1] = {rows * 2};
-    const uint32_t box[2] = {64, 1};
+    const uint32_t box[2] = {64, Q4_KG};
     if (!make_map_ex(&maps.scales[s], segs[s].w.scales, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE,
                      2, dims, strides, box) ||
         !make_map_ex(&maps.offsets[s], segs[s].w.offsets, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -697,14 +833,24 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
 
 // ------------------------------------------------------------------ attention launchers
 
+// Ragged batch (tab != nullptr): L is the longest sequence's new tokens, Mtot
+// the packed rows in all and T the most keys any sequence sees; the per-
+// sequence values come from the device table.
 llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int L, int p0,
-                               const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status) {
+                               const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status,
+                               const SeqTab* tab = nullptr, int Mtot = 0, int Tmax = 0) {
   TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_prefill_kernel), ATT_SMEM));
   const int hd = d.head_dim;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
-  const int T = p0 + L;
+  const int T = tab != nullptr ? Tmax : p0 + L;
   CUtensorMap tq, tk, tv;
-  {
+  if (tab != nullptr) {
+    // packed rows of all sequences
+    const uint64_t dims[2] = {(uint64_t)qkvn, (uint64_t)Mtot};
+    const uint64_t strides[1] = {(uint64_t)qkvn * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_map(&tq, qkv, 2, dims, strides, box)) return LLAMA_ERR_CUDA;
+  } else {
     const uint64_t dims[3] = {(uint64_t)qkvn, (uint64_t)L, (uint64_t)B};
     const uint64_t strides[2] = {(uint64_t)qkvn * 2, (uint64_t)L * qkvn * 2};
     const uint32_t box[3] = {64, 128, 1};
@@ -723,12 +869,17 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.nh = d.n_heads;
   p.nkv = d.n_kv_heads;
   p.hd = hd;
-  p.n_qblocks = cdiv(L, 256);
+  // GQA (group >= 2): a CTA takes two query heads of one KV group over 128
+  // query rows, sharing every K/V tile; MHA: one head over 256 query rows
+  p.head_pair = (d.n_heads / d.n_kv_heads) >= 2 ? 1 : 0;
+  p.n_qblocks = cdiv(L, p.head_pair ? 128 : 256);
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
-  dim3 grid(d.n_heads, B, p.n_qblocks);   // heaviest query blocks dispatched first (see the kernel)
+  p.tab = tab;
+  // heaviest query blocks dispatched first (see the kernel)
+  dim3 grid(p.head_pair ? d.n_heads / 2 : d.n_heads, B, p.n_qblocks);
   TRACE(K_ATTN_PREFILL, st);
   CUDA_TRY(launch_k(attn_prefill_kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
   LAUNCH_CHECK();
@@ -752,9 +903,12 @@ llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv
 // Decode attention for GQA groups of 4 or 8 on the tensor cores.
 llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                              int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
-                             float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits) {
+                             float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits,
+                             const SeqTab* tab) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   CUtensorMap tk, tv;
+  // a head_dim of 96 runs as 128: the second 64-dim box reads dims 64..95 and
+  // the bounds fill 96..127 with zeros
   const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)T, (uint64_t)B * d.n_kv_heads};
   const uint64_t strides[2] = {(uint64_t)hd * 2, (uint64_t)capacity * hd * 2};
   const uint32_t box[3] = {64, (uint32_t)DEC_CHUNK, 1};
@@ -763,6 +917,7 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   AttnDecodeMmaParams p{};
   p.qkv = qkv;
   p.ld_qkv = ld_qkv;
+  p.hd = hd;
   p.T = T;
   p.nh = d.n_heads;
   p.nkv = d.n_kv_heads;
@@ -772,9 +927,11 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   p.out = out;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
+  p.tab = tab;
   const int base = B * d.n_kv_heads;
   int splits = cdiv(2 * num_sms(), base);
   splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 256))));
+  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, DEC_CHUNK)));
   splits = std::max(std::min(min_splits, cdiv(T, DEC_CHUNK)), std::min(splits, max_splits));
   int kps = cdiv(cdiv(T, splits), DEC_CHUNK) * DEC_CHUNK;
   splits = cdiv(T, kps);
@@ -784,16 +941,18 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   llama_status r = LLAMA_ERR_UNSUPPORTED;
   {
     TRACE(K_ATTN_DECODE, st);
-    if (hd == 128 && grp == 8) r = launch_attn_decode_mma<128, 8>(tk, tv, p, grid, st);
-    else if (hd == 128 && grp == 4) r = launch_attn_decode_mma<128, 4>(tk, tv, p, grid, st);
-    else if (hd == 64 && grp == 8) r = launch_attn_decode_mma<64, 8>(tk, tv, p, grid, st);
-    else if (hd == 64 && grp == 4) r = launch_attn_decode_mma<64, 4>(tk, tv, p, grid, st);
+#define DEC_MMA_CASE(HD_, G_) \
+    if ((hd == HD_ || (HD_ == 128 && hd == 96)) && grp == G_) r = launch_attn_decode_mma<HD_, G_>(tk, tv, p, grid, st);
+    DEC_MMA_CASE(128, 8) else DEC_MMA_CASE(128, 4) else DEC_MMA_CASE(128, 2) else DEC_MMA_CASE(128, 1)
+    else DEC_MMA_CASE(64, 8) else DEC_MMA_CASE(64, 4) else DEC_MMA_CASE(64, 2) else DEC_MMA_CASE(64, 1)
+#undef DEC_MMA_CASE
   }
   if (r != LLAMA_OK) return r;
   LAUNCH_CHECK();
   if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
-    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
+    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits,
+                      early_trigger()));
   }
   LAUNCH_CHECK();
   return LLAMA_OK;
@@ -801,14 +960,16 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
 
 // Decode attention of one new token per sequence over keys [0, T).  Splits of
 // the key range are chosen by a heuristic, clamped to [min_splits, max_splits].
+// Ragged batch (tab != nullptr): T is the most keys any sequence sees;
+// sequence b sees tab->p0[b] + 1.
 llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                               int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
                               float* part_ml, float* part_o, DevStatus* status, int min_splits = 1,
-                              int max_splits = kMaxAttnSplits) {
+                              int max_splits = kMaxAttnSplits, const SeqTab* tab = nullptr) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
-  if (grp >= 4 && (hd == 64 || hd == 128))
+  if (use_decode_mma(hd, grp))
     return attn_decode_mma(st, d, kc, vc, capacity, B, T, qkv, ld_qkv, out, part_ml, part_o, status, min_splits,
-                           max_splits);
+                           max_splits, tab);
   AttnDecodeParams p{};
   p.qkv = qkv;
   p.ld_qkv = ld_qkv;
@@ -822,6 +983,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   p.part_ml = part_ml;
   p.part_o = part_o;
   p.out = out;
+  p.tab = tab;
   // One CTA per (sequence, KV head) when that alone fills 4 CTAs per SM;
   // otherwise split the keys for about 8 CTAs per SM, >= 64 keys per split
   // (more, shorter splits keep more loads in flight; with a long cache and a
@@ -829,6 +991,7 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   const int base = B * d.n_kv_heads;
   int splits = base >= 4 * num_sms() ? 1 : cdiv(8 * num_sms(), base);
   splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 64))));
+  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, 32)));
   splits = std::max(std::min(min_splits, cdiv(T, 32)), std::min(splits, max_splits));
   int kps = cdiv(T, splits);
   kps = cdiv(kps, 32) * 32;
@@ -848,7 +1011,8 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   LAUNCH_CHECK();
   if (splits > 1) {
     TRACE(K_ATTN_COMBINE, st);
-    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits));
+    CUDA_TRY(launch_k(attn_decode_combine_kernel, dim3(d.n_heads, B), 128, 0, st, part_ml, part_o, out, d.n_heads, hd, splits,
+                      early_trigger()));
     LAUNCH_CHECK();
   }
   return LLAMA_OK;
@@ -863,6 +1027,7 @@ llama_status check_layer_call(const llama_dims* dims, const llama_layer_weights*
   if (kv == nullptr || x_in == nullptr || x_out == nullptr || ws == nullptr) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || L <= 0) return LLAMA_ERR_INVALID_ARG;
   if (!same_dims(*dims, kv->dims) || B != kv->batch) return LLAMA_ERR_INVALID_ARG;
+  if (!kv->lens.empty()) return LLAMA_ERR_INVALID_ARG;   // per-sequence lengths: llama_layer_forward_ragged
   if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(ws)) return LLAMA_ERR_ALIGNMENT;
   const size_t xb = (size_t)B * L * dims->dim * 4;
   if (overlap(x_in, xb, x_out, xb)) return LLAMA_ERR_INVALID_ARG;
@@ -895,7 +1060,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     {
       TRACE(K_RMSNORM, st);
       // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
-      const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta};
+      const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta, early_trigger()};
       CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
                         d.eps, rt));
     }
@@ -925,7 +1090,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
         TRACE(K_ROPE_APPEND, st);
         CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
                           reinterpret_cast<bf*>(kv->v), L, p0, nh, nkv, hd, kv->capacity, d.rope_theta,
-                          d.rope_style));
+                          d.rope_style, static_cast<const SeqTab*>(nullptr)));
       }
       LAUNCH_CHECK();
     }
@@ -945,7 +1110,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     {
       TRACE(K_RMSNORM, st);
       CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim,
-                        d.eps, RopeTab{}));
+                        d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
     }
     LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
@@ -988,7 +1153,8 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     {
       TRACE(K_ROPE_APPEND, st);
       rope_append_kernel<float><<<M, 256, 0, st>>>(qkv, static_cast<float*>(kv->k), static_cast<float*>(kv->v), L,
-                                                    p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style);
+                                                    p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style,
+                                                    nullptr);
     }
     LAUNCH_CHECK();
     const int Tmax = p0 + L;
@@ -1032,6 +1198,108 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
   return LLAMA_OK;
 }
 
+// ------------------------------------------------------------------ one block, ragged batch
+
+// Enqueue one block over a ragged batch: sequence b brings n_new[b] >= 1 new
+// tokens, packed in sequence order in x_in, at positions from its own cache
+// length on.  Decode rows and prefill chunks may be mixed: with every
+// n_new[b] == 1 the split-KV decode attention runs, otherwise the flash
+// attention in its varlen form (a one-token sequence is a one-row query block).
+llama_status run_layer_ragged(const llama_dims& d, const llama_layer_weights& w, llama_kv_cache* kv, int B,
+                              const int32_t* n_new, const float* x_in, float* x_out, uint8_t* ws,
+                              const WsLayout& lay, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+  const int qkvn = (nh + 2 * nkv) * hd;
+  SeqTab tab{};
+  tab.n = B;
+  int M = 0, maxL = 0, Tmax = 0;
+  bool all_one = true;
+  for (int b = 0; b < B; ++b) {
+    const int p0 = kv->lens.empty() ? kv->length : kv->lens[b];
+    tab.start[b] = M;
+    tab.len[b] = n_new[b];
+    tab.p0[b] = p0;
+    M += n_new[b];
+    maxL = std::max(maxL, n_new[b]);
+    Tmax = std::max(Tmax, p0 + n_new[b]);
+    all_one = all_one && n_new[b] == 1;
+  }
+  SeqTab* dtab = reinterpret_cast<SeqTab*>(ws + lay.seqtab);
+  {
+    TRACE(K_SEQTAB, st);
+    CUDA_TRY(launch_k(seqtab_kernel, 1, 128, 0, st, tab, dtab));
+  }
+  LAUNCH_CHECK();
+  const bool sk = M <= kSwapMaxTokens;   // few token rows: the swapped stream-K GEMMs
+  bf* qkv = reinterpret_cast<bf*>(ws + lay.qkv);
+  bf* h = reinterpret_cast<bf*>(ws + lay.h);
+  bf* att = reinterpret_cast<bf*>(ws + lay.attn);
+  bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
+  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
+  {
+    TRACE(K_RMSNORM, st);
+    CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
+                      d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
+  }
+  LAUNCH_CHECK();
+  const size_t rb = (size_t)d.dim * 2;
+  WSeg segs[3];
+  int nseg;
+  if (w.wk == (const uint8_t*)w.wq + (size_t)nh * hd * rb && w.wv == (const uint8_t*)w.wk + (size_t)nkv * hd * rb) {
+    segs[0] = {w.wq, qkvn, 0};
+    nseg = 1;
+  } else {
+    segs[0] = {w.wq, nh * hd, 0};
+    segs[1] = {w.wk, nkv * hd, nh * hd};
+    segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
+    nseg = 3;
+  }
+  TRY(gemm_bf16(st, sk, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
+  {
+    TRACE(K_ROPE_APPEND, st);
+    CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
+                      reinterpret_cast<bf*>(kv->v), 1, 0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style,
+                      static_cast<const SeqTab*>(dtab)));
+  }
+  LAUNCH_CHECK();
+  if (all_one) {
+    TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, Tmax, qkv, qkvn, att,
+                         reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o), status,
+                         1, kMaxAttnSplits, dtab));
+  } else {
+    TRY(attn_prefill_bf16(st, d, kv, B, maxL, 0, qkv, att, status, dtab, M, Tmax));
+  }
+  WSeg so{w.wo, d.dim, 0};
+  TRY(gemm_bf16(st, sk, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status, K_GEMM_O));
+  {
+    TRACE(K_RMSNORM, st);
+    CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim,
+                      d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
+  }
+  LAUNCH_CHECK();
+  WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
+  TRY(gemm_bf16(st, sk, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
+                K_GEMM_GATE_UP));
+  WSeg sd{w.w2, d.dim, 0};
+  TRY(gemm_bf16(st, sk, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
+                K_GEMM_DOWN));
+  // every sequence's length advances by its new tokens
+  std::vector<int32_t> lens(B);
+  for (int b = 0; b < B; ++b) lens[b] = tab.p0[b] + n_new[b];
+  bool same = true;
+  for (int b = 1; b < B; ++b) same = same && lens[b] == lens[0];
+  if (same) {
+    kv->length = lens[0];
+    kv->lens.clear();
+  } else {
+    kv->length = -2;
+    kv->lens = std::move(lens);
+  }
+  return LLAMA_OK;
+}
+
 // ------------------------------------------------------------------ one block, 4-bit weights (decode)
 
 llama_status check_q4(const llama_q4_weight& w) {
@@ -1070,7 +1338,7 @@ llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_
   {
     TRACE(K_RMSNORM, st);
     CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, B, d.dim,
-                      d.eps, RopeTab{}));
+                      d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
   }
   LAUNCH_CHECK();
   const Q4Seg sq[3] = {{w.wq, nh * hd, 0}, {w.wk, nkv * hd, nh * hd}, {w.wv, nkv * hd, (nh + nkv) * hd}};
@@ -1078,7 +1346,8 @@ llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_
   {
     TRACE(K_ROPE_APPEND, st);
     CUDA_TRY(launch_k(rope_append_kernel<bf>, B, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
-                      reinterpret_cast<bf*>(kv->v), 1, p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style));
+                      reinterpret_cast<bf*>(kv->v), 1, p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style,
+                      static_cast<const SeqTab*>(nullptr)));
   }
   LAUNCH_CHECK();
   TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
@@ -1088,7 +1357,7 @@ llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_
   {
     TRACE(K_RMSNORM, st);
     CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, B, d.dim,
-                      d.eps, RopeTab{}));
+                      d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
   }
   LAUNCH_CHECK();
   const Q4Seg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
@@ -1203,6 +1472,31 @@ llama_status llama_kv_cache_set_length(llama_kv_cache* c, int32_t len) {
   if (c == nullptr || len < 0) return LLAMA_ERR_INVALID_ARG;
   if (len > c->capacity) return LLAMA_ERR_CACHE_FULL;
   c->length = len;
+  c->lens.clear();
+  return LLAMA_OK;
+}
+
+llama_status llama_kv_cache_set_lengths(llama_kv_cache* c, const int32_t* lens) {
+  if (c == nullptr || lens == nullptr) return LLAMA_ERR_INVALID_ARG;
+  bool same = true;
+  for (int b = 0; b < c->batch; ++b) {
+    if (lens[b] < 0) return LLAMA_ERR_INVALID_ARG;
+    if (lens[b] > c->capacity) return LLAMA_ERR_CACHE_FULL;
+    same = same && lens[b] == lens[0];
+  }
+  if (same) {
+    c->length = lens[0];
+    c->lens.clear();
+  } else {
+    c->length = -2;
+    c->lens.assign(lens, lens + c->batch);
+  }
+  return LLAMA_OK;
+}
+
+llama_status llama_kv_cache_lengths(const llama_kv_cache* c, int32_t* lens) {
+  if (c == nullptr || lens == nullptr) return LLAMA_ERR_INVALID_ARG;
+  for (int b = 0; b < c->batch; ++b) lens[b] = c->lens.empty() ? c->length : c->lens[b];
   return LLAMA_OK;
 }
 
@@ -1261,7 +1555,7 @@ llama_status llama_layer_decode_q4(const llama_dims* dims, const llama_layer_wei
   if (cache == nullptr || x_in == nullptr || x_out == nullptr || workspace == nullptr || batch <= 0)
     return LLAMA_ERR_INVALID_ARG;
   if (batch > kSwapMaxTokens) return LLAMA_ERR_UNSUPPORTED;
-  if (!same_dims(*dims, cache->dims) || batch != cache->batch) return LLAMA_ERR_INVALID_ARG;
+  if (!same_dims(*dims, cache->dims) || batch != cache->batch || !cache->lens.empty()) return LLAMA_ERR_INVALID_ARG;
   if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(workspace)) return LLAMA_ERR_ALIGNMENT;
   const size_t xb = (size_t)batch * dims->dim * 4;
   if (overlap(x_in, xb, x_out, xb)) return LLAMA_ERR_INVALID_ARG;
@@ -1270,6 +1564,38 @@ llama_status llama_layer_decode_q4(const llama_dims* dims, const llama_layer_wei
   if (ws_bytes < lay.total) return LLAMA_ERR_WORKSPACE_TOO_SMALL;
   return run_layer_decode_q4(*dims, *w, cache, batch, x_in, x_out, static_cast<uint8_t*>(workspace), lay,
                              static_cast<cudaStream_t>(stream));
+}
+
+size_t llama_workspace_size_ragged(const llama_dims* dims, int32_t batch, int32_t total_tokens) {
+  if (check_dims(dims) != LLAMA_OK || batch <= 0 || batch > kMaxRagged || total_tokens < batch) return 0;
+  return plan_ws(*dims, batch, 1, 0, total_tokens).total;
+}
+
+llama_status llama_layer_forward_ragged(const llama_dims* dims, const llama_layer_weights* w, llama_kv_cache* cache,
+                                        int32_t batch, const int32_t* n_new, const float* x_in, float* x_out,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  TRY(check_dims(dims));
+  TRY(check_weights(w));
+  if (cache == nullptr || n_new == nullptr || x_in == nullptr || x_out == nullptr || workspace == nullptr)
+    return LLAMA_ERR_INVALID_ARG;
+  if (dims->dtype != LLAMA_BF16) return LLAMA_ERR_UNSUPPORTED;
+  if (batch <= 0 || batch != cache->batch || !same_dims(*dims, cache->dims)) return LLAMA_ERR_INVALID_ARG;
+  if (batch > kMaxRagged) return LLAMA_ERR_UNSUPPORTED;
+  long long M = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (n_new[b] < 1) return LLAMA_ERR_INVALID_ARG;
+    const long long p0 = cache->lens.empty() ? cache->length : cache->lens[b];
+    if (p0 + n_new[b] > cache->capacity) return LLAMA_ERR_CACHE_FULL;
+    M += n_new[b];
+  }
+  if (M > (1LL << 30)) return LLAMA_ERR_UNSUPPORTED;
+  if (!aligned16(x_in) || !aligned16(x_out) || !aligned16(workspace)) return LLAMA_ERR_ALIGNMENT;
+  const size_t xb = (size_t)M * dims->dim * 4;
+  if (overlap(x_in, xb, x_out, xb)) return LLAMA_ERR_INVALID_ARG;
+  const WsLayout lay = plan_ws(*dims, batch, 1, 0, (int)M);
+  if (ws_bytes < lay.total) return LLAMA_ERR_WORKSPACE_TOO_SMALL;
+  return run_layer_ragged(*dims, *w, cache, batch, n_new, x_in, x_out, static_cast<uint8_t*>(workspace), lay,
+                          static_cast<cudaStream_t>(stream));
 }
 
 size_t llama_model_workspace_size(const llama_model* m, int32_t batch, int32_t seq_len) {
@@ -1332,7 +1658,7 @@ llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, 
   const int len0 = caches[0] ? caches[0]->length : -1;
   for (int l = 0; l < m->n_layers; ++l) {
     llama_kv_cache* c = caches[l];
-    if (c == nullptr || !same_dims(c->dims, d) || c->batch != batch || c->length != len0)
+    if (c == nullptr || !same_dims(c->dims, d) || c->batch != batch || c->length != len0 || !c->lens.empty())
       return LLAMA_ERR_INVALID_ARG;
     if ((long long)c->length + seq_len > c->capacity) return LLAMA_ERR_CACHE_FULL;
     TRY(check_weights(&m->layers[l]));
@@ -1376,7 +1702,7 @@ llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, 
     {
       TRACE(K_RMSNORM, st);
       CUDA_TRY(launch_k(rmsnorm_kernel<__nv_bfloat16>, batch, rmsnorm_threads(d.dim), 0, st, xl, d.dim,
-                        m->final_norm, hl, batch, d.dim, d.eps, RopeTab{}));
+                        m->final_norm, hl, batch, d.dim, d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
     }
     LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};

@@ -25,6 +25,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ragged.cuh"
 
 namespace llama {
 
@@ -36,11 +37,19 @@ struct AttnPrefillParams {
   int L;         // new tokens per sequence
   int p0;        // position of token 0 (cache length before the call)
   int nh, nkv, hd;
-  int n_qblocks; // blocks of 256 query rows (two 128-row tiles)
+  int n_qblocks; // query blocks per (head pair or head, sequence)
+  // 1: a CTA takes two query heads of one KV group over the same 128 query
+  // rows (GQA, group >= 2: every K/V tile serves both heads); 0: one head over
+  // 256 query rows (two 128-row tiles)
+  int head_pair;
   float scale_log2;   // log2(e) / sqrt(hd)
-  __nv_bfloat16* out; // [B*L, nh*hd]
+  __nv_bfloat16* out; // [B*L, nh*hd] (ragged: [sum of new tokens, nh*hd])
   DevStatus* status;
   unsigned long long limit_ns;
+  // ragged batch: sequence b has tab->len[b] new tokens at packed rows
+  // tab->start[b] .., positions tab->p0[b] ..; tmQ is then a 2-D map over the
+  // packed rows.  nullptr: every sequence has L tokens at positions p0 ...
+  const SeqTab* tab;
 };
 
 constexpr int ATT_REGION = 128 * 128;           // bytes of a [128 rows x 64 bf16] region
@@ -81,17 +90,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // with the block index in z every (head, sequence) starts its heaviest
   // (latest) block in the first wave and the light ones fill in behind.
   const int qb = p.n_qblocks - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int g = h / (p.nh / p.nkv);
+  const int b = blockIdx.y;
+  const bool hp = p.head_pair != 0;
+  // query tile t: head h_t, rows q_row0 + qoff_t of the sequence
+  const int h0 = hp ? 2 * blockIdx.x : blockIdx.x;
+  const int g = h0 / (p.nh / p.nkv);             // both heads of a pair share it
   const int hd = p.hd;
   const int nreg = hd > 64 ? 2 : 1;             // 64-column regions per head row
   const int hd_pad = nreg * 64;
-  const int q_row0 = qb * 256;
-  const bool q1_valid = q_row0 + 128 < p.L;
+  const int q_row0 = qb * (hp ? 128 : 256);
+  const int qoff1 = hp ? 0 : 128;                // rows of tile 1 after q_row0
+  // this sequence's new tokens, their first position and first packed row
+  int Ls = p.L, p0s = p.p0, row_base = b * p.L;
+  if (p.tab != nullptr) {
+    pdl_wait();   // the table is written by an earlier kernel
+    Ls = p.tab->len[b];
+    p0s = p.tab->p0[b];
+    row_base = p.tab->start[b];
+  }
+  const bool q0_valid = q_row0 < Ls;
+  const bool q1_valid = q_row0 + qoff1 < Ls;
   // kv tiles with any key visible to tile t (0 for an empty tile)
-  const int last0 = min(p.L, q_row0 + 128) - 1;
-  const int n_kv0 = (p.p0 + last0) / 128 + 1;
-  const int n_kv1 = q1_valid ? (p.p0 + min(p.L, q_row0 + 256) - 1) / 128 + 1 : 0;
+  const int last0 = min(Ls, q_row0 + 128) - 1;
+  const int n_kv0 = q0_valid ? (p0s + last0) / 128 + 1 : 0;
+  const int n_kv1 = q1_valid ? (p0s + min(Ls, q_row0 + qoff1 + 128) - 1) / 128 + 1 : 0;
   const int n_kv = max(n_kv0, n_kv1);
 
   const uint32_t bar0 = smem_u32(bars);
@@ -140,12 +162,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int last_fill[ATT_SLOTS] = {-1, -1, -1};
-      const int nq = q1_valid ? 2 : 1;
+      const int nq = q1_valid ? 2 : (q0_valid ? 1 : 0);
       mbar_arrive_expect_tx(q_full, nq * nreg * ATT_REGION);
       for (int t = 0; t < nq; ++t)
-        for (int r = 0; r < nreg; ++r)
-          tma_load_3d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64,
-                      q_row0 + t * 128, b);
+        for (int r = 0; r < nreg; ++r) {
+          const int col = (h0 + (hp ? t : 0)) * hd + r * 64, row = q_row0 + (t ? qoff1 : 0);
+          if (p.tab != nullptr)
+            tma_load_2d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, col, row_base + row);
+          else
+            tma_load_3d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, col, row, b);
+        }
       const int zkv = b * p.nkv + g;
       for (int f = 0; f < 2 * n_kv; ++f) {   // fill f: K_{f/2} (f even) or V_{f/2} (f odd)
         const int s = f % ATT_SLOTS;
@@ -227,9 +253,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int t = (warp - 2) >> 2;             // query tile of this warpgroup
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int tok = q_row0 + t * 128 + row;    // token within the sequence
-    const int pos = p.p0 + tok;
-    const int pos_min = p.p0 + q_row0 + t * 128;
+    const int tok = q_row0 + (t ? qoff1 : 0) + row;   // token within the sequence
+    const int pos = p0s + tok;
+    const int pos_min = p0s + q_row0 + (t ? qoff1 : 0);
+    const int h = h0 + (hp ? t : 0);                     // this tile's query head
     const int my_kv = t == 0 ? n_kv0 : n_kv1;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
@@ -349,12 +376,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (ok && my_kv > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done(t), (my_kv - 1) & 1, wc, 12))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((size_t)b * p.L + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
+      __nv_bfloat16* orow = p.out + ((size_t)row_base + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
       for (int c = 0; c < hd_pad; c += 32) {
         float v[32];
         tmem_ld32(tO + c, v);
         tmem_ld_wait();
-        if (tok < p.L) {
+        if (tok < Ls) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (c + 8 * q < hd) {
@@ -392,6 +419,7 @@ struct AttnDecodeParams {
   float* part_ml;             // [B*nh][splits][2]   (splits > 1)
   float* part_o;              // [B*nh][splits][hd]
   __nv_bfloat16* out;         // [B, nh*hd]
+  const SeqTab* tab;          // ragged: sequence b sees tab->p0[b] + 1 keys; nullptr: all see T
 };
 
 // Log-sum-exp merge of the `splits` partial results of query head hq of
@@ -428,8 +456,9 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPK, sub = lane % LPK;
+  const int T = p.tab != nullptr ? p.tab->p0[b] + 1 : p.T;
   const int j0 = split * p.keys_per_split;
-  const int j1 = min(p.T, j0 + p.keys_per_split);
+  const int j1 = min(T, j0 + p.keys_per_split);
 
   float q[G][VEC];
 #pragma unroll
@@ -603,6 +632,8 @@ constexpr int DEC_CHUNK = 64;                          // keys per chunk
 constexpr int DEC_STAGES = 4;
 constexpr int DEC_REGION = DEC_CHUNK * 128;            // [64 keys x 64 dims] bf16 = 8 KB
 
+// HD: head dimension as laid out in shared memory (64 or 128); a head_dim of 96
+// runs as 128 with dims 96..127 zero-filled by the TMA bounds (no HBM bytes).
 template <int HD>
 struct DecMmaCfg {
   static constexpr int NREG = HD / 64;                 // 64-dim regions per key row
@@ -636,6 +667,7 @@ __device__ __forceinline__ uint32_t sw128(int key, int chunk) {
 struct AttnDecodeMmaParams {
   const __nv_bfloat16* qkv;
   int ld_qkv;
+  int hd;                     // head_dim in memory (<= the kernel's HD; 96 runs as 128)
   int T;
   int nh, nkv;
   int splits, keys_per_split;
@@ -645,6 +677,7 @@ struct AttnDecodeMmaParams {
   __nv_bfloat16* out;
   DevStatus* status;
   unsigned long long limit_ns;
+  const SeqTab* tab;          // ragged: sequence b sees tab->p0[b] + 1 keys; nullptr: all see T
 };
 
 template <int HD, int G>
@@ -664,8 +697,10 @@ __global__ void __launch_bounds__(160, 1)
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.tab != nullptr) pdl_wait();   // the ragged table is written by an earlier kernel
+  const int T = p.tab != nullptr ? p.tab->p0[b] + 1 : p.T;
   const int j0 = split * p.keys_per_split;
-  const int j1 = min(p.T, j0 + p.keys_per_split);
+  const int j1 = min(T, j0 + p.keys_per_split);
   const int n_chunks = j1 > j0 ? (j1 - j0 + DEC_CHUNK - 1) / DEC_CHUNK : 0;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -710,18 +745,20 @@ __global__ void __launch_bounds__(160, 1)
     // Q as A fragments: rows = query heads of the group (rows >= G are zero)
     uint32_t qa[KS][4];
     {
-      const __nv_bfloat16* qrow0 = p.qkv + (size_t)b * p.ld_qkv + (size_t)(g * G) * HD;
+      const int hdm = p.hd;
+      const __nv_bfloat16* qrow0 = p.qkv + (size_t)b * p.ld_qkv + (size_t)(g * G) * hdm;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         const int k0 = ks * 16 + qd * 2;
         uint32_t lo = 0, hi = 0, lo8 = 0, hi8 = 0;
-        if (r0 < G) {
-          lo = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * HD + k0);
-          lo8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * HD + k0 + 8);
+        // dims past head_dim stay zero (head_dim is a multiple of 16 here)
+        if (r0 < G && k0 < hdm) {
+          lo = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * hdm + k0);
+          lo8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * hdm + k0 + 8);
         }
-        if (r0 + 8 < G) {
-          hi = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * HD + k0);
-          hi8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * HD + k0 + 8);
+        if (r0 + 8 < G && k0 < hdm) {
+          hi = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * hdm + k0);
+          hi8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * hdm + k0 + 8);
         }
         qa[ks][0] = lo;
         qa[ks][1] = hi;
@@ -844,8 +881,9 @@ __global__ void __launch_bounds__(160, 1)
   }
   __syncthreads();
   pdl_trigger();
-  for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
-    const int gi = idx / HD, d = idx % HD;
+  const int hdm = p.hd;
+  for (int idx = threadIdx.x; idx < G * hdm; idx += blockDim.x) {
+    const int gi = idx / hdm, d = idx % hdm;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][gi]);
@@ -860,10 +898,10 @@ __global__ void __launch_bounds__(160, 1)
     }
     const int hq = g * G + gi;
     if (p.splits == 1) {
-      p.out[(size_t)b * p.nh * HD + (size_t)hq * HD + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+      p.out[(size_t)b * p.nh * hdm + (size_t)hq * hdm + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
     } else {
       const size_t r = ((size_t)b * p.nh + hq) * p.splits + split;
-      p.part_o[r * HD + d] = O;
+      p.part_o[r * hdm + d] = O;
       if (d == 0) {
         p.part_ml[2 * r] = M;
         p.part_ml[2 * r + 1] = Lsum;
@@ -874,7 +912,9 @@ __global__ void __launch_bounds__(160, 1)
 
 // out[b, h*hd + d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s
 __global__ void attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
-                                           __nv_bfloat16* __restrict__ out, int nh, int hd, int splits) {
+                                           __nv_bfloat16* __restrict__ out, int nh, int hd, int splits,
+                                           int early_trigger) {
+  if (early_trigger) pdl_trigger();   // the next kernel is the o_proj GEMM
   pdl_wait();
   combine_head(part_ml, part_o, out, nh, hd, splits, blockIdx.y, blockIdx.x);
 }

@@ -9,18 +9,20 @@
 // the weight fills the MMA's M = 128, the few token rows are N = BN, the
 // (weight tile, 64-wide k-block) units are split evenly over the CTAs and the
 // CTA that ends a tile adds the others' pieces and applies the epilogue
-// (streamk_epilogue).  What changes is the main loop -- one k-block of a
-// weight tile is exactly one quantisation group:
-//   warp 0       TMA producer: packed codes (128 rows x 32 B), the group's
-//                128 scales and 128 offsets, and the activation tile; the
-//                weight parts are issued before the PDL wait (they do not
-//                depend on the previous kernel), the activations after it;
-//   warps 10-13  dequantisers: thread r owns weight row r of the tile; it
-//                turns its 64 codes into bf16 w = fma(q, s, b) (bf16x2 FMA,
-//                one rounding of the exact value) and writes them into a
-//                128-byte-swizzled K-major A tile, the layout the MMA reads;
-//   warp 1       MMA issuer: 4 x tcgen05.mma (M 128, N BN, K 16) per unit
-//                from the dequantised A tile and the activation tile;
+// (streamk_epilogue).  What changes is the main loop -- a k-block of a
+// weight tile is four quantisation groups:
+//   warp 0       TMA producer: per unit of 4 groups (256 inputs), the packed
+//                codes (128 rows x 128 contiguous bytes), the groups' scales
+//                and offsets, and the activation tiles; the weight parts are
+//                issued before the PDL wait (they do not depend on the
+//                previous kernel), the activations after it;
+//   warps 10-17  dequantisers: thread (row r, half h) owns groups h and h + 2
+//                of weight row r; it turns 64 codes into bf16 w = fma(q, s, b)
+//                (bf16x2 FMA, one rounding of the exact value) and writes them
+//                into a 128-byte-swizzled K-major A tile per group, the layout
+//                the MMA reads;
+//   warp 1       MMA issuer: 4 x tcgen05.mma (M 128, N BN, K 16) per group
+//                from the dequantised tile and the group's activation tile;
 //   warps 2-9    stream-K epilogue.
 // HBM moves 32 B of codes + 4 B of scale/offset per 64 weights: 0.5625 B per
 // weight against 2 B in bf16.
@@ -30,34 +32,40 @@
 
 namespace llama {
 
-constexpr int Q4_CONV_WARPS = 4;
-constexpr int Q4_THREADS = GEMM_THREADS + 32 * Q4_CONV_WARPS;   // 448
+constexpr int Q4_CONV_WARPS = 8;
+constexpr int Q4_THREADS = GEMM_THREADS + 32 * Q4_CONV_WARPS;   // 576
 constexpr int Q4_CONV_WARP0 = GEMM_THREADS / 32;                // 10
+constexpr int Q4_KG = 4;                                        // quantisation groups (64 inputs) per unit
 
+// One unit = one weight tile (128 rows) x Q4_KG groups: a stage reads 128
+// contiguous bytes of codes of every row.
 template <int BN>
 struct Q4Cfg {
-  static constexpr int ACT_BYTES = BN * 64 * 2;                 // activation tile, 128-byte swizzled
-  static constexpr int CODE_BYTES = 128 * 32;                   // 128 rows x 8 words
-  static constexpr int SO_BYTES = 128 * 2;                      // 128 bf16 scales (or offsets)
+  static constexpr int ACT_SUB = BN * 64 * 2;                   // activation sub-tile of one group, swizzled
+  static constexpr int ACT_BYTES = Q4_KG * ACT_SUB;
+  static constexpr int CODE_BYTES = 128 * 32 * Q4_KG;           // 128 rows x 8 words per group
+  static constexpr int SO_BYTES = 128 * 2 * Q4_KG;              // bf16 scales (or offsets): [half][group][64]
   static constexpr int STAGE_RAW = ACT_BYTES + CODE_BYTES + 2 * SO_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int A_BYTES = 128 * 128;                     // dequantised tile, 128 rows x 64 bf16
-  static constexpr int LSTAGES = 8;                             // load ring
-  static constexpr int ASTAGES = (200 * 1024 - LSTAGES * STAGE) / A_BYTES > 6 ? 6
-                                 : (200 * 1024 - LSTAGES * STAGE) / A_BYTES;
+  static constexpr int A_BYTES = 128 * 128;                     // dequantised tile of one group
+  static constexpr int LS_RAW = (120 * 1024) / STAGE;
+  static constexpr int LSTAGES = LS_RAW < 2 ? 2 : (LS_RAW > 4 ? 4 : LS_RAW);
+  static constexpr int AS_RAW = (204 * 1024 - LSTAGES * STAGE) / A_BYTES;
+  static constexpr int ASTAGES = AS_RAW > 8 ? 8 : AS_RAW;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : 256;
   static constexpr int EXCH_BYTES = 2 * 64 * 16 * 4;
   static constexpr int SMEM_BYTES = 1024 + LSTAGES * STAGE + ASTAGES * A_BYTES + 512 + EXCH_BYTES;
   static_assert(ASTAGES >= 2, "dequantised tile ring too small");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// Tensor maps of one weight segment: codes uint32 [rows][K/8] (box 8 x 64),
-// scales and offsets bf16 [K/64][rows] (box 64 x 1).
+// Tensor maps of one weight segment: codes uint32 [rows][K/8] (box 32 words
+// x 64 rows), scales and offsets bf16 [K/64][rows] (box 64 rows x 4 groups).
 struct Q4Maps {
   CUtensorMap codes[3], scales[3], offsets[3];
 };
 
-// 64 codes of one row (8 words) -> 64 bf16 weights s*q + b into row r of a
+// 8 words (64 codes) of one row -> 64 bf16 weights s*q + b into row r of a
 // 128-byte-swizzled K-major tile.
 __device__ __forceinline__ void q4_dequant_row(const uint32_t* words, __nv_bfloat16 s, __nv_bfloat16 b,
                                                uint8_t* a_tile, int r) {
@@ -94,7 +102,7 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
     gemm_q4_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ Q4Maps maps,
                    const GemmParams p) {
   using C = Q4Cfg<BN>;
-  constexpr int LS = C::LSTAGES, AS = C::ASTAGES;
+  constexpr int LS = C::LSTAGES, AS = C::ASTAGES, KG = Q4_KG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_ring = smem + LS * C::STAGE;
@@ -105,8 +113,9 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
-  // wfull: codes + scales + offsets landed; xfull: activations landed;
-  // lempty: the stage's MMAs are done; afull / aempty: dequantised tile ring
+  // wfull: codes + scales + offsets of a unit landed; xfull: its activations
+  // landed; lempty: the unit's MMAs are done; afull / aempty: one dequantised
+  // group tile of the ring (tile t = unit * KG + group)
   auto wfull = [&](int s) { return bar0 + 8u * s; };
   auto xfull = [&](int s) { return bar0 + 8u * (LS + s); };
   auto lempty = [&](int s) { return bar0 + 8u * (2 * LS + s); };
@@ -116,7 +125,7 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
   auto acce_bar = [&](int b) { return bar0 + 8u * (3 * LS + 2 * AS + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (3 * LS + 2 * AS + 4);
   const uint32_t epi_bar = bar0 + 8u * (3 * LS + 2 * AS + 5);
-  static_assert(8 * (3 * LS + 2 * 6 + 6) <= 512, "barrier area");
+  static_assert(8 * (3 * LS + 2 * AS + 6) <= 512, "barrier area");
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
       mbar_init(lempty(s), 1);
     }
     for (int a = 0; a < AS; ++a) {
-      mbar_init(afull(a), Q4_CONV_WARPS);
+      mbar_init(afull(a), Q4_CONV_WARPS / 2);   // the four warps that own a group's rows
       mbar_init(aempty(a), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.early_trigger) pdl_trigger();
   const uint32_t tmem_base = tmem_base_sh;
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, 5};
 
@@ -174,14 +184,16 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
             seg = seg_of_tile(p, wtile);
             r0 = (wtile - p.seg_tile0[seg]) * 128 + 64 * h;
           }
-          tma_load_2d(codes + h * (C::CODE_BYTES / 2), &maps.codes[seg], wfull(s), kb * 8, r0);
-          tma_load_2d(scl + h * (C::SO_BYTES / 2), &maps.scales[seg], wfull(s), r0, kb);
-          tma_load_2d(off + h * (C::SO_BYTES / 2), &maps.offsets[seg], wfull(s), r0, kb);
+          tma_load_2d(codes + h * (C::CODE_BYTES / 2), &maps.codes[seg], wfull(s), kb * 8 * KG, r0);
+          tma_load_2d(scl + h * (C::SO_BYTES / 2), &maps.scales[seg], wfull(s), r0, kb * KG);
+          tma_load_2d(off + h * (C::SO_BYTES / 2), &maps.offsets[seg], wfull(s), r0, kb * KG);
         }
       };
       auto load_act = [&](int s, int kb) {
+        const uint32_t st = smem_u32(smem + s * C::STAGE);
         mbar_arrive_expect_tx(xfull(s), C::ACT_BYTES);
-        tma_load_2d(smem_u32(smem + s * C::STAGE), &tmAct, xfull(s), kb * 64, 0);
+#pragma unroll
+        for (int g = 0; g < KG; ++g) tma_load_2d(st + g * C::ACT_SUB, &tmAct, xfull(s), (kb * KG + g) * 64, 0);
       };
       int wfilled[LS], xfilled[LS];
 #pragma unroll
@@ -244,23 +256,32 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
         if (!mbar_wait(acce_bar(abuf), aphase ^ 1u, wc, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * BN);
-        for (int kb = item.kb0; kb < item.kb1; ++kb, ++u) {
-          const int s = (int)(u % LS), a = (int)(u % AS);
-          if (!mbar_wait(afull(a), (uint32_t)((u / AS) & 1), wc, 3) ||
-              !mbar_wait(xfull(s), (uint32_t)((u / LS) & 1), wc, 3)) {
+        for (int kb = item.kb0; kb < item.kb1 && ok; ++kb, ++u) {
+          const int s = (int)(u % LS);
+          if (!mbar_wait(xfull(s), (uint32_t)((u / LS) & 1), wc, 3)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(a_ring + a * C::A_BYTES);
           const uint32_t sb = smem_u32(smem + s * C::STAGE);
+          for (int g = 0; g < KG; ++g) {
+            const long long t = u * KG + g;
+            const int a = (int)(t % AS);
+            if (!mbar_wait(afull(a), (uint32_t)((t / AS) & 1), wc, 3)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(a_ring + a * C::A_BYTES);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(d_tmem, smem_desc_sw128(sa + k * 32, 16, 1024), smem_desc_sw128(sb + k * 32, 16, 1024), IDESC,
-                      (kb > item.kb0 || k > 0) ? 1u : 0u);
-          issued = true;
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(d_tmem, smem_desc_sw128(sa + k * 32, 16, 1024),
+                        smem_desc_sw128(sb + g * C::ACT_SUB + k * 32, 16, 1024), IDESC,
+                        (kb > item.kb0 || g > 0 || k > 0) ? 1u : 0u);
+            issued = true;
+            umma_commit(aempty(a));
+          }
+          if (!ok) break;
           umma_commit(lempty(s));
-          umma_commit(aempty(a));
         }
         if (!ok) break;
         umma_commit(accf_bar(abuf));
@@ -276,7 +297,9 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
     }
   } else if (warp >= Q4_CONV_WARP0) {
     // ------------------------------------------------------------ dequantisers
-    const int r = (warp - Q4_CONV_WARP0) * 32 + lane;   // weight row of the tile
+    // thread (row r, half h): groups h and h + 2 of every unit
+    const int ct = (warp - Q4_CONV_WARP0) * 32 + lane;
+    const int r = ct & 127, h = ct >> 7;
     long long u = 0;
     bool ok = true;
     GemmIter it;
@@ -284,19 +307,29 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
     GemmItem item;
     while (ok && it.next(item)) {
       for (int kb = item.kb0; kb < item.kb1; ++kb, ++u) {
-        const int s = (int)(u % LS), a = (int)(u % AS);
-        if (!__all_sync(0xffffffffu, mbar_wait(wfull(s), (uint32_t)((u / LS) & 1), wc, 10) &&
-                                         mbar_wait(aempty(a), (uint32_t)(((u / AS) & 1) ^ 1), wc, 11))) {
+        const int s = (int)(u % LS);
+        if (!__all_sync(0xffffffffu, mbar_wait(wfull(s), (uint32_t)((u / LS) & 1), wc, 10))) {
           ok = false;
           break;
         }
         const uint8_t* st = smem + s * C::STAGE + C::ACT_BYTES;
-        const uint32_t* words = reinterpret_cast<const uint32_t*>(st) + r * 8;
+        const uint32_t* words = reinterpret_cast<const uint32_t*>(st) + r * (8 * KG);
         const __nv_bfloat16* scl = reinterpret_cast<const __nv_bfloat16*>(st + C::CODE_BYTES);
-        q4_dequant_row(words, scl[r], scl[128 + r], a_ring + a * C::A_BYTES, r);
-        fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
-        __syncwarp();
-        if (lane == 0) mbar_arrive(afull(a));
+        const __nv_bfloat16* ofs = reinterpret_cast<const __nv_bfloat16*>(st + C::CODE_BYTES + C::SO_BYTES);
+        const int so = (r >> 6) * (64 * KG) + (r & 63);   // [half][group][64]
+        for (int g = h; g < KG; g += 2) {
+          const long long t = u * KG + g;
+          const int a = (int)(t % AS);
+          if (!__all_sync(0xffffffffu, mbar_wait(aempty(a), (uint32_t)(((t / AS) & 1) ^ 1), wc, 11))) {
+            ok = false;
+            break;
+          }
+          q4_dequant_row(words + 8 * g, scl[so + 64 * g], ofs[so + 64 * g], a_ring + a * C::A_BYTES, r);
+          fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(afull(a));
+        }
+        if (!ok) break;
       }
     }
   } else {

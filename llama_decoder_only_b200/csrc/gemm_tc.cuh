@@ -81,18 +81,29 @@ struct GemmParams {
   long long units;     // n_tiles * num_kb
   DevStatus* status;
   unsigned long long limit_ns;
+  // 1: signal dependents right after set-up, so the next kernel's CTAs launch
+  // (and fetch their weights) while this one runs; 0: at the end of the work
+  int early_trigger;
+  // decode GEMMs with dynamically assigned chunks (gemm_dyn_kernel)
+  int chunk_units;     // units per chunk (<= num_kb, so a chunk touches at most two tiles)
+  int n_chunks;
+  unsigned* dyn_ctr;   // [2]: next chunk past the grid's first ones, CTAs done grabbing
+  unsigned* tile_ctr;  // [n_tiles]: k-blocks of the tile summed so far (pieces of partial chunks)
 };
 
 constexpr int GEMM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 
 // PAIR: tile mode on a CTA pair (M = 256 per MMA); this CTA holds 128 rows of
-// A and BN / 2 rows of B per stage.
-template <int BN, bool PAIR>
+// A and BN / 2 rows of B per stage.  KS: 64-wide k sub-blocks per unit (decode:
+// a stage then reads KS x 128 contiguous bytes of every weight row).
+template <int BN, bool PAIR, int KS = 1>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;
+  static constexpr int A_SUB = BM * BK * 2;
+  static constexpr int B_SUB = (PAIR ? BN / 2 : BN) * BK * 2;
+  static constexpr int A_BYTES = KS * A_SUB;
+  static constexpr int B_BYTES = KS * B_SUB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
@@ -309,13 +320,14 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
   }
 }
 
-template <int BN, bool SWAP, int EPI>
+template <int BN, bool SWAP, int EPI, int KS = 1>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW0,
                    const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                    const GemmParams p) {
   constexpr bool PAIR = !SWAP;            // tile mode runs 256 x BN tiles on CTA pairs
-  using C = GemmCfg<BN, PAIR>;
+  static_assert(KS == 1 || SWAP, "k sub-blocks are a decode (stream-K) form");
+  using C = GemmCfg<BN, PAIR, KS>;
   constexpr int STAGES = C::STAGES;
   constexpr int WROWS = SWAP ? 128 : BN;  // weight rows per tile
   extern __shared__ uint8_t smem_raw[];
@@ -371,6 +383,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // other CTA, so both must be initialised before either proceeds
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
+  if (p.early_trigger) pdl_trigger();
   // stream-K (decode): the producer starts the weight stream before its PDL wait
   if (!(SWAP && warp == 0)) pdl_wait();
   const uint32_t tmem_base = tmem_base_sh;
@@ -384,17 +397,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int filled_parity[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) filled_parity[s] = -1;
-      // weight tile of k-block kb of weight tile wtile (stream-K mode) into A stage sa
+      // weight tile of unit kb (KS sub-blocks of 64) of weight tile wtile (stream-K mode) into A stage sa
       auto load_weight_swap = [&](uint32_t sa, uint32_t bar, int wtile, int kb) {
-        if (EPI == EPI_SWIGLU_BF16) {
-          // 64 gate rows into lanes 0..63 of the tile, the same 64 up rows into 64..127
-          tma_load_2d(sa, &tmW0, bar, kb * 64, wtile * 64);
-          tma_load_2d(sa + 64 * 128, &tmW1, bar, kb * 64, wtile * 64);
-        } else {
-          const int seg = seg_of_tile(p, wtile);
-          const CUtensorMap* wm = seg == 0 ? &tmW0 : (seg == 1 ? &tmW1 : &tmW2);
-          tma_load_2d(sa, wm, bar, kb * 64, (wtile - p.seg_tile0[seg]) * 128);
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          const int x = (kb * KS + i) * 64;
+          const uint32_t dst = sa + i * C::A_SUB;
+          if (EPI == EPI_SWIGLU_BF16) {
+            // 64 gate rows into lanes 0..63 of the tile, the same 64 up rows into 64..127
+            tma_load_2d(dst, &tmW0, bar, x, wtile * 64);
+            tma_load_2d(dst + 64 * 128, &tmW1, bar, x, wtile * 64);
+          } else {
+            const int seg = seg_of_tile(p, wtile);
+            const CUtensorMap* wm = seg == 0 ? &tmW0 : (seg == 1 ? &tmW1 : &tmW2);
+            tma_load_2d(dst, wm, bar, x, (wtile - p.seg_tile0[seg]) * 128);
+          }
         }
+      };
+      auto load_act_swap = [&](uint32_t sb, uint32_t bar, int kb) {
+#pragma unroll
+        for (int i = 0; i < KS; ++i) tma_load_2d(sb + i * C::B_SUB, &tmAct, bar, (kb * KS + i) * 64, 0);
       };
       int skip = 0;   // k-blocks already issued before the PDL wait
       if (SWAP) {
@@ -414,7 +436,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         pdl_wait();
         for (int s = 0; s < skip; ++s) {
-          tma_load_2d(smem_u32(smem + s * C::STAGE_BYTES) + C::A_BYTES, &tmAct, full_bar(s), pre_kb[s] * 64, 0);
+          load_act_swap(smem_u32(smem + s * C::STAGE_BYTES) + C::A_BYTES, full_bar(s), pre_kb[s]);
           filled_parity[s] = 0;
         }
         stage = skip % STAGES;
@@ -450,7 +472,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (SWAP) {
             mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
             load_weight_swap(sa, full_bar(stage), wtile, kb);
-            tma_load_2d(sb, &tmAct, full_bar(stage), kb * 64, 0);
+            load_act_swap(sb, full_bar(stage), kb);
           } else {
             // both CTAs' bytes land on rank 0's full barrier, which rank 0 arms
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
@@ -503,14 +525,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = smem_desc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + k * 32, 16, 1024);
-            if constexpr (PAIR)
-              umma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > item.kb0 || k > 0) ? 1u : 0u);
-            else
-              umma_bf16(d_tmem, ad, bd, IDESC, (kb > item.kb0 || k > 0) ? 1u : 0u);
-          }
+          for (int i = 0; i < KS; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = smem_desc_sw128(sa + i * C::A_SUB + k * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(sb + i * C::B_SUB + k * 32, 16, 1024);
+              const uint32_t acc = (kb > item.kb0 || i > 0 || k > 0) ? 1u : 0u;
+              if constexpr (PAIR)
+                umma_bf16_pair(d_tmem, ad, bd, IDESC, acc);
+              else
+                umma_bf16(d_tmem, ad, bd, IDESC, acc);
+            }
           issued = true;
           if constexpr (PAIR) umma_commit_pair(empty_bar(stage), 3); else umma_commit(empty_bar(stage));
           if (++stage == STAGES) {

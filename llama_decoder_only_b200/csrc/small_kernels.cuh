@@ -3,6 +3,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ragged.cuh"
 
 namespace llama {
 
@@ -51,6 +52,7 @@ struct RopeTab {
   float* tab;   // nullptr: none
   int hd, L, p0;
   float theta;
+  int early_trigger;   // 1: signal dependents at entry (the next kernel is a GEMM)
 };
 
 template <typename OutT>
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__
                                                        const float* __restrict__ g, OutT* __restrict__ h, int rows,
                                                        int dim, float eps, RopeTab rt) {
   __shared__ float red[32];
+  if (rt.early_trigger) pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x;
   if (row >= rows) return;
@@ -119,16 +122,25 @@ __global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__
 //   cache [batch][nkv][cap][hd]
 // style 0: rotate-half pairs (i, i + hd/2); style 1: adjacent pairs (2i, 2i+1).
 // Each thread moves 16 bytes at a time (8 bf16 or 4 fp32 elements).
+// A ragged batch (tab != nullptr): token m is row m - start[b] of sequence b
+// = seq_of_row(m), at position p0[b] + that row.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T* __restrict__ kc,
                                                           T* __restrict__ vc, int L, int p0, int nh, int nkv,
-                                                          int hd, int cap, float theta, int style) {
+                                                          int hd, int cap, float theta, int style,
+                                                          const SeqTab* __restrict__ tab) {
   constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
   __shared__ float cs[64], sn[64];
   const int m = blockIdx.x;
-  const int b = m / L;
-  const int t = m % L;
-  const int p = p0 + t;
+  int b, p;
+  if (tab == nullptr) {
+    b = m / L;
+    p = p0 + m % L;
+  } else {
+    pdl_wait();   // the table is written by the kernel before
+    b = seq_of_row(tab, m);
+    p = tab->p0[b] + (m - tab->start[b]);
+  }
   const int half = hd >> 1;
   for (int i = threadIdx.x; i < half; i += blockDim.x) rope_cos_sin(p, i, hd, theta, cs[i], sn[i]);
   __syncthreads();
@@ -286,6 +298,18 @@ __global__ void gather_last_rows_kernel(const float* __restrict__ src, float* __
   const float* s = src + ((size_t)b * L + (L - 1)) * dim;
   float* d = dst + (size_t)b * dim;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < dim; i += gridDim.x * blockDim.x) d[i] = s[i];
+}
+
+// Copy a ragged batch's table (kernel parameter) into the workspace, where the
+// call's later kernels read it.
+__global__ void seqtab_kernel(const __grid_constant__ SeqTab t, SeqTab* __restrict__ dst) {
+  pdl_wait();   // earlier kernels may still read the previous call's table
+  if (threadIdx.x == 0) dst->n = t.n;
+  for (int i = threadIdx.x; i < t.n; i += blockDim.x) {
+    dst->start[i] = t.start[i];
+    dst->len[i] = t.len[i];
+    dst->p0[i] = t.p0[i];
+  }
 }
 
 // Device-side failure self-test: wait on an mbarrier that nothing arrives on;

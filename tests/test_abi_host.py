@@ -162,11 +162,11 @@ def test_workspace_grows_with_tokens():
 
 
 def test_workspace_tensors_start_past_the_fixed_header():
-    """The first 1024 bytes of every workspace (status word, decode-GEMM flags)
-    sit at the same place for every call shape and are never part of a tensor:
-    a prefill call's data must not land on the words a later decode call
-    expects to read zero, whatever the two calls' shapes."""
-    header = 1024
+    """The first 4096 bytes of every workspace (status word, decode-GEMM flags,
+    chunk and tile counters) sit at the same place for every call shape and are
+    never part of a tensor: a prefill call's data must not land on the words a
+    later decode call expects to read zero, whatever the two calls' shapes."""
+    header = 4096
     for dims in [L.make_dims(4096, 32, 32, 128, 11008, 1e-6, 1e4, "half", "bf16"),
                  L.make_dims(3072, 32, 32, 96, 8192, 1e-5, 1e4, "half", "bf16"),
                  L.make_dims(256, 8, 2, 32, 688, 1e-5, 1e4, "half", "f32")]:
@@ -224,6 +224,76 @@ def test_noalloc_attention_validates_before_any_launch():
     assert call(d, 1, q, 64 * 128 + 4, k, v, 4096, 100, o) == 4     # ld_q not a multiple of 8
 
 
+# ------------------------------------------------------------------ ragged batches, 4-bit weights, sampling
+
+def test_ragged_lengths_and_validation():
+    lib = L.lib()
+    d = dims()
+    h = cache(d, batch=3, cap=64)
+    lens = (ctypes.c_int32 * 3)(5, 9, 5)
+    assert lib.llama_kv_cache_set_lengths(h, lens) == 0
+    assert lib.llama_kv_cache_length(h) == -2
+    out = (ctypes.c_int32 * 3)()
+    assert lib.llama_kv_cache_lengths(h, out) == 0 and list(out) == [5, 9, 5]
+    # a uniform call refuses a cache whose lengths differ (before any launch)
+    w = fake_weights()
+    ws = lib.llama_workspace_size(ctypes.byref(d), 3, 1)
+    assert lib.llama_layer_decode(ctypes.byref(d), ctypes.byref(w), h, 3, FAKE, FAKE + 0x4000000, FAKE + 0x8000000,
+                                  ws, None) == 1
+    n_new = (ctypes.c_int32 * 3)(1, 60, 1)          # 9 + 60 > 64
+    wsr = lib.llama_workspace_size_ragged(ctypes.byref(d), 3, 62)
+    assert wsr > 0
+    assert lib.llama_layer_forward_ragged(ctypes.byref(d), ctypes.byref(w), h, 3, n_new, FAKE, FAKE + 0x4000000,
+                                          FAKE + 0x8000000, wsr, None) == 3
+    n_new = (ctypes.c_int32 * 3)(1, 0, 1)           # every sequence brings at least one token
+    assert lib.llama_layer_forward_ragged(ctypes.byref(d), ctypes.byref(w), h, 3, n_new, FAKE, FAKE + 0x4000000,
+                                          FAKE + 0x8000000, wsr, None) == 1
+    n_new = (ctypes.c_int32 * 3)(1, 2, 1)
+    small = lib.llama_workspace_size_ragged(ctypes.byref(d), 3, 3)
+    assert lib.llama_layer_forward_ragged(ctypes.byref(d), ctypes.byref(w), h, 3, n_new, FAKE, FAKE + 0x4000000,
+                                          FAKE + 0x8000000, small, None) == 5
+    assert out[1] == 9 and lib.llama_kv_cache_lengths(h, out) == 0 and list(out) == [5, 9, 5]   # unchanged
+    assert lib.llama_workspace_size_ragged(ctypes.byref(d), 129, 200) == 0                        # > 128 sequences
+    assert lib.llama_workspace_size_ragged(ctypes.byref(d), 3, 62) >= lib.llama_workspace_size_ragged(
+        ctypes.byref(d), 3, 3)
+    equal = (ctypes.c_int32 * 3)(7, 7, 7)
+    assert lib.llama_kv_cache_set_lengths(h, equal) == 0 and lib.llama_kv_cache_length(h) == 7
+    big = (ctypes.c_int32 * 3)(7, 65, 7)
+    assert lib.llama_kv_cache_set_lengths(h, big) == 3
+    lib.llama_kv_cache_destroy(h)
+
+
+def test_q4_layer_validation():
+    lib = L.lib()
+    d = dims(ffn_dim=1408)                                                      # every K a multiple of 64
+    h = cache(d, batch=2, cap=64)
+    q = L.Q4Weight(FAKE, FAKE + 0x100000, FAKE + 0x200000)
+    w = L.LayerWeightsQ4(FAKE, q, q, q, q, FAKE, q, q, q)
+    ws = lib.llama_workspace_size(ctypes.byref(d), 2, 1)
+    bad = L.LayerWeightsQ4(FAKE, q, q, L.Q4Weight(FAKE + 4, FAKE, FAKE), q, FAKE, q, q, q)
+    assert lib.llama_layer_decode_q4(ctypes.byref(d), ctypes.byref(bad), h, 2, FAKE, FAKE + 0x4000000,
+                                     FAKE + 0x8000000, ws, None) == 4          # misaligned codes
+    d1 = dims(ffn_dim=1352)                                                     # 1352 % 64 != 0
+    h1 = cache(d1, batch=2, cap=64)
+    assert lib.llama_layer_decode_q4(ctypes.byref(d1), ctypes.byref(w), h1, 2, FAKE, FAKE + 0x4000000,
+                                     FAKE + 0x8000000, lib.llama_workspace_size(ctypes.byref(d1), 2, 1), None) == 2
+    assert lib.llama_layer_decode_q4(ctypes.byref(d), ctypes.byref(w), h, 2, FAKE, FAKE + 0x4000000,
+                                     FAKE + 0x8000000, ws - 1, None) == 5      # workspace too small
+    assert lib.llama_kv_cache_length(h) == 0
+    lib.llama_kv_cache_destroy(h)
+    lib.llama_kv_cache_destroy(h1)
+
+
+@pytest.mark.parametrize("t,p,u,expect", [
+    (-1.0, 0.9, FAKE, 1), (float("nan"), 0.9, FAKE, 1), (1.0, 0.0, FAKE, 1), (1.0, 1.01, FAKE, 1),
+    (1.0, 0.9, None, 1), (1.0, 0.9, FAKE + 4, 4),
+])
+def test_sampling_validation(t, p, u, expect):
+    lib = L.lib()
+    assert lib.llama_sample_top_p(FAKE, 2, 100, t, p, u, FAKE + 0x100000, None) == expect
+
+
+# runs last: it reloads the binding
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(L, "_lib", None)

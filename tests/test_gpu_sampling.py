@@ -5,10 +5,11 @@ fp64 oracle ``oracle/sampling.py`` ([DeepDive] class LLaMA, generate;
 The draw is an input (one uniform per sequence), so the sampled ids are
 deterministic and must equal the oracle's exactly -- except on rows where
 the result is decided within floating-point noise: the GPU forms z = logit /
-temperature and the probabilities in fp32 (the oracle in fp64), so a row
-whose top_p or u lies within 1e-5 of a cumulative boundary, or whose chosen
+temperature and exp(z - max z) in fp32 (about 1e-7 relative error per token;
+the masses are then summed exactly as integers), the oracle in fp64.  A row
+whose top_p or u lies within 1e-6 of a cumulative boundary, or whose chosen
 token shares its z with a neighbour to within 4 fp32 ulps, may land on the
-neighbouring token.  Those rows are counted and must stay a small fraction.
+neighbouring token.  Those rows are counted and must stay a minority.
 """
 
 import numpy as np
@@ -20,7 +21,7 @@ from oracle import sampling as osm
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
-NEAR = 1e-5
+NEAR = 1e-6
 
 
 def _near_boundary(row, temperature, top_p, u):
@@ -72,7 +73,7 @@ def test_sample_top_p_matches_oracle(V, temperature, top_p, scale):
     print(f"[sampling] V {V} T {temperature} top_p {top_p}: {int(near.sum())} of {B} rows near a boundary, "
           f"{int((got != want).sum())} differ")
     assert not bad.any(), f"rows {np.nonzero(bad)[0]}: gpu {got[bad]} oracle {want[bad]}"
-    assert near.sum() <= B // 8
+    assert near.sum() <= B // 4
     assert np.all((got >= 0) & (got < V))
 
 
