@@ -19,8 +19,8 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "decode_layer.cuh"
 #include "f32_path.cuh"
-#include "gemm_decode.cuh"
 #include "gemm_q4.cuh"
 #include "gemm_tc.cuh"
 #include "sampling.cuh"
@@ -43,17 +43,14 @@ namespace {
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 constexpr int kMaxSkGrid = 192;     // upper bound on stream-K CTAs (workspace sizing)
 constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
-// workspace header (see plan_ws): status word, the static decode GEMMs' flags,
-// the dynamic decode GEMMs' chunk counters and tile counters
+// workspace header (see plan_ws): status word, the decode GEMMs' flags and the
+// fused RMSNorm's counters (the rest of the 4 KB is reserved)
 constexpr size_t kWsFlagsOffset = 256;
-constexpr size_t kWsDynCtrOffset = 1024;
-constexpr size_t kWsTileCtrOffset = 2048;
+constexpr size_t kWsNormCtrOffset = 1024;   // [2]: the fused RMSNorm's tile and CTA counters
+constexpr size_t kWsGridBarOffset = 1056;   // [2]: the persistent decode block's grid barrier
 constexpr size_t kWsHeaderBytes = 4096;
-static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsDynCtrOffset, "GEMM flags overflow their area");
-static_assert(kWsTileCtrOffset + DYN_MAX_TILES * 4 <= kWsHeaderBytes, "tile counters overflow the header");
-// chunks per CTA of the dynamic decode GEMM (more chunks balance better, each
-// partial slot costs 128 x BN fp32 of L2 traffic)
-inline int dyn_chunks_per_cta(int bn) { return bn <= 32 ? 3 : 2; }
+static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsNormCtrOffset, "GEMM flags overflow their area");
+constexpr int kMaxNormTiles = 512;           // tiles of a residual GEMM with a fused RMSNorm
 constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K form up to here
 
 // ------------------------------------------------------------------ tracing
@@ -64,12 +61,12 @@ constexpr int kSwapMaxTokens = 128; // decode GEMMs use the swapped stream-K for
 enum KernelKind : int {
   K_RMSNORM = 0, K_GEMM_QKV, K_ROPE_APPEND, K_ATTN_PREFILL, K_ATTN_DECODE, K_ATTN_COMBINE, K_GEMM_O,
   K_GEMM_GATE_UP, K_GEMM_DOWN, K_EMBED, K_GATHER_LAST, K_GEMM_LM_HEAD, K_ARGMAX,
-  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_SAMPLE, K_SEQTAB, K_COUNT
+  K_GEMM_F32, K_ATTN_F32, K_SELFTEST, K_SAMPLE, K_SEQTAB, K_DECODE_LAYER, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
   "rmsnorm", "gemm_qkv", "rope_kv_append", "attn_prefill", "attn_decode", "attn_decode_combine", "gemm_o_proj",
   "gemm_gate_up_swiglu", "gemm_down", "embed", "gather_last_rows", "gemm_lm_head", "argmax",
-  "gemm_f32", "attn_f32", "selftest", "sample_top_p", "seq_table"};
+  "gemm_f32", "attn_f32", "selftest", "sample_top_p", "seq_table", "decode_layer"};
 
 struct ProfRec {
   cudaEvent_t a, b;
@@ -287,6 +284,18 @@ bool use_decode_mma(int hd, int grp) {
   return grp >= 4 && (hd == 64 || hd == 128);
 }
 
+// Of the four 32-key chunks of a prefill softmax row, how many take their
+// exponentials from the FMA pipe (exp2_poly) instead of the MUFU unit
+// (LLAMA_ATTN_EXP_POLY=0..4, default 1).
+int exp_poly_chunks() {
+  static const int n = [] {
+    const char* e = std::getenv("LLAMA_ATTN_EXP_POLY");
+    const int v = e != nullptr ? std::atoi(e) : 1;
+    return v < 0 ? 0 : (v > 4 ? 4 : v);
+  }();
+  return n;
+}
+
 // LLAMA_EARLY_TRIGGER=1: the decode GEMMs, RMSNorm and the split combine signal
 // their dependents at entry instead of at the end of their work.
 int early_trigger() {
@@ -296,6 +305,7 @@ int early_trigger() {
   }();
   return on;
 }
+
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -392,21 +402,15 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // ------------------------------------------------------------------ workspace layout
 
 struct WsLayout {
-  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab, seqtab;   // layer scratch
+  size_t qkv, h, attn, mbuf, partial, sk_flags, att_ml, att_o, rope_tab, seqtab, ssq;   // layer scratch
   size_t xa, xb, xl, hl, logits;                            // model scratch
   size_t total;
 };
 
 int swap_bn(int tokens) { return tokens <= 16 ? 16 : tokens <= 32 ? 32 : tokens <= 64 ? 64 : 128; }
 
-// Partial buffer of one decode GEMM (floats): the static form keeps one
-// [128][BN] piece per CTA, the dynamic form two per chunk.
-size_t sk_partial_floats(int tokens) {
-  const int bn = swap_bn(tokens);
-  const size_t stat = (size_t)kMaxSkGrid * bn * 128;
-  const size_t dyn = (size_t)2 * (dyn_chunks_per_cta(bn) * kMaxSkGrid + 1) * bn * 128;
-  return std::max(stat, dyn);
-}
+// Stream-K partial buffer of one decode GEMM (floats): one [128][BN] piece per CTA.
+size_t sk_partial_floats(int tokens) { return (size_t)kMaxSkGrid * swap_bn(tokens) * 128; }
 
 // ragged_tokens >= 0: a ragged batch of `batch` sequences with that many new
 // tokens in all (seq_len unused); it adds the sequence table at the end.
@@ -450,6 +454,8 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab, int rag
     w.logits = take((size_t)batch * vocab * 4);
   }
   w.seqtab = take(ragged ? sizeof(SeqTab) : 0);
+  // per-tile sums of squares of the decode residual GEMMs with the next RMSNorm fused in
+  w.ssq = take(sk ? (size_t)kMaxNormTiles * swap_bn(sk_tokens) * 4 : 0);
   w.total = off;
   return w;
 }
@@ -480,43 +486,6 @@ llama_status launch_gemm_tc(const CUtensorMap& a, const CUtensorMap* w, const Ge
   return LLAMA_OK;
 }
 
-// LLAMA_DECODE_DYN=0: the decode GEMMs use the static stream-K split instead
-// of dynamically assigned chunks.
-bool decode_dyn() {
-  static const bool on = [] {
-    const char* e = std::getenv("LLAMA_DECODE_DYN");
-    return !(e != nullptr && e[0] == '0');
-  }();
-  return on;
-}
-
-template <int BN, int EPI, int KS>
-llama_status launch_gemm_dyn(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
-                             cudaStream_t st, int kind) {
-  using C = GemmCfg<BN, false, KS>;
-  constexpr int SMEM = 1024 + C::STAGES * C::STAGE_BYTES + 512 + C::EXCH_BYTES;
-  static_assert(SMEM <= 227 * 1024, "shared memory");
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(gemm_dyn_kernel<BN, EPI, KS>), SMEM));
-  {
-    TRACE(kind, st);
-    CUDA_TRY(launch_k(gemm_dyn_kernel<BN, EPI, KS>, grid, GEMM_THREADS, SMEM, st, a, w[0], w[1], w[2], p));
-  }
-  LAUNCH_CHECK();
-  return LLAMA_OK;
-}
-
-template <int BN, int KS>
-llama_status launch_gemm_dyn_epi(int epi, const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
-                                 cudaStream_t st, int kind) {
-  switch (epi) {
-    case EPI_BF16: return launch_gemm_dyn<BN, EPI_BF16, KS>(a, w, p, grid, st, kind);
-    case EPI_RESID_F32: return launch_gemm_dyn<BN, EPI_RESID_F32, KS>(a, w, p, grid, st, kind);
-    case EPI_SWIGLU_BF16: return launch_gemm_dyn<BN, EPI_SWIGLU_BF16, KS>(a, w, p, grid, st, kind);
-    case EPI_F32: return launch_gemm_dyn<BN, EPI_F32, KS>(a, w, p, grid, st, kind);
-  }
-  return LLAMA_ERR_INVALID_ARG;
-}
-
 // k sub-blocks of 64 per decode GEMM unit (LLAMA_DECODE_KSUB=1 or 2, default 2):
 // 2 makes every stage read 256 contiguous bytes of each weight row.
 int decode_ksub() {
@@ -531,6 +500,14 @@ int decode_ksub() {
 struct SkScratch {
   float* partial;
   unsigned* flags;   // the workspace header's flag area (chunk and tile counters follow it)
+  float* ssq;        // per-tile sums of squares for a fused RMSNorm
+};
+
+// An RMSNorm fused into the end of a decode residual GEMM: out = bf16(g * x * rstd(x row)).
+struct NormFuse {
+  const float* g;
+  void* out;
+  float eps;
 };
 
 template <int BN, int KS>
@@ -630,15 +607,13 @@ llama_status gemm_prefill(cudaStream_t st, const void* act, int M, int K, const 
   return LLAMA_ERR_INVALID_ARG;
 }
 
-// Stream-K (decode) GEMM: out = epilogue(act[M, K] · W^T) with W as the MMA's
-// A operand.  The CTA that ends a weight tile adds the other CTAs' pieces of
-// it (published in `sk.partial` under `sk.flags`) and applies the epilogue.
-llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
-                         void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
-                         int kind) {
-  const int BN = swap_bn(M);
-  const int KS = decode_ksub();
-  GemmParams p{};
+// Stream-K parameters and tensor maps of one decode GEMM (bf16, swapped:
+// weight rows fill the MMA's M, the M token rows are its N = BN) over at most
+// `max_grid` CTAs; *grid_out = the CTAs that share its units.
+llama_status prep_decode_gemm(const void* act, int M, int K, const WSeg* segs, int nseg, int epi, void* out,
+                              int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status, int BN, int KS,
+                              int max_grid, GemmParams& p, CUtensorMap& ta, CUtensorMap* tw, int* grid_out) {
+  p = GemmParams{};
   p.K = K;
   p.num_kb = cdiv(K, 64 * KS);
   p.act_rows = M;
@@ -653,8 +628,7 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.partial = sk.partial;
   p.flags = sk.flags;
   p.early_trigger = early_trigger();
-  CUtensorMap ta, tw[3];
-  std::memset(tw, 0, sizeof(tw));
+  std::memset(tw, 0, 3 * sizeof(CUtensorMap));
   if (!make_map_2d(&ta, act, K, M, BN)) return LLAMA_ERR_CUDA;
   int t = 0;
   if (epi == EPI_SWIGLU_BF16) {
@@ -678,30 +652,32 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
   p.n_tiles = t;
   p.units = (long long)p.n_tiles * p.num_kb;
   // no CTA may have an empty unit range: a tile's finisher waits on every CTA between
-  int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
+  const int grid = (int)std::min<long long>(max_grid, p.units);
   if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;  // 32-bit unit math
-  if (decode_dyn() && p.n_tiles <= DYN_MAX_TILES) {
-    // chunks of equal units, at most one tile long; the first `grid` are the CTAs' own
-    const long long want = (long long)dyn_chunks_per_cta(BN) * grid;
-    p.chunk_units = (int)std::max<long long>(1, std::min<long long>(p.num_kb, (p.units + want - 1) / want));
-    p.n_chunks = (int)((p.units + p.chunk_units - 1) / p.chunk_units);
-    grid = std::min(grid, p.n_chunks);
-    p.dyn_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsDynCtrOffset);
-    p.tile_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsTileCtrOffset);
-    if (KS == 2) {
-      switch (BN) {
-        case 16: return launch_gemm_dyn_epi<16, 2>(epi, ta, tw, p, grid, st, kind);
-        case 32: return launch_gemm_dyn_epi<32, 2>(epi, ta, tw, p, grid, st, kind);
-        case 64: return launch_gemm_dyn_epi<64, 2>(epi, ta, tw, p, grid, st, kind);
-        default: return launch_gemm_dyn_epi<128, 2>(epi, ta, tw, p, grid, st, kind);
-      }
-    }
-    switch (BN) {
-      case 16: return launch_gemm_dyn_epi<16, 1>(epi, ta, tw, p, grid, st, kind);
-      case 32: return launch_gemm_dyn_epi<32, 1>(epi, ta, tw, p, grid, st, kind);
-      case 64: return launch_gemm_dyn_epi<64, 1>(epi, ta, tw, p, grid, st, kind);
-      default: return launch_gemm_dyn_epi<128, 1>(epi, ta, tw, p, grid, st, kind);
-    }
+  p.sk_grid = grid;
+  *grid_out = grid;
+  return LLAMA_OK;
+}
+
+// Stream-K (decode) GEMM: out = epilogue(act[M, K] · W^T) with W as the MMA's
+// A operand.  The CTA that ends a weight tile adds the other CTAs' pieces of
+// it (published in `sk.partial` under `sk.flags`) and applies the epilogue.
+llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
+                         void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
+                         int kind, const NormFuse* norm = nullptr) {
+  const int BN = swap_bn(M);
+  const int KS = decode_ksub();
+  GemmParams p;
+  CUtensorMap ta, tw[3];
+  int grid = 0;
+  TRY(prep_decode_gemm(act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, BN, KS,
+                       std::min(num_sms(), kMaxSkGrid), p, ta, tw, &grid));
+  if (norm != nullptr) {
+    p.norm_g = norm->g;
+    p.norm_out = norm->out;
+    p.norm_eps = norm->eps;
+    p.ssq = sk.ssq;
+    p.norm_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsNormCtrOffset);
   }
   if (KS == 2) {
     switch (BN) {
@@ -722,10 +698,24 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
                        int epi, void* out, int ldo, const float* resid, int ldr, SkScratch sk,
-                       DevStatus* status, int kind) {
+                       DevStatus* status, int kind, const NormFuse* norm = nullptr) {
   if (decode && M <= kSwapMaxTokens)
-    return gemm_decode(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, kind);
+    return gemm_decode(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, kind, norm);
   return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
+}
+
+// Whether a decode residual GEMM over M token rows and `dim` output columns
+// takes the following RMSNorm into its own end.  Off unless LLAMA_FUSE_NORM=1:
+// the grid-wide wait at the GEMM's end measured no faster than a stand-alone
+// RMSNorm kernel behind a programmatic-dependent launch (13B-shaped layer at
+// batch 16: 0.346 vs 0.344 ms per step; Phi-3-mini-shaped model at batch 8:
+// 3.38 vs 3.29 ms).
+bool norm_fusable(const llama_dims& d, int M) {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_FUSE_NORM");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on && d.dtype == LLAMA_BF16 && M <= kSwapMaxTokens && cdiv(d.dim, 128) <= kMaxNormTiles;
 }
 
 // ------------------------------------------------------------------ 4-bit group-64 decode GEMMs
@@ -764,7 +754,7 @@ llama_status launch_gemm_q4_epi(int epi, const CUtensorMap& a, const Q4Maps& map
 // up to three segments (or, for EPI_SWIGLU_BF16, gate = segs[0], up = segs[1]).
 llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, const Q4Seg* segs, int nseg, int epi,
                             void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
-                            int kind) {
+                            int kind, const NormFuse* norm = nullptr) {
   if (M > kSwapMaxTokens || K % 64 != 0) return LLAMA_ERR_UNSUPPORTED;
   const int BN = swap_bn(M);
   GemmParams p{};
@@ -782,6 +772,13 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
   p.partial = sk.partial;
   p.flags = sk.flags;
   p.early_trigger = early_trigger();
+  if (norm != nullptr) {
+    p.norm_g = norm->g;
+    p.norm_out = norm->out;
+    p.norm_eps = norm->eps;
+    p.ssq = sk.ssq;
+    p.norm_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsNormCtrOffset);
+  }
   CUtensorMap ta;
   Q4Maps maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -823,6 +820,7 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
   p.units = (long long)p.n_tiles * p.num_kb;
   const int grid = (int)std::min<long long>(std::min(num_sms(), kMaxSkGrid), p.units);
   if ((p.units + 1) * (kMaxSkGrid + 1) >= (1LL << 32)) return LLAMA_ERR_UNSUPPORTED;
+  p.sk_grid = grid;
   switch (BN) {
     case 16: return launch_gemm_q4_epi<16>(epi, ta, maps, p, grid, st, kind);
     case 32: return launch_gemm_q4_epi<32>(epi, ta, maps, p, grid, st, kind);
@@ -873,6 +871,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   // query rows, sharing every K/V tile; MHA: one head over 256 query rows
   p.head_pair = (d.n_heads / d.n_kv_heads) >= 2 ? 1 : 0;
   p.n_qblocks = cdiv(L, p.head_pair ? 128 : 256);
+  p.exp_poly_chunks = exp_poly_chunks();
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
@@ -887,8 +886,9 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
 }
 
 template <int HD, int G>
-cudaError_t launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st) {
-  return launch_k(attn_decode_kernel<HD, G>, grid, 128, 0, st, p);
+cudaError_t launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_t st, bool rope) {
+  if (rope) return launch_k(attn_decode_kernel<HD, G, true>, grid, 128, 0, st, p);
+  return launch_k(attn_decode_kernel<HD, G, false>, grid, 128, 0, st, p);
 }
 
 template <int HD, int G>
@@ -958,18 +958,64 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   return LLAMA_OK;
 }
 
+// Key splits of the CUDA-core decode attention (and keys per split, a multiple
+// of 32).  One CTA per (sequence, KV head) when that alone fills 4 CTAs per SM,
+// or fills every SM once and the cache is short (then there is no combine pass,
+// which costs more than the extra loads in flight would save); otherwise split
+// the keys for about 8 CTAs per SM, >= 64 keys per split (more, shorter splits
+// keep more loads in flight).  Clamped to [min_splits, max_splits].
+int simt_decode_splits(const llama_dims& d, int B, int T, int min_splits, int max_splits, int* kps_out) {
+  const int base = B * d.n_kv_heads;
+  int splits = (base >= 4 * num_sms() || (base >= num_sms() && T <= 2048)) ? 1 : cdiv(8 * num_sms(), base);
+  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 64))));
+  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, 32)));
+  splits = std::max(std::min(min_splits, cdiv(T, 32)), std::min(splits, max_splits));
+  int kps = cdiv(T, splits);
+  kps = cdiv(kps, 32) * 32;
+  if (kps_out != nullptr) *kps_out = kps;
+  return cdiv(T, kps);
+}
+
+// LLAMA_FUSE_ROPE=0 keeps RoPE + KV append a kernel of its own in decode.
+bool rope_fuse_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_FUSE_ROPE");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+// Whether the decode attention over keys [0, T) does RoPE + KV append itself
+// (attn_decode_bf16 with `rope`): the CUDA-core kernel with one key split, so
+// that one CTA owns the new token's q heads and k/v row of its KV head.
+bool decode_rope_fusable(const llama_dims& d, int B, int T, int min_splits = 1, int max_splits = kMaxAttnSplits) {
+  if (!rope_fuse_enabled() || d.dtype != LLAMA_BF16) return false;
+  if (use_decode_mma(d.head_dim, d.n_heads / d.n_kv_heads)) return false;
+  return simt_decode_splits(d, B, T, min_splits, max_splits, nullptr) == 1;
+}
+
+struct RopeFuse {
+  float theta;
+  int style;
+};
+
 // Decode attention of one new token per sequence over keys [0, T).  Splits of
 // the key range are chosen by a heuristic, clamped to [min_splits, max_splits].
 // Ragged batch (tab != nullptr): T is the most keys any sequence sees;
 // sequence b sees tab->p0[b] + 1.
+// rope != nullptr (only where decode_rope_fusable holds): qkv holds the raw
+// projections and the kernel does RoPE + KV append of the new token itself.
 llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                               int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
                               float* part_ml, float* part_o, DevStatus* status, int min_splits = 1,
-                              int max_splits = kMaxAttnSplits, const SeqTab* tab = nullptr) {
+                              int max_splits = kMaxAttnSplits, const SeqTab* tab = nullptr,
+                              const RopeFuse* rope = nullptr) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
-  if (use_decode_mma(hd, grp))
+  if (use_decode_mma(hd, grp)) {
+    if (rope != nullptr) return LLAMA_ERR_UNSUPPORTED;
     return attn_decode_mma(st, d, kc, vc, capacity, B, T, qkv, ld_qkv, out, part_ml, part_o, status, min_splits,
                            max_splits, tab);
+  }
   AttnDecodeParams p{};
   p.qkv = qkv;
   p.ld_qkv = ld_qkv;
@@ -984,25 +1030,18 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
   p.part_o = part_o;
   p.out = out;
   p.tab = tab;
-  // One CTA per (sequence, KV head) when that alone fills 4 CTAs per SM;
-  // otherwise split the keys for about 8 CTAs per SM, >= 64 keys per split
-  // (more, shorter splits keep more loads in flight; with a long cache and a
-  // full grid, extra splits only add the combine pass)
-  const int base = B * d.n_kv_heads;
-  int splits = base >= 4 * num_sms() ? 1 : cdiv(8 * num_sms(), base);
-  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 64))));
-  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, 32)));
-  splits = std::max(std::min(min_splits, cdiv(T, 32)), std::min(splits, max_splits));
-  int kps = cdiv(T, splits);
-  kps = cdiv(kps, 32) * 32;
-  splits = cdiv(T, kps);
+  int kps = 0;
+  const int splits = simt_decode_splits(d, B, T, min_splits, max_splits, &kps);
+  if (rope != nullptr && splits != 1) return LLAMA_ERR_UNSUPPORTED;
   p.splits = splits;
   p.keys_per_split = kps;
+  p.theta = rope != nullptr ? rope->theta : 0.f;
+  p.rope_style = rope != nullptr ? rope->style : 0;
   dim3 grid(splits, d.n_kv_heads, B);
   {
   TRACE(K_ATTN_DECODE, st);
 #define DEC_CASE(HD_, G_) \
-  if (hd == HD_ && grp == G_) CUDA_TRY((launch_attn_decode<HD_, G_>(p, grid, st)));
+  if (hd == HD_ && grp == G_) CUDA_TRY((launch_attn_decode<HD_, G_>(p, grid, st, rope != nullptr)));
   DEC_CASE(64, 1) DEC_CASE(64, 2) DEC_CASE(64, 4) DEC_CASE(64, 8)
   DEC_CASE(96, 1) DEC_CASE(96, 2) DEC_CASE(96, 4) DEC_CASE(96, 8)
   DEC_CASE(128, 1) DEC_CASE(128, 2) DEC_CASE(128, 4) DEC_CASE(128, 8)
@@ -1016,6 +1055,116 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
     LAUNCH_CHECK();
   }
   return LLAMA_OK;
+}
+
+// ------------------------------------------------------------------ persistent decode block
+
+// Whether a decode step of B token rows runs as one persistent kernel
+// (decode_layer_kernel): bf16, B <= 16, head_dim 64 / 96 / 128, GQA group 1 or
+// 2, and the attention's (sequence, KV head) units fit the CTAs' two groups in
+// one round or the cache is short (the kernel runs one key split per unit).
+// LLAMA_DECODE_LAYER=0 keeps the kernel-per-step path.
+bool decode_layer_fusable(const llama_dims& d, int B, int T) {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_DECODE_LAYER");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
+  if (!on || d.dtype != LLAMA_BF16 || B < 1 || B > DL_BN) return false;
+  if (!(hd == 64 || hd == 96 || hd == 128) || !(grp == 1 || grp == 2)) return false;
+  if (use_decode_mma(hd, grp)) return false;   // forced tensor-core decode attention (LLAMA_DECODE_ATTN=mma)
+  if (d.dim % 64 != 0 || cdiv(d.dim, 128) > kMaxNormTiles || num_sms() > kMaxSkGrid) return false;
+  return B * d.n_kv_heads <= 2 * num_sms() || T <= 2048;
+}
+
+template <int HD, int G>
+llama_status launch_decode_layer(const DecLayerParams& P, cudaStream_t st) {
+  using S = DecLayerSmem<HD, G>;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(decode_layer_kernel<HD, G>), S::BYTES));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(num_sms());   // one CTA per SM, all resident (cooperative launch)
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = S::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    TRACE(K_DECODE_LAYER, st);
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_layer_kernel<HD, G>, P));
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+// One decode step of a block (bf16, B token rows at cache length p0) as one
+// persistent kernel; the caller has checked decode_layer_fusable.
+llama_status run_decode_layer(const llama_dims& d, const llama_layer_weights& w, llama_kv_cache* kv, int B,
+                              const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay, cudaStream_t st,
+                              const WSeg* segs, int nseg) {
+  using bf = __nv_bfloat16;
+  const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
+  const int qkvn = (nh + 2 * nkv) * hd;
+  const int p0 = kv->length, T = p0 + 1;
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  bf* qkv = reinterpret_cast<bf*>(ws + lay.qkv);
+  bf* h = reinterpret_cast<bf*>(ws + lay.h);
+  bf* att = reinterpret_cast<bf*>(ws + lay.attn);
+  bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
+  const SkScratch sk{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags),
+                     reinterpret_cast<float*>(ws + lay.ssq)};
+  const int G = num_sms();
+  DecLayerParams P;
+  std::memset(&P, 0, sizeof(P));
+  int grid = 0;
+  TRY(prep_decode_gemm(h, B, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, sk, status, DL_BN, DL_KS, G,
+                       P.g[DL_QKV], P.act[DL_QKV], P.w[DL_QKV], &grid));
+  const WSeg so{w.wo, d.dim, 0};
+  TRY(prep_decode_gemm(att, B, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, sk, status, DL_BN, DL_KS,
+                       G, P.g[DL_O], P.act[DL_O], P.w[DL_O], &grid));
+  P.g[DL_O].norm_g = w.ffn_norm;   // per-tile sums of squares for RMSNorm-2 (no counter)
+  P.g[DL_O].ssq = sk.ssq;
+  const WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
+  TRY(prep_decode_gemm(h, B, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, sk, status, DL_BN, DL_KS, G,
+                       P.g[DL_GU], P.act[DL_GU], P.w[DL_GU], &grid));
+  const WSeg sd{w.w2, d.dim, 0};
+  TRY(prep_decode_gemm(mb, B, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, sk, status, DL_BN,
+                       DL_KS, G, P.g[DL_DOWN], P.act[DL_DOWN], P.w[DL_DOWN], &grid));
+  AttnDecodeParams& a = P.attn;
+  a.qkv = qkv;
+  a.ld_qkv = qkvn;
+  a.kc = reinterpret_cast<const bf*>(kv->k);
+  a.vc = reinterpret_cast<const bf*>(kv->v);
+  a.cap = kv->capacity;
+  a.T = T;
+  a.nh = nh;
+  a.nkv = nkv;
+  a.splits = 1;
+  a.keys_per_split = cdiv(T, 32) * 32;
+  a.scale_log2 = kLog2e / sqrtf((float)hd);
+  a.out = att;
+  a.theta = d.rope_theta;
+  a.rope_style = d.rope_style;
+  P.x_in = x_in;
+  P.x_out = x_out;
+  P.attn_norm = w.attn_norm;
+  P.ffn_norm = w.ffn_norm;
+  P.h = h;
+  P.ssq = sk.ssq;
+  P.bar = reinterpret_cast<unsigned*>(ws + kWsGridBarOffset);
+  P.status = status;
+  P.limit_ns = g_wait_limit_ns.load();
+  P.eps = d.eps;
+  P.dim = d.dim;
+  P.B = B;
+  const int grp = nh / nkv;
+#define DL_CASE(HD_, G_) \
+  if (hd == HD_ && grp == G_) return launch_decode_layer<HD_, G_>(P, st);
+  DL_CASE(64, 1) DL_CASE(64, 2) DL_CASE(96, 1) DL_CASE(96, 2) DL_CASE(128, 1) DL_CASE(128, 2)
+#undef DL_CASE
+  return LLAMA_ERR_UNSUPPORTED;
 }
 
 // ------------------------------------------------------------------ one block
@@ -1037,8 +1186,14 @@ llama_status check_layer_call(const llama_dims* dims, const llama_layer_weights*
 }
 
 // Enqueue one block.  `decode` selects the one-token-per-sequence kernels.
+// Decode with the fused norms (norm_fusable): RMSNorm-2 runs at the end of the
+// o_proj GEMM; `next_norm` (if any) is the RMSNorm that follows this block --
+// the next block's first one, or the model's final one -- run at the end of
+// the down GEMM into `next_out`; `h_ready`: this block's RMSNorm-1 output is
+// already in the workspace (the previous block's down GEMM wrote it).
 llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_kv_cache* kv, int B, int L,
-                       const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay, cudaStream_t st) {
+                       const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay, cudaStream_t st,
+                       const float* next_norm = nullptr, void* next_out = nullptr, bool h_ready = false) {
   DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   const int M = B * L;
   const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
@@ -1055,16 +1210,18 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     // prefill with head_dim 64 / 128: RoPE and the cache append run in the QKV GEMM's epilogue
     const bool fuse_rope = !decode && (hd == 64 || hd == 128);
     float* rtab = reinterpret_cast<float*>(ws + lay.rope_tab);
-    const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
+    const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags),
+                         reinterpret_cast<float*>(ws + lay.ssq)};
+    const bool fuse_norm = decode && norm_fusable(d, M);
     // a2: RMSNorm-1 -> h (bf16)
-    {
+    if (!(fuse_norm && h_ready)) {
       TRACE(K_RMSNORM, st);
       // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
       const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta, early_trigger()};
       CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
                         d.eps, rt));
+      LAUNCH_CHECK();
     }
-    LAUNCH_CHECK();
     // a3: QKV projection
     const size_t rb = (size_t)d.dim * 2;  // bytes per weight row
     WSeg segs[3];
@@ -1078,6 +1235,13 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
+    const bool rope_in_attn = decode && decode_rope_fusable(d, B, p0 + 1);
+    const RopeFuse rf{d.rope_theta, d.rope_style};
+    if (decode && !fuse_norm && decode_layer_fusable(d, B, p0 + 1)) {
+      TRY(run_decode_layer(d, w, kv, B, x_in, x_out, ws, lay, st, segs, nseg));
+      kv->length = p0 + L;
+      return LLAMA_OK;
+    }
     if (fuse_rope) {
       // a3 + a4 in one kernel: rotated q -> qkv, rotated k and v -> the cache
       const RopeArgs ra{kv->k, kv->v, rtab, L, p0, nh, nkv, hd, kv->capacity, d.rope_style};
@@ -1085,41 +1249,43 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
                        &ra));
     } else {
       TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
-      // a4: RoPE + KV append
-      {
+      // a4: RoPE + KV append (decode with one key split: inside the attention kernel)
+      if (!rope_in_attn) {
         TRACE(K_ROPE_APPEND, st);
         CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
                           reinterpret_cast<bf*>(kv->v), L, p0, nh, nkv, hd, kv->capacity, d.rope_theta,
                           d.rope_style, static_cast<const SeqTab*>(nullptr)));
+        LAUNCH_CHECK();
       }
-      LAUNCH_CHECK();
     }
     // a5 / a6: attention
     if (decode) {
       TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
                            reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o),
-                           status));
+                           status, 1, kMaxAttnSplits, nullptr, rope_in_attn ? &rf : nullptr));
     } else {
       TRY(attn_prefill_bf16(st, d, kv, B, L, p0, qkv, att, status));
     }
-    // a7: o_proj + residual -> x_out holds x_mid
+    // a7: o_proj + residual -> x_out holds x_mid (decode: RMSNorm-2 at its end)
     WSeg so{w.wo, d.dim, 0};
+    const NormFuse n2{w.ffn_norm, h, d.eps};
     TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status,
-                  K_GEMM_O));
+                  K_GEMM_O, fuse_norm ? &n2 : nullptr));
     // a8: RMSNorm-2 + gate_up + SiLU·mul
-    {
+    if (!fuse_norm) {
       TRACE(K_RMSNORM, st);
       CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim,
                         d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
+      LAUNCH_CHECK();
     }
-    LAUNCH_CHECK();
     WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
     TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
                   K_GEMM_GATE_UP));
-    // a9: down + residual (in place on x_out)
+    // a9: down + residual (in place on x_out); decode: the next RMSNorm at its end
     WSeg sd{w.w2, d.dim, 0};
+    const NormFuse nn{next_norm, next_out, d.eps};
     TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
-                  K_GEMM_DOWN));
+                  K_GEMM_DOWN, (fuse_norm && next_norm != nullptr) ? &nn : nullptr));
   } else {
     float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
     float* h = reinterpret_cast<float*>(ws + lay.h);
@@ -1237,7 +1403,8 @@ llama_status run_layer_ragged(const llama_dims& d, const llama_layer_weights& w,
   bf* h = reinterpret_cast<bf*>(ws + lay.h);
   bf* att = reinterpret_cast<bf*>(ws + lay.attn);
   bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
-  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
+  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags),
+                         reinterpret_cast<float*>(ws + lay.ssq)};
   {
     TRACE(K_RMSNORM, st);
     CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
@@ -1257,17 +1424,20 @@ llama_status run_layer_ragged(const llama_dims& d, const llama_layer_weights& w,
     nseg = 3;
   }
   TRY(gemm_bf16(st, sk, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
-  {
+  // one new token per sequence and one key split: RoPE + KV append inside the attention kernel
+  const bool rope_in_attn = all_one && decode_rope_fusable(d, B, Tmax);
+  const RopeFuse rf{d.rope_theta, d.rope_style};
+  if (!rope_in_attn) {
     TRACE(K_ROPE_APPEND, st);
     CUDA_TRY(launch_k(rope_append_kernel<bf>, M, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
                       reinterpret_cast<bf*>(kv->v), 1, 0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style,
                       static_cast<const SeqTab*>(dtab)));
+    LAUNCH_CHECK();
   }
-  LAUNCH_CHECK();
   if (all_one) {
     TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, Tmax, qkv, qkvn, att,
                          reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o), status,
-                         1, kMaxAttnSplits, dtab));
+                         1, kMaxAttnSplits, dtab, rope_in_attn ? &rf : nullptr));
   } else {
     TRY(attn_prefill_bf16(st, d, kv, B, maxL, 0, qkv, att, status, dtab, M, Tmax));
   }
@@ -1334,7 +1504,8 @@ llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_
   bf* h = reinterpret_cast<bf*>(ws + lay.h);
   bf* att = reinterpret_cast<bf*>(ws + lay.attn);
   bf* mb = reinterpret_cast<bf*>(ws + lay.mbuf);
-  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)};
+  const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags),
+                         reinterpret_cast<float*>(ws + lay.ssq)};
   {
     TRACE(K_RMSNORM, st);
     CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, B, d.dim,
@@ -1343,23 +1514,30 @@ llama_status run_layer_decode_q4(const llama_dims& d, const llama_layer_weights_
   LAUNCH_CHECK();
   const Q4Seg sq[3] = {{w.wq, nh * hd, 0}, {w.wk, nkv * hd, nh * hd}, {w.wv, nkv * hd, (nh + nkv) * hd}};
   TRY(gemm_decode_q4(st, h, B, d.dim, sq, 3, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
-  {
+  const bool rope_in_attn = decode_rope_fusable(d, B, p0 + 1);
+  const RopeFuse rf{d.rope_theta, d.rope_style};
+  if (!rope_in_attn) {
     TRACE(K_ROPE_APPEND, st);
     CUDA_TRY(launch_k(rope_append_kernel<bf>, B, 256, 0, st, qkv, reinterpret_cast<bf*>(kv->k),
                       reinterpret_cast<bf*>(kv->v), 1, p0, nh, nkv, hd, kv->capacity, d.rope_theta, d.rope_style,
                       static_cast<const SeqTab*>(nullptr)));
+    LAUNCH_CHECK();
   }
-  LAUNCH_CHECK();
   TRY(attn_decode_bf16(st, d, kv->k, kv->v, kv->capacity, B, p0 + 1, qkv, qkvn, att,
-                       reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o), status));
+                       reinterpret_cast<float*>(ws + lay.att_ml), reinterpret_cast<float*>(ws + lay.att_o), status,
+                       1, kMaxAttnSplits, nullptr, rope_in_attn ? &rf : nullptr));
+  // o_proj + residual, with RMSNorm-2 at its end
   const Q4Seg so{w.wo, d.dim, 0};
-  TRY(gemm_decode_q4(st, att, B, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status, K_GEMM_O));
-  {
+  const bool fuse_norm = norm_fusable(d, B);
+  const NormFuse n2{w.ffn_norm, h, d.eps};
+  TRY(gemm_decode_q4(st, att, B, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status, K_GEMM_O,
+                     fuse_norm ? &n2 : nullptr));
+  if (!fuse_norm) {
     TRACE(K_RMSNORM, st);
     CUDA_TRY(launch_k(rmsnorm_kernel<bf>, B, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, B, d.dim,
                       d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
+    LAUNCH_CHECK();
   }
-  LAUNCH_CHECK();
   const Q4Seg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
   TRY(gemm_decode_q4(st, h, B, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
                      K_GEMM_GATE_UP));
@@ -1680,9 +1858,16 @@ llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, 
                                                     m->vocab, status);
   }
   LAUNCH_CHECK();
-  // blocks
+  // blocks (decode with fused norms: each block's down GEMM ends with the next
+  // block's RMSNorm-1, the last one with the final RMSNorm into the lm_head's input)
+  const bool chain = d.dtype == LLAMA_BF16 && seq_len == 1 && norm_fusable(d, batch);
+  void* hbuf = ws + lay.h;
+  void* hl_buf = ws + lay.hl;
   for (int l = 0; l < m->n_layers; ++l) {
-    TRY(run_layer(d, m->layers[l], caches[l], batch, seq_len, xa, xb, ws, lay, st));
+    const bool last = l + 1 == m->n_layers;
+    const float* nn = chain ? (last ? m->final_norm : m->layers[l + 1].attn_norm) : nullptr;
+    TRY(run_layer(d, m->layers[l], caches[l], batch, seq_len, xa, xb, ws, lay, st, nn, last ? hl_buf : hbuf,
+                  chain && l > 0));
     std::swap(xa, xb);
   }
   // a10: final norm + lm_head on the last row of each sequence + argmax
@@ -1699,12 +1884,12 @@ llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, 
   float* logits = logits_or_null ? logits_or_null : reinterpret_cast<float*>(ws + lay.logits);
   if (d.dtype == LLAMA_BF16) {
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + lay.hl);
-    {
+    if (!chain) {
       TRACE(K_RMSNORM, st);
       CUDA_TRY(launch_k(rmsnorm_kernel<__nv_bfloat16>, batch, rmsnorm_threads(d.dim), 0, st, xl, d.dim,
                         m->final_norm, hl, batch, d.dim, d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
+      LAUNCH_CHECK();
     }
-    LAUNCH_CHECK();
     WSeg s{m->lm_head, m->vocab, 0};
     TRY(gemm_bf16(st, true, hl, batch, d.dim, &s, 1, EPI_F32, logits, m->vocab, nullptr, 0,
                   SkScratch{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags)},

@@ -4,12 +4,13 @@
 //    块的内部结构" names FlashAttention: tile Q/K/V through on-chip memory
 //    instead of materialising the score matrix in HBM).  One CTA per
 //    (256-query block, head, sequence) = two 128-row query tiles that share
-//    every K/V tile; K/V tiles of 128 keys arrive by TMA into a 3-slot ring;
+//    every K/V tile (for GQA: two query heads of one KV group over 128 query
+//    rows); K/V tiles of 128 keys arrive by TMA into a 4-slot ring;
 //    S_t = Q_t K^T lands in TMEM, a softmax warpgroup per tile reads it with
 //    tcgen05.ld, keeps the running max / sum in fp32 (online softmax), writes
-//    P_t as bf16 into shared memory, and the MMA warp accumulates
-//    O_t += P_t V in TMEM; the two tiles ping-pong so one tile's softmax
-//    overlaps the other tile's MMAs.  The running max is only moved (and
+//    P_t as bf16 back into TMEM over S_t (tcgen05.st), and the MMA warp
+//    accumulates O_t += P_t V with P_t as the TMEM A operand; the two tiles
+//    ping-pong so one tile's softmax overlaps the other tile's MMAs.  The running max is only moved (and
 //    O rescaled) when it grows by more than 2^8, which is exact because the
 //    final division uses the same stale maximum for numerator and sum.
 //  * attn_decode_kernel (and attn_decode_mma_kernel for GQA groups >= 4):
@@ -26,6 +27,7 @@
 
 #include "common.cuh"
 #include "ragged.cuh"
+#include "small_kernels.cuh"
 
 namespace llama {
 
@@ -42,6 +44,7 @@ struct AttnPrefillParams {
   // rows (GQA, group >= 2: every K/V tile serves both heads); 0: one head over
   // 256 query rows (two 128-row tiles)
   int head_pair;
+  int exp_poly_chunks;  // of the four 32-key chunks of a score row, the last this many take exp2_poly
   float scale_log2;   // log2(e) / sqrt(hd)
   __nv_bfloat16* out; // [B*L, nh*hd] (ragged: [sum of new tokens, nh*hd])
   DevStatus* status;
@@ -54,12 +57,39 @@ struct AttnPrefillParams {
 
 constexpr int ATT_REGION = 128 * 128;           // bytes of a [128 rows x 64 bf16] region
 constexpr int ATT_TILE = 2 * ATT_REGION;        // one 128-row tile of a head (two 64-column regions)
-constexpr int ATT_SLOTS = 3;                    // K/V ring: K_j, V_j, K_{j+1} in flight
+constexpr int ATT_SLOTS = 4;                    // K/V ring: K_j, V_j, K_{j+1}, V_{j+1} in flight
 constexpr int ATT_THREADS = 320;                // producer, MMA, 2 softmax warpgroups
 constexpr int ATT_SMEM = 1024 + 2 * ATT_TILE    // Q0, Q1
                          + ATT_SLOTS * ATT_TILE  // K/V ring
-                         + 2 * ATT_TILE          // P0, P1
                          + 256;
+
+// 32 lanes x 16 consecutive 32-bit columns from registers (thread t -> lane
+// quadrant*32 + t), the store form of tmem_ld16.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  __syncwarp();
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// 2^x on the FMA pipe, for x <= 8 (a softmax exponent against a maximum that
+// lags by at most 2^8): x = i + f with i = floor(x), f in [0, 1); 2^f by a
+// cubic fitted here for the least maximum relative error on [0, 1)
+// (7.5e-5 = 2^-13.7, far below the 2^-9 rounding of the bf16 P it feeds); the
+// integer i goes straight into the exponent field.  x is clamped at -126, so a
+// masked score (-inf) gives 2^-126 ~ 1e-38 instead of 0 -- nothing at bf16 or
+// fp32 accumulation scale.  Relieves the MUFU unit, which ex2.approx shares
+// with every other special function.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float xi = floorf(x);
+  const float f = x - xi;
+  const float p = fmaf(fmaf(fmaf(0.07802403f, f, 0.22606707f), f, 0.69583399f), f, 0.99992513f);
+  return __int_as_float(__float_as_int(p) + ((int)xi << 23));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -80,8 +110,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                   // tile t at t * ATT_TILE
   uint8_t* sKV = sQ + 2 * ATT_TILE;                     // slot s at s * ATT_TILE
-  uint8_t* sP = sKV + ATT_SLOTS * ATT_TILE;             // tile t at t * ATT_TILE
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * ATT_TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + ATT_SLOTS * ATT_TILE);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -161,7 +190,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int last_fill[ATT_SLOTS] = {-1, -1, -1};
+      int last_fill[ATT_SLOTS];
+      for (int s = 0; s < ATT_SLOTS; ++s) last_fill[s] = -1;
       const int nq = q1_valid ? 2 : (q0_valid ? 1 : 0);
       mbar_arrive_expect_tx(q_full, nq * nreg * ATT_REGION);
       for (int t = 0; t < nq; ++t)
@@ -214,16 +244,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         issued = true;
         return true;
       };
+      // O_t += P_t V_j with P_t the A operand in TMEM: bf16 pairs in the first 64
+      // columns of S_t (written there by the softmax warps); issued before S_t's
+      // next MMA, and tcgen05 MMAs run in order, so P is read before S is rewritten
       auto issue_pv = [&](int t, int j) -> bool {
         if (!mbar_wait(p_full(t), j & 1, wc, 5)) return false;
         tc_fence_after();
-        const uint32_t aP = smem_u32(sP + t * ATT_TILE);
         const uint32_t aV = smem_u32(sKV + ((2 * j + 1) % ATT_SLOTS) * ATT_TILE);
-        for (int ks = 0; ks < 8; ++ks) {   // 128 keys, 16 per MMA
-          const uint32_t pa = aP + (ks >> 2) * ATT_REGION + (ks & 3) * 32;
+        for (int ks = 0; ks < 8; ++ks) {   // 128 keys, 16 per MMA (8 TMEM columns of bf16 pairs)
           const uint32_t va = aV + ks * 16 * 128;
-          umma_bf16(tmem + 256 + t * 128, smem_desc_sw128(pa, 16, 1024), smem_desc_sw128(va, ATT_REGION, 1024),
-                    idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + 8 * ks, smem_desc_sw128(va, ATT_REGION, 1024), idesc_o,
+                       (j > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(pv_done(t));
         return true;
@@ -263,7 +294,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t tO = tmem + lane_off + 256 + t * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow0 = sP + t * ATT_TILE + row * 128;
     for (int j = 0; j < my_kv && ok; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(s_full(t), j & 1, wc, 10))) {
         ok = false;
@@ -312,24 +342,32 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      // P = 2^(s - m_used) as bf16 into the swizzled K-major A tile
+      // P = 2^(s - m_used) as bf16 pairs into this row's TMEM lane, over the
+      // first 64 columns of S (already read into registers)
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
       const float sc = p.scale_log2;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {   // 16-byte chunk c holds keys 8c .. 8c+7
-        uint32_t w[4];
+      for (int g4 = 0; g4 < 4; ++g4) {   // keys 32 g4 .. 32 g4 + 31 -> columns 16 g4 .. 16 g4 + 15
+        uint32_t pw[16];
+        if (g4 >= 4 - p.exp_poly_chunks) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = 8 * c + 2 * e;
-          const float a = ex2_approx(fmaf(sv[i0 >> 5][i0 & 31], sc, -mref));
-          const float bb = ex2_approx(fmaf(sv[(i0 + 1) >> 5][(i0 + 1) & 31], sc, -mref));
-          ps[e] += a + bb;
-          w[e] = pack_bf16x2(a, bb);
+          for (int e = 0; e < 16; ++e) {
+            const float a = exp2_poly(fmaf(sv[g4][2 * e], sc, -mref));
+            const float bb = exp2_poly(fmaf(sv[g4][2 * e + 1], sc, -mref));
+            ps[e & 3] += a + bb;
+            pw[e] = pack_bf16x2(a, bb);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = ex2_approx(fmaf(sv[g4][2 * e], sc, -mref));
+            const float bb = ex2_approx(fmaf(sv[g4][2 * e + 1], sc, -mref));
+            ps[e & 3] += a + bb;
+            pw[e] = pack_bf16x2(a, bb);
+          }
         }
-        const int region = c >> 3, cc = c & 7;
-        uint8_t* dst = prow0 + region * ATT_REGION + ((cc ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st16u(tS + 16 * g4, pw);
       }
       // rescale O after P is written: the scores are dead by now, which keeps
       // the 128 loaded O columns from competing with them for registers
@@ -366,10 +404,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           tmem_st32(tO + 0, v0);
           tmem_st32(tO + 32, v1);
         }
-        tmem_st_wait();
       }
+      tmem_st_wait();   // P (and a rescaled O) in TMEM before the MMA warp is told
       l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full(t));
     }
@@ -420,6 +457,11 @@ struct AttnDecodeParams {
   float* part_o;              // [B*nh][splits][hd]
   __nv_bfloat16* out;         // [B, nh*hd]
   const SeqTab* tab;          // ragged: sequence b sees tab->p0[b] + 1 keys; nullptr: all see T
+  // RoPE + KV append fused in (one key split): qkv holds the raw projections;
+  // the kernel rotates q and the new k at position T - 1, appends k and v to the
+  // cache there and writes the rotated q back into qkv
+  float theta;
+  int rope_style;
 };
 
 // Log-sum-exp merge of the `splits` partial results of query head hq of
@@ -444,38 +486,128 @@ __device__ __forceinline__ void combine_head(const float* part_ml, const float* 
 }
 
 
+// Lane slice [sub * VEC, sub * VEC + VEC) of one head row (bf16) -> fp32,
+// read through L2 (the row may have been written by another CTA of the same
+// kernel).
+template <int VEC>
+__device__ __forceinline__ void load_slice(const __nv_bfloat16* src, float (&x)[VEC]) {
+#pragma unroll
+  for (int v = 0; v < VEC / 8; ++v) {
+    uint4 u = __ldcg(reinterpret_cast<const uint4*>(src + 8 * v));
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      x[8 * v + 2 * e] = f.x;
+      x[8 * v + 2 * e + 1] = f.y;
+    }
+  }
+}
+
+// RoPE of one lane's slice (dims sub*VEC ...) of a head row, rounded to bf16
+// as the stand-alone RoPE kernel stores it: rotate-half pairs d with d + HD/2
+// (held by lane sub ^ LPK/2 of the same key group), interleaved pairs (2i, 2i+1)
+// within the slice; cs/sn: the position's cos/sin per pair index.
+template <int HD, int LPK, int VEC>
+__device__ __forceinline__ void rope_slice(float (&x)[VEC], int sub, int style, const float* cs, const float* sn) {
+  if (style == 0) {
+    const bool lower = sub < LPK / 2;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[e], LPK / 2);
+      const int d = sub * VEC + e, i = lower ? d : d - HD / 2;
+      const float c = cs[i], s = sn[i];
+      x[e] = lower ? rope_lo(x[e], other, c, s) : rope_hi(other, x[e], c, s);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < VEC; e += 2) {
+      const int i = (sub * VEC + e) >> 1;
+      const float c = cs[i], s = sn[i], x0 = x[e], x1 = x[e + 1];
+      x[e] = rope_lo(x0, x1, c, s);
+      x[e + 1] = rope_hi(x0, x1, c, s);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) x[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+}
+
+template <int VEC>
+__device__ __forceinline__ void store_slice(__nv_bfloat16* dst, const float (&x)[VEC]) {
+#pragma unroll
+  for (int v = 0; v < VEC / 8; ++v) {
+    uint4 w;
+    w.x = pack_bf16x2(x[8 * v + 0], x[8 * v + 1]);
+    w.y = pack_bf16x2(x[8 * v + 2], x[8 * v + 3]);
+    w.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
+    w.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
+    *reinterpret_cast<uint4*>(dst + 8 * v) = w;
+  }
+}
+
+// Shared memory of one 128-thread decode-attention group.
 template <int HD, int G>
-__global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams p) {
+struct DecAttnSmem {
+  float rcs[HD / 2], rsn[HD / 2];   // RoPE: cos / sin of the new token's angles
+  float m[4][G], l[4][G];           // per-warp softmax state
+  float o[4][G][HD];
+};
+
+// The new token's RoPE angles (position: the cache length before this step).
+template <int HD, int G>
+__device__ __forceinline__ void dec_attn_angles(const AttnDecodeParams& p, int b, int tid, DecAttnSmem<HD, G>& sh) {
+  const int pos = p.tab != nullptr ? p.tab->p0[b] : p.T - 1;
+  for (int i = tid; i < HD / 2; i += 128) rope_cos_sin(pos, i, HD, p.theta, sh.rcs[i], sh.rsn[i]);
+}
+
+// Decode attention of (key split `split`, KV head g, sequence b), run by 128
+// threads (tid 0..127, four whole warps) that meet at `sync`.  ROPE: the
+// angles must be in sh.rcs / sh.rsn before the call (dec_attn_angles).
+template <int HD, int G, bool ROPE, typename Sync>
+__device__ __forceinline__ void attn_decode_body(const AttnDecodeParams& p, int split, int g, int b, int tid,
+                                                 DecAttnSmem<HD, G>& sh, Sync&& sync) {
   constexpr int LPK = HD == 96 ? 4 : HD / 8;    // lanes per key (power of two)
   constexpr int VEC = HD / LPK;                 // elements per lane
   constexpr int NV = VEC / 8;                   // 16-byte loads per lane per row
   constexpr int KPW = 32 / LPK;                 // keys per warp step
   constexpr int NK = 4;                         // keys per lane group per step
   constexpr int NW = 4;
-  pdl_wait();
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* rcs = sh.rcs;
+  const float* rsn = sh.rsn;
+  const int warp = tid >> 5, lane = tid & 31;
   const int grp = lane / LPK, sub = lane % LPK;
   const int T = p.tab != nullptr ? p.tab->p0[b] + 1 : p.T;
   const int j0 = split * p.keys_per_split;
   const int j1 = min(T, j0 + p.keys_per_split);
+  const int j1c = ROPE ? min(j1, T - 1) : j1;   // keys read from the cache
 
   float q[G][VEC];
+  const __nv_bfloat16* row = p.qkv + (size_t)b * p.ld_qkv;
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
-    const __nv_bfloat16* qr = p.qkv + (size_t)b * p.ld_qkv + (size_t)(g * G + gi) * HD + sub * VEC;
+    load_slice<VEC>(row + (size_t)(g * G + gi) * HD + sub * VEC, q[gi]);
+    if (ROPE) rope_slice<HD, LPK, VEC>(q[gi], sub, p.rope_style, rcs, rsn);
+  }
+  float kn[VEC], vn[VEC];   // the new token's rotated key and value (ROPE)
+  if (ROPE) {
+    load_slice<VEC>(row + (size_t)(p.nh + g) * HD + sub * VEC, kn);
+    load_slice<VEC>(row + (size_t)(p.nh + p.nkv + g) * HD + sub * VEC, vn);
+    rope_slice<HD, LPK, VEC>(kn, sub, p.rope_style, rcs, rsn);
+    sync();   // every thread has read the raw q before it is overwritten
+    if (warp == 0 && grp == 0) {
+      const int pos = T - 1;
+      const size_t c = (((size_t)b * p.nkv + g) * p.cap + pos) * HD + sub * VEC;
+      store_slice<VEC>(const_cast<__nv_bfloat16*>(p.kc) + c, kn);
+      store_slice<VEC>(const_cast<__nv_bfloat16*>(p.vc) + c, vn);
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      uint4 u = *reinterpret_cast<const uint4*>(qr + 8 * v);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        q[gi][8 * v + 2 * e] = f.x * p.scale_log2;
-        q[gi][8 * v + 2 * e + 1] = f.y * p.scale_log2;
-      }
+      for (int gi = 0; gi < G; ++gi)
+        store_slice<VEC>(const_cast<__nv_bfloat16*>(row) + (size_t)(g * G + gi) * HD + sub * VEC, q[gi]);
     }
   }
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) q[gi][e] *= p.scale_log2;
   float m[G], l[G], o[G][VEC];
 #pragma unroll
   for (int gi = 0; gi < G; ++gi) {
@@ -488,14 +620,14 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
   const __nv_bfloat16* K = p.kc + head_off;
   const __nv_bfloat16* V = p.vc + head_off;
   constexpr int STEP = NW * KPW * NK;
-  for (int wb = j0 + warp * KPW * NK; wb < j1; wb += STEP) {
+  for (int wb = j0 + warp * KPW * NK; wb < j1c; wb += STEP) {
     uint4 kr[NK][NV], vr[NK][NV];
 #pragma unroll
     for (int kk = 0; kk < NK; ++kk) {
       const int j = wb + grp * NK + kk;
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        if (j < j1) {
+        if (j < j1c) {
           kr[kk][v] = __ldg(reinterpret_cast<const uint4*>(K + (size_t)j * HD) + v);
           vr[kk][v] = __ldg(reinterpret_cast<const uint4*>(V + (size_t)j * HD) + v);
         } else {
@@ -525,7 +657,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
         for (int e = 0; e < VEC; ++e) d = fmaf(q[gi][e], kf[e], d);
 #pragma unroll
         for (int off = LPK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        s[kk][gi] = (wb + grp * NK + kk < j1) ? d : -INFINITY;
+        s[kk][gi] = (wb + grp * NK + kk < j1c) ? d : -INFINITY;
       }
     }
 #pragma unroll
@@ -557,6 +689,25 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
       }
     }
   }
+  if (ROPE && j1 == T && warp == 0) {
+    // the new key (position T - 1) from registers, in lane group 0 of warp 0
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) d = fmaf(q[gi][e], kn[e], d);
+#pragma unroll
+      for (int off = LPK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if (grp == 0) {
+        const float mn = fmaxf(m[gi], d);
+        const float alpha = exp2f(m[gi] - mn), pk = exp2f(d - mn);
+        m[gi] = mn;
+        l[gi] = l[gi] * alpha + pk;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) o[gi][e] = fmaf(pk, vn[e], o[gi][e] * alpha);
+      }
+    }
+  }
   // merge the lane groups of the warp (same `sub`, different keys)
 #pragma unroll
   for (int off = LPK; off < 32; off <<= 1) {
@@ -577,8 +728,9 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
     }
   }
   // merge the warps through shared memory
-  __shared__ float sm_m[NW][G], sm_l[NW][G];
-  __shared__ float sm_o[NW][G][HD];
+  float (*sm_m)[G] = sh.m;
+  float (*sm_l)[G] = sh.l;
+  float (*sm_o)[G][HD] = sh.o;
   if (grp == 0) {
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
@@ -590,8 +742,8 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
       for (int e = 0; e < VEC; ++e) sm_o[warp][gi][sub * VEC + e] = o[gi][e];
     }
   }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
+  sync();
+  for (int idx = tid; idx < G * HD; idx += 128) {
     const int gi = idx / HD, d = idx % HD;
     float M = -INFINITY;
 #pragma unroll
@@ -617,6 +769,18 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
       }
     }
   }
+}
+
+template <int HD, int G, bool ROPE>
+__global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams p) {
+  __shared__ DecAttnSmem<HD, G> sh;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // a ragged table is written by an earlier kernel, so its angles wait for it
+  if (ROPE && p.tab == nullptr) dec_attn_angles<HD, G>(p, b, threadIdx.x, sh);
+  pdl_wait();
+  if (ROPE && p.tab != nullptr) dec_attn_angles<HD, G>(p, b, threadIdx.x, sh);
+  if (ROPE) __syncthreads();
+  attn_decode_body<HD, G, ROPE>(p, split, g, b, threadIdx.x, sh, [] { __syncthreads(); });
 }
 
 // ---------------------------------------------------------------------- decode, GQA groups >= 4

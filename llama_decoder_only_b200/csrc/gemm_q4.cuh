@@ -77,23 +77,20 @@ __device__ __forceinline__ void q4_dequant_row(const uint32_t* words, __nv_bfloa
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t w = wv[j];
+    // bytes (q0, q2, q4, q6) and (q1, q3, q5, q7), then interleaved: (q0..q3), (q4..q7)
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    const uint32_t t03 = __byte_perm(lo, hi, 0x5140), t47 = __byte_perm(lo, hi, 0x7362);
+    // each code under the bf16 exponent byte of 128: the pairs (128 + q_2i, 128 + q_2i+1), exact
+    const uint32_t e[4] = {__byte_perm(t03, 0x43434343u, 0x4140), __byte_perm(t03, 0x43434343u, 0x4342),
+                           __byte_perm(t47, 0x43434343u, 0x4140), __byte_perm(t47, 0x43434343u, 0x4342)};
     uint32_t d[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      // codes i and i + 4 of the word in the low 4 bits of each half, over the
-      // bf16 bit pattern of 128: the pair (128 + q_i, 128 + q_{i+4}), exact
-      const uint32_t t = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
-      __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&t), c128);   // exact
-      __nv_bfloat162 v = __hfma2(q, s2, b2);                                            // one rounding
+      __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&e[i]), c128);   // exact
+      __nv_bfloat162 v = __hfma2(q, s2, b2);                                               // one rounding
       d[i] = *reinterpret_cast<uint32_t*>(&v);
     }
-    // (q0,q4) (q1,q5) (q2,q6) (q3,q7) -> (q0,q1) (q2,q3) (q4,q5) (q6,q7)
-    uint4 o;
-    o.x = __byte_perm(d[0], d[1], 0x5410);
-    o.y = __byte_perm(d[2], d[3], 0x5410);
-    o.z = __byte_perm(d[0], d[1], 0x7632);
-    o.w = __byte_perm(d[2], d[3], 0x7632);
-    *reinterpret_cast<uint4*>(a_tile + r * 128 + ((j ^ (r & 7)) << 4)) = o;
+    *reinterpret_cast<uint4*>(a_tile + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(d[0], d[1], d[2], d[3]);
   }
 }
 
@@ -110,6 +107,8 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
   float* xch_base = reinterpret_cast<float*>(a_ring + AS * C::A_BYTES + 512);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  __shared__ float red_sh[GEMM_EPI_WARPS][16];   // fused RMSNorm: per-warp sums
+  __shared__ float rstd_sh[128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
@@ -354,7 +353,7 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(abuf * BN);
       streamk_epilogue<BN, EPI>(p, item, tbase, row, half, xch_base + half * (64 * 16), threadIdx.x == 64,
-                                &abort_sh, epi_sync);
+                                &abort_sh, epi_sync, red_sh);
       tc_fence_before();
       mbar_arrive(acce_bar(abuf));
       if (++abuf == 2) {
@@ -362,6 +361,8 @@ __global__ void __launch_bounds__(Q4_THREADS, 1)
         aphase ^= 1u;
       }
     }
+    if constexpr (EPI == EPI_RESID_F32)
+      if (p.norm_g != nullptr) fused_rmsnorm<BN>(p, threadIdx.x == 64, &abort_sh, epi_sync, rstd_sh);
   }
 
   pdl_trigger();

@@ -84,11 +84,14 @@ struct GemmParams {
   // 1: signal dependents right after set-up, so the next kernel's CTAs launch
   // (and fetch their weights) while this one runs; 0: at the end of the work
   int early_trigger;
-  // decode GEMMs with dynamically assigned chunks (gemm_dyn_kernel)
-  int chunk_units;     // units per chunk (<= num_kb, so a chunk touches at most two tiles)
-  int n_chunks;
-  unsigned* dyn_ctr;   // [2]: next chunk past the grid's first ones, CTAs done grabbing
-  unsigned* tile_ctr;  // [n_tiles]: k-blocks of the tile summed so far (pieces of partial chunks)
+  // decode GEMM with the residual epilogue: the RMSNorm of the rows it
+  // finishes, norm_out = bf16(norm_g * (out * rstd(out row))) (norm_g == nullptr: none)
+  const float* norm_g;
+  void* norm_out;
+  float norm_eps;
+  float* ssq;          // [n_tiles][BN]: per tile, the sum of squares of each token row's columns
+  unsigned* norm_ctr;  // [2]: tiles finished, CTAs finished normalising (nullptr: ssq only)
+  int sk_grid;         // stream-K: CTAs 0 .. sk_grid-1 share the units (<= gridDim.x, <= units)
 };
 
 constexpr int GEMM_EPI_WARPS = 8;
@@ -135,9 +138,13 @@ struct GemmIter {
       tile_stride = gridDim.x >> 1;
       tile_count = p.m_tiles * p.n_tiles;
     } else {
-      const long long G = gridDim.x;
-      u0 = p.units * (long long)blockIdx.x / G;
-      u = p.units * (long long)(blockIdx.x + 1) / G;
+      const long long G = p.sk_grid;
+      if ((long long)blockIdx.x >= G) {
+        u0 = u = 0;   // no share of this GEMM
+      } else {
+        u0 = p.units * (long long)blockIdx.x / G;
+        u = p.units * (long long)(blockIdx.x + 1) / G;
+      }
     }
   }
   __device__ bool next(GemmItem& it) {
@@ -188,7 +195,8 @@ __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
 // gate/up exchange buffer in shared memory.
 template <int BN, int EPI, typename Sync>
 __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const GemmItem& item, uint32_t tbase, int row,
-                                                 int half, float* xch, bool leader, int* abort_sh, Sync& epi_sync) {
+                                                 int half, float* xch, bool leader, int* abort_sh, Sync& epi_sync,
+                                                 float (*red)[16]) {
   // accumulator: TMEM lane `row` = weight row of the tile, column j = token j
   if (item.kb1 < p.num_kb) {
     // a piece that does not end its tile: publish it for the tile's finisher
@@ -209,7 +217,7 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
       asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + blockIdx.x), "r"(1u) : "memory");
   } else {
     // this CTA ends the tile: add the partials of the lower CTAs that share it
-    const unsigned U = (unsigned)p.units, G = gridDim.x, KB = (unsigned)p.num_kb;
+    const unsigned U = (unsigned)p.units, G = (unsigned)p.sk_grid, KB = (unsigned)p.num_kb;
     const unsigned x = (unsigned)item.tile * KB;
     int c_first = (int)(((x + 1) * G + U - 1) / U) - 1;
     c_first = c_first < 0 ? 0 : c_first;
@@ -294,17 +302,23 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
               o[(size_t)(c + j) * p.ldo + n] = __float2bfloat16_rn(silu_f(v[j]) * xch[j * 64 + row]);
         }
         epi_sync();
-      } else if (active && n_ok) {
+      } else {
+        float xo[16];   // the outputs this thread writes (zero elsewhere), for a fused RMSNorm
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xo[j] = 0.f;
         const int nj = p.act_rows - c < 16 ? p.act_rows - c : 16;
-        if (EPI == EPI_RESID_F32) {
+        if (EPI == EPI_RESID_F32 && active && n_ok) {
           // all residual loads first (out may alias resid: same element, same thread)
           float r[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = j < nj ? p.resid[(size_t)(c + j) * p.ldr + n] : 0.f;
+          for (int j = 0; j < 16; ++j) r[j] = j < nj ? __ldcg(p.resid + (size_t)(c + j) * p.ldr + n) : 0.f;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < nj) reinterpret_cast<float*>(p.out)[(size_t)(c + j) * p.ldo + n] = r[j] + v[j];
-        } else {
+            if (j < nj) {
+              xo[j] = r[j] + v[j];
+              reinterpret_cast<float*>(p.out)[(size_t)(c + j) * p.ldo + n] = xo[j];
+            }
+        } else if (active && n_ok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j >= nj) break;
@@ -315,7 +329,88 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
               reinterpret_cast<float*>(p.out)[o_idx] = v[j];
           }
         }
+        if (EPI == EPI_RESID_F32 && p.norm_g != nullptr) {
+          // this tile's share of each token row's sum of squares: over the warp's
+          // 32 rows by shuffles, then over the four warps of the same column half
+          const int ew = (int)(threadIdx.x >> 5) - 2, lane = (int)(threadIdx.x & 31);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float q = warp_sum(xo[j] * xo[j]);
+            if (lane == j) red[ew][j] = q;
+          }
+          epi_sync();
+          const int e = (int)threadIdx.x - 64;
+          if (e < 32) {
+            const int hh = e >> 4, j = e & 15, c2 = c0 + 16 * hh + j;
+            if (c2 < BN) {
+              float q = 0.f;
+#pragma unroll
+              for (int w = 0; w < 4; ++w) q += red[4 * hh + w][j];
+              p.ssq[(size_t)item.tile * BN + c2] = q;
+            }
+          }
+          epi_sync();
+        }
       }
+    }
+    if (EPI == EPI_RESID_F32 && p.norm_g != nullptr && p.norm_ctr != nullptr && leader) {
+      // the tile's outputs and sums are written (ordered by the group barriers): count it
+      asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.norm_ctr), "r"(1u) : "memory");
+    }
+  }
+}
+
+// RMSNorm of the rows a decode residual GEMM finished ([MLX-13B] 4. RMSNorm;
+// [DeepDive] LLaMARMSNorm), run by the epilogue threads of every CTA once
+// their own tiles are done: wait (bounded) until every tile is counted, rstd
+// of each token row from the tiles' sums of squares, then this CTA's share of
+// the columns, h = g * (x * rstd).  The last CTA re-arms the counters.
+template <int BN, typename Sync>
+__device__ __forceinline__ void fused_rmsnorm(const GemmParams& p, bool leader, int* abort_sh, Sync& epi_sync,
+                                              float* rstd_sh) {
+  if (leader) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      unsigned f;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.norm_ctr) : "memory");
+      if (f >= (unsigned)p.n_tiles || *reinterpret_cast<volatile int*>(abort_sh)) break;
+      if (globaltimer_ns() - t0 > p.limit_ns) {
+        *abort_sh = 1;
+        record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 11, 0);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  epi_sync();
+  const int e = (int)threadIdx.x - 64;
+  const int dim = p.seg_rows[0];
+  const bool ok = *reinterpret_cast<volatile int*>(abort_sh) == 0;
+  if (ok) {
+    for (int j = e; j < p.act_rows; j += 32 * GEMM_EPI_WARPS) {
+      float q = 0.f;
+      for (int t = 0; t < p.n_tiles; ++t) q += __ldcg(p.ssq + (size_t)t * BN + j);
+      rstd_sh[j] = rsqrtf(q / (float)dim + p.norm_eps);
+    }
+  }
+  epi_sync();
+  if (ok) {
+    const int n0 = (int)((long long)dim * blockIdx.x / gridDim.x);
+    const int n1 = (int)((long long)dim * (blockIdx.x + 1) / gridDim.x);
+    const int w = n1 - n0;
+    const float* x = reinterpret_cast<const float*>(p.out);
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.norm_out);
+    for (int i = e; i < w * p.act_rows; i += 32 * GEMM_EPI_WARPS) {
+      const int j = i / w, n = n0 + i % w;
+      h[(size_t)j * dim + n] = __float2bfloat16_rn(__ldg(p.norm_g + n) * (__ldcg(x + (size_t)j * p.ldo + n) * rstd_sh[j]));
+    }
+  }
+  epi_sync();
+  if (leader) {
+    __threadfence();
+    if (atomicAdd(p.norm_ctr + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.norm_ctr, 0u);
+      atomicExch(p.norm_ctr + 1, 0u);
     }
   }
 }
@@ -336,6 +431,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, epilogue group
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  __shared__ float red_sh[SWAP ? GEMM_EPI_WARPS : 1][16];   // fused RMSNorm: per-warp sums
+  __shared__ float rstd_sh[SWAP ? 128 : 1];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -602,7 +699,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (SWAP) {
         streamk_epilogue<BN, EPI>(p, item, tbase, row, half,
                                   reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16),
-                                  threadIdx.x == 64, &abort_sh, epi_sync);
+                                  threadIdx.x == 64, &abort_sh, epi_sync, red_sh);
       } else {
         int mt, wtile;
         tile_coords(p, item.tile, mt, wtile);
@@ -796,6 +893,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         aphase ^= 1u;
       }
     }
+    if constexpr (SWAP && EPI == EPI_RESID_F32)
+      if (p.norm_g != nullptr) fused_rmsnorm<BN>(p, threadIdx.x == 64, &abort_sh, epi_sync, rstd_sh);
   }
 
   pdl_trigger();   // the next kernel may start its prologue while this CTA tears down

@@ -46,6 +46,16 @@ __device__ __forceinline__ void rope_cos_sin(int pos, int i, int hd, float theta
   sincosf((float)a, &s, &c);
 }
 
+// The rotation of one pair (x0, x1) by the angle with cosine c and sine s,
+// rounded step by step (no contraction into fma), so that every kernel that
+// applies RoPE to a decode token produces the same bits.
+__device__ __forceinline__ float rope_lo(float x0, float x1, float c, float s) {
+  return __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
+}
+__device__ __forceinline__ float rope_hi(float x0, float x1, float c, float s) {
+  return __fadd_rn(__fmul_rn(x1, c), __fmul_rn(x0, s));
+}
+
 // Optional second output of an RMSNorm: per token row r (position p0 + r % L),
 // tab[r * hd + i] = cos and tab[r * hd + hd/2 + i] = sin of pair i's angle.
 struct RopeTab {
@@ -162,8 +172,8 @@ __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T
       for (int k = 0; k < VE; ++k) {
         const float x0 = to_f32(xa[k]), x1 = to_f32(xb[k]);
         const float c = cs[i0 + k], s = sn[i0 + k];
-        xa[k] = from_f32<T>(x0 * c - x1 * s);
-        xb[k] = from_f32<T>(x1 * c + x0 * s);
+        xa[k] = from_f32<T>(rope_lo(x0, x1, c, s));
+        xb[k] = from_f32<T>(rope_hi(x0, x1, c, s));
       }
       T* dst = hv;
       if (head >= nh) dst = kc + (((size_t)b * nkv + (head - nh)) * cap + p) * hd;
@@ -183,8 +193,8 @@ __global__ void __launch_bounds__(256) rope_append_kernel(T* __restrict__ qkv, T
         const float x0 = to_f32(x[k]), x1 = to_f32(x[k + 1]);
         const int pi = (i0 + k) >> 1;
         const float c = cs[pi], s = sn[pi];
-        x[k] = from_f32<T>(x0 * c - x1 * s);
-        x[k + 1] = from_f32<T>(x1 * c + x0 * s);
+        x[k] = from_f32<T>(rope_lo(x0, x1, c, s));
+        x[k + 1] = from_f32<T>(rope_hi(x0, x1, c, s));
       }
       T* dst = hv;
       if (head >= nh) dst = kc + (((size_t)b * nkv + (head - nh)) * cap + p) * hd;

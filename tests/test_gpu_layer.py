@@ -169,6 +169,15 @@ DECODE = [
     ("gqa8_b20", 1024, 16, 2, 128, 2816, 20, 513, "half"),
     ("gqa4_hd64_b7", 512, 8, 2, 64, 1376, 7, 129, "half"),
     ("mha_hd96_b8", 384, 4, 4, 96, 1024, 8, 600, "half"),
+    # one key split per (sequence, KV head) -- the CUDA-core attention then
+    # does RoPE + KV append itself: >= 148 such pairs, or a cache <= 64 keys
+    ("mha_hd96_b40_onesplit", 384, 4, 4, 96, 1024, 40, 700, "half"),
+    ("gqa2_hd64_b40_onesplit", 512, 8, 4, 64, 1376, 40, 200, "interleaved"),
+    ("mha_short_cache", 640, 5, 5, 128, 1728, 3, 40, "interleaved"),
+    # batch <= 16 with GQA group 1 or 2 runs the block as one persistent kernel
+    # (mha_b3, mha_hd96_b8 and mha_short_cache above too)
+    ("gqa2_hd128_b16", 1024, 16, 8, 128, 2816, 16, 300, "half"),
+    ("mha_hd64_b1", 512, 8, 8, 64, 1376, 1, 77, "interleaved"),
 ]
 
 
