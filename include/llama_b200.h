@@ -153,9 +153,11 @@ void llama_kv_cache_destroy(llama_kv_cache* cache);
  * `seq_len` new tokens needs (seq_len = 1 for decode).  0 on invalid dims.
  * The workspace is caller-owned scratch.  Zero-fill it once before its first
  * use: a fixed 4096-byte header at its start (the same for every batch and
- * seq_len) holds the device status word and the decode GEMMs' per-CTA flags,
- * chunk counters and per-tile counters, which every launch leaves at zero; after that the library keeps it consistent,
- * also when prefill and decode calls of different shapes share it.  After a
+ * seq_len) holds the device status word, the decode GEMMs' per-CTA flags,
+ * the fused RMSNorm's counters and the grid-barrier counters of the
+ * persistent decode-block kernel, which every launch leaves at zero; after
+ * that the library keeps it consistent, also when prefill and decode calls
+ * of different shapes share it.  After a
  * call that recorded LLAMA_ERR_DEVICE_TIMEOUT, zero-fill it again before
  * reusing it. */
 size_t llama_workspace_size(const llama_dims* dims, int32_t batch, int32_t seq_len);

@@ -47,7 +47,7 @@ constexpr int kMaxAttnSplits = 64;  // upper bound on decode attention splits
 // fused RMSNorm's counters (the rest of the 4 KB is reserved)
 constexpr size_t kWsFlagsOffset = 256;
 constexpr size_t kWsNormCtrOffset = 1024;   // [2]: the fused RMSNorm's tile and CTA counters
-constexpr size_t kWsGridBarOffset = 1056;   // [2]: the persistent decode block's grid barrier
+constexpr size_t kWsGridBarOffset = 1056;   // [8]: the persistent decode block's grid barriers
 constexpr size_t kWsHeaderBytes = 4096;
 static_assert(kWsFlagsOffset + kMaxSkGrid * 4 <= kWsNormCtrOffset, "GEMM flags overflow their area");
 constexpr int kMaxNormTiles = 512;           // tiles of a residual GEMM with a fused RMSNorm
@@ -284,18 +284,6 @@ bool use_decode_mma(int hd, int grp) {
   return grp >= 4 && (hd == 64 || hd == 128);
 }
 
-// Of the four 32-key chunks of a prefill softmax row, how many take their
-// exponentials from the FMA pipe (exp2_poly) instead of the MUFU unit
-// (LLAMA_ATTN_EXP_POLY=0..4, default 1).
-int exp_poly_chunks() {
-  static const int n = [] {
-    const char* e = std::getenv("LLAMA_ATTN_EXP_POLY");
-    const int v = e != nullptr ? std::atoi(e) : 1;
-    return v < 0 ? 0 : (v > 4 ? 4 : v);
-  }();
-  return n;
-}
-
 // LLAMA_EARLY_TRIGGER=1: the decode GEMMs, RMSNorm and the split combine signal
 // their dependents at entry instead of at the end of their work.
 int early_trigger() {
@@ -455,7 +443,8 @@ WsLayout plan_ws(const llama_dims& d, int batch, int seq_len, int vocab, int rag
   }
   w.seqtab = take(ragged ? sizeof(SeqTab) : 0);
   // per-tile sums of squares of the decode residual GEMMs with the next RMSNorm fused in
-  w.ssq = take(sk ? (size_t)kMaxNormTiles * swap_bn(sk_tokens) * 4 : 0);
+  // (+ [CTA][16] shares of the persistent decode block's first RMSNorm)
+  w.ssq = take(sk ? ((size_t)kMaxNormTiles * swap_bn(sk_tokens) + (size_t)kMaxSkGrid * 16) * 4 : 0);
   w.total = off;
   return w;
 }
@@ -871,7 +860,6 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   // query rows, sharing every K/V tile; MHA: one head over 256 query rows
   p.head_pair = (d.n_heads / d.n_kv_heads) >= 2 ? 1 : 0;
   p.n_qblocks = cdiv(L, p.head_pair ? 128 : 256);
-  p.exp_poly_chunks = exp_poly_chunks();
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
@@ -891,13 +879,32 @@ cudaError_t launch_attn_decode(const AttnDecodeParams& p, dim3 grid, cudaStream_
   return launch_k(attn_decode_kernel<HD, G, false>, grid, 128, 0, st, p);
 }
 
+// K/V chunks in flight per CTA of the tensor-core decode attention
+// (LLAMA_DECODE_MMA_STAGES=3 or 4, default 3): three 32 KB stages let two CTAs
+// share an SM (70B-shaped decode, batch 64, cache 4096: attention 163 vs 177
+// us, block 0.499 vs 0.513 ms with four).
+int decode_mma_stages() {
+  static const int n = [] {
+    const char* e = std::getenv("LLAMA_DECODE_MMA_STAGES");
+    return (e != nullptr && e[0] == '4') ? 4 : 3;
+  }();
+  return n;
+}
+
+template <int HD, int G, int ST>
+llama_status launch_attn_decode_mma_st(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
+                                       dim3 grid, cudaStream_t st) {
+  using C = DecMmaCfg<HD, ST>;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_mma_kernel<HD, G, ST>), C::SMEM));
+  CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G, ST>, grid, 32 * (ST + 1), C::SMEM, st, tk, tv, p));
+  return LLAMA_OK;
+}
+
 template <int HD, int G>
 llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
                                     dim3 grid, cudaStream_t st) {
-  using C = DecMmaCfg<HD>;
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_mma_kernel<HD, G>), C::SMEM));
-  CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G>, grid, 160, C::SMEM, st, tk, tv, p));
-  return LLAMA_OK;
+  if (decode_mma_stages() == 3) return launch_attn_decode_mma_st<HD, G, 3>(tk, tv, p, grid, st);
+  return launch_attn_decode_mma_st<HD, G, 4>(tk, tv, p, grid, st);
 }
 
 // Decode attention for GQA groups of 4 or 8 on the tensor cores.
@@ -1060,14 +1067,16 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
 // ------------------------------------------------------------------ persistent decode block
 
 // Whether a decode step of B token rows runs as one persistent kernel
-// (decode_layer_kernel): bf16, B <= 16, head_dim 64 / 96 / 128, GQA group 1 or
-// 2, and the attention's (sequence, KV head) units fit the CTAs' two groups in
-// one round or the cache is short (the kernel runs one key split per unit).
-// LLAMA_DECODE_LAYER=0 keeps the kernel-per-step path.
+// (decode_layer_kernel): only with LLAMA_DECODE_LAYER=1, and for bf16, B <= 16,
+// head_dim 64 / 96 / 128, GQA group 1 or 2, when the attention's (sequence, KV
+// head) units fit the CTAs' two groups in one round or the cache is short (the
+// kernel runs one key split per unit).  Off by default: measured slower than
+// the kernel-per-step chain (Phi-3-mini-shaped block, batch 8, cache 512:
+// 0.125 vs 0.097 ms; 13B-shaped, batch 16: 0.216 vs 0.172 ms).
 bool decode_layer_fusable(const llama_dims& d, int B, int T) {
   static const bool on = [] {
     const char* e = std::getenv("LLAMA_DECODE_LAYER");
-    return !(e != nullptr && e[0] == '0');
+    return e != nullptr && e[0] == '1';
   }();
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   if (!on || d.dtype != LLAMA_BF16 || B < 1 || B > DL_BN) return false;
@@ -1075,6 +1084,16 @@ bool decode_layer_fusable(const llama_dims& d, int B, int T) {
   if (use_decode_mma(hd, grp)) return false;   // forced tensor-core decode attention (LLAMA_DECODE_ATTN=mma)
   if (d.dim % 64 != 0 || cdiv(d.dim, 128) > kMaxNormTiles || num_sms() > kMaxSkGrid) return false;
   return B * d.n_kv_heads <= 2 * num_sms() || T <= 2048;
+}
+
+// LLAMA_DL_PREFETCH=1: the persistent decode block's producer also prefetches
+// upcoming weight tiles and the attention's cache rows into L2.
+bool dl_l2_prefetch() {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_DL_PREFETCH");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
 }
 
 template <int HD, int G>
@@ -1153,12 +1172,14 @@ llama_status run_decode_layer(const llama_dims& d, const llama_layer_weights& w,
   P.ffn_norm = w.ffn_norm;
   P.h = h;
   P.ssq = sk.ssq;
+  P.slots = sk.ssq + (size_t)kMaxNormTiles * DL_BN;
   P.bar = reinterpret_cast<unsigned*>(ws + kWsGridBarOffset);
   P.status = status;
   P.limit_ns = g_wait_limit_ns.load();
   P.eps = d.eps;
   P.dim = d.dim;
   P.B = B;
+  P.l2_prefetch = dl_l2_prefetch();
   const int grp = nh / nkv;
 #define DL_CASE(HD_, G_) \
   if (hd == HD_ && grp == G_) return launch_decode_layer<HD_, G_>(P, st);
@@ -1213,16 +1234,7 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     const SkScratch part{reinterpret_cast<float*>(ws + lay.partial), reinterpret_cast<unsigned*>(ws + lay.sk_flags),
                          reinterpret_cast<float*>(ws + lay.ssq)};
     const bool fuse_norm = decode && norm_fusable(d, M);
-    // a2: RMSNorm-1 -> h (bf16)
-    if (!(fuse_norm && h_ready)) {
-      TRACE(K_RMSNORM, st);
-      // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
-      const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta, early_trigger()};
-      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
-                        d.eps, rt));
-      LAUNCH_CHECK();
-    }
-    // a3: QKV projection
+    // a QKV projection reads one weight buffer when q, k and v sit back to back
     const size_t rb = (size_t)d.dim * 2;  // bytes per weight row
     WSeg segs[3];
     int nseg;
@@ -1235,13 +1247,24 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       segs[2] = {w.wv, nkv * hd, (nh + nkv) * hd};
       nseg = 3;
     }
-    const bool rope_in_attn = decode && decode_rope_fusable(d, B, p0 + 1);
-    const RopeFuse rf{d.rope_theta, d.rope_style};
+    // decode at batch <= 16: the whole block in one persistent kernel
     if (decode && !fuse_norm && decode_layer_fusable(d, B, p0 + 1)) {
       TRY(run_decode_layer(d, w, kv, B, x_in, x_out, ws, lay, st, segs, nseg));
       kv->length = p0 + L;
       return LLAMA_OK;
     }
+    // a2: RMSNorm-1 -> h (bf16)
+    if (!(fuse_norm && h_ready)) {
+      TRACE(K_RMSNORM, st);
+      // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
+      const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta, early_trigger()};
+      CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_in, d.dim, w.attn_norm, h, M, d.dim,
+                        d.eps, rt));
+      LAUNCH_CHECK();
+    }
+    // a3: QKV projection
+    const bool rope_in_attn = decode && decode_rope_fusable(d, B, p0 + 1);
+    const RopeFuse rf{d.rope_theta, d.rope_style};
     if (fuse_rope) {
       // a3 + a4 in one kernel: rotated q -> qkv, rotated k and v -> the cache
       const RopeArgs ra{kv->k, kv->v, rtab, L, p0, nh, nkv, hd, kv->capacity, d.rope_style};

@@ -44,7 +44,6 @@ struct AttnPrefillParams {
   // rows (GQA, group >= 2: every K/V tile serves both heads); 0: one head over
   // 256 query rows (two 128-row tiles)
   int head_pair;
-  int exp_poly_chunks;  // of the four 32-key chunks of a score row, the last this many take exp2_poly
   float scale_log2;   // log2(e) / sqrt(hd)
   __nv_bfloat16* out; // [B*L, nh*hd] (ragged: [sum of new tokens, nh*hd])
   DevStatus* status;
@@ -73,22 +72,6 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[1
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
-}
-
-// 2^x on the FMA pipe, for x <= 8 (a softmax exponent against a maximum that
-// lags by at most 2^8): x = i + f with i = floor(x), f in [0, 1); 2^f by a
-// cubic fitted here for the least maximum relative error on [0, 1)
-// (7.5e-5 = 2^-13.7, far below the 2^-9 rounding of the bf16 P it feeds); the
-// integer i goes straight into the exponent field.  x is clamped at -126, so a
-// masked score (-inf) gives 2^-126 ~ 1e-38 instead of 0 -- nothing at bf16 or
-// fp32 accumulation scale.  Relieves the MUFU unit, which ex2.approx shares
-// with every other special function.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float xi = floorf(x);
-  const float f = x - xi;
-  const float p = fmaf(fmaf(fmaf(0.07802403f, f, 0.22606707f), f, 0.69583399f), f, 0.99992513f);
-  return __int_as_float(__float_as_int(p) + ((int)xi << 23));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -350,22 +333,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
       for (int g4 = 0; g4 < 4; ++g4) {   // keys 32 g4 .. 32 g4 + 31 -> columns 16 g4 .. 16 g4 + 15
         uint32_t pw[16];
-        if (g4 >= 4 - p.exp_poly_chunks) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a = exp2_poly(fmaf(sv[g4][2 * e], sc, -mref));
-            const float bb = exp2_poly(fmaf(sv[g4][2 * e + 1], sc, -mref));
-            ps[e & 3] += a + bb;
-            pw[e] = pack_bf16x2(a, bb);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a = ex2_approx(fmaf(sv[g4][2 * e], sc, -mref));
-            const float bb = ex2_approx(fmaf(sv[g4][2 * e + 1], sc, -mref));
-            ps[e & 3] += a + bb;
-            pw[e] = pack_bf16x2(a, bb);
-          }
+        for (int e = 0; e < 16; ++e) {
+          const float a = ex2_approx(fmaf(sv[g4][2 * e], sc, -mref));
+          const float bb = ex2_approx(fmaf(sv[g4][2 * e + 1], sc, -mref));
+          ps[e & 3] += a + bb;
+          pw[e] = pack_bf16x2(a, bb);
         }
         tmem_st16u(tS + 16 * g4, pw);
       }
@@ -788,21 +761,22 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(const AttnDecodeParams
 // G..15 are zero), so S = Q K^T and O += P V run on the tensor cores
 // (mma.sync m16n8k16, bf16 -> fp32) and the kernel stays bound by the K/V
 // stream.  One producer warp stages 64-key chunks of K and V by TMA (128-byte
-// swizzle, 3-D maps over [head_dim, length, batch*n_kv]); four consumer warps
-// take chunks round robin, each with its own online-softmax state; the warps'
-// states are merged through shared memory at the end.
+// swizzle, 3-D maps over [head_dim, length, batch*n_kv]); one consumer warp
+// per stage takes the chunks of its stage, each with its own online-softmax
+// state; the warps' states are merged through shared memory at the end.
 
 constexpr int DEC_CHUNK = 64;                          // keys per chunk
-constexpr int DEC_STAGES = 4;
 constexpr int DEC_REGION = DEC_CHUNK * 128;            // [64 keys x 64 dims] bf16 = 8 KB
 
 // HD: head dimension as laid out in shared memory (64 or 128); a head_dim of 96
 // runs as 128 with dims 96..127 zero-filled by the TMA bounds (no HBM bytes).
-template <int HD>
+// STAGES: K/V chunks in flight (3 at HD 128 keeps two CTAs on an SM).
+template <int HD, int STAGES_ = 4>
 struct DecMmaCfg {
+  static constexpr int STAGES = STAGES_;
   static constexpr int NREG = HD / 64;                 // 64-dim regions per key row
   static constexpr int STAGE = 2 * NREG * DEC_REGION;  // K then V
-  static constexpr int SMEM = 1024 + DEC_STAGES * STAGE + 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE + 256;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -844,12 +818,15 @@ struct AttnDecodeMmaParams {
   const SeqTab* tab;          // ragged: sequence b sees tab->p0[b] + 1 keys; nullptr: all see T
 };
 
-template <int HD, int G>
-__global__ void __launch_bounds__(160, 1)
+// ST stages and ST consumer warps: warp w takes chunks w, w + ST, ... so each
+// stage has one consumer, and its full / empty phases alternate in chunk order.
+template <int HD, int G, int ST>
+__global__ void __launch_bounds__(32 * (ST + 1), 1)
     attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const AttnDecodeMmaParams p) {
-  using C = DecMmaCfg<HD>;
-  constexpr int NW = 4;                // consumer warps
+  using C = DecMmaCfg<HD, ST>;
+  constexpr int DEC_STAGES = C::STAGES;
+  constexpr int NW = ST;               // consumer warps, one per stage
   constexpr int KS = HD / 16;          // k-steps of S = Q K^T
   constexpr int NT_O = HD / 8;         // 8-dim output tiles
   extern __shared__ uint8_t smem_raw[];

@@ -20,8 +20,12 @@
 // attention (two groups of four warps, one (sequence, KV head) each, with
 // RoPE + KV append inside, one key split).
 //
-// Phases and grid barriers (barrier k completes when every CTA arrived k times):
-//   P0 RMSNorm-1 (every CTA: rstd of all rows, its column slice of h) -> 1
+// Phases and grid barriers (one counter per barrier; barrier k completes when
+// every CTA has arrived at it -- a single running count would let a CTA with
+// no work in a phase arrive at the next barrier early and stand in for one
+// still busy):
+//   P0 RMSNorm-1: every CTA's share of each row's sum of squares    -> 0
+//      then rstd of every row from the shares, its column slice of h -> 1
 //   P1 QKV projection into qkv (raw)                                  -> 2
 //   P2 RoPE + KV append + attention into att                          -> 3
 //   P3 o_proj + residual into x_out (x_mid), per-tile sums of squares -> 4
@@ -59,11 +63,13 @@ struct alignas(64) DecLayerParams {
   const float* ffn_norm;
   __nv_bfloat16* h;       // [B, dim] RMSNorm output (first RMSNorm-1, then RMSNorm-2)
   float* ssq;             // [o_proj tiles][16] per-tile sums of squares of x_mid rows
-  unsigned* bar;          // [2] grid barrier: arrivals, CTAs done
+  float* slots;           // [CTAs][16] each CTA's share of the sums of squares of the x_in rows
+  unsigned* bar;          // [8] grid barriers 0..6 at [0..6], CTAs done at [7]
   DevStatus* status;
   unsigned long long limit_ns;
   float eps;
   int dim, B;
+  int l2_prefetch;        // 1: the producer prefetches upcoming weights and the cache into L2
 };
 static_assert(sizeof(DecLayerParams) <= 4096, "kernel parameters exceed 4 KB");
 
@@ -71,7 +77,23 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Bounded wait until the grid barrier counter reaches `target`.
+// L2 prefetch of one box of a tensor map (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+// L2 prefetch of a contiguous range (16-byte aligned address and size).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes) : "memory");
+}
+
+// Bytes each L2 prefetch batch of the producer may bring in, over all CTAs: a
+// few batches stay well inside the 126 MB L2.
+constexpr long long kDlPrefetchBatch = 32ll << 20;
+
+// Bounded wait until every CTA has arrived at a grid barrier (its counter
+// reaches `target`).
 __device__ __forceinline__ bool dl_grid_wait(const unsigned* bar, unsigned target, int* abort_sh, DevStatus* st,
                                              unsigned long long limit_ns, int detail) {
   const uint64_t t0 = globaltimer_ns();
@@ -99,8 +121,9 @@ struct DecLayerSmem {
 };
 
 template <int HD, int G>
-__global__ void __maxnreg__(200)
-    decode_layer_kernel(const __grid_constant__ DecLayerParams P) {
+// 320 threads at one CTA per SM: ptxas caps the kernel at 168 registers a
+// thread (a 200-register build failed to launch).
+__global__ void __launch_bounds__(GEMM_THREADS, 1) decode_layer_kernel(const __grid_constant__ DecLayerParams P) {
   using C = DLCfg;
   using S = DecLayerSmem<HD, G>;
   constexpr int STAGES = C::STAGES;
@@ -164,6 +187,57 @@ __global__ void __maxnreg__(200)
       for (int s = 0; s < STAGES; ++s) filled_parity[s] = -1;
       bool ok = true;
       constexpr unsigned kBarrierBefore[4] = {1, 3, 5, 6};
+      const long long budget = kDlPrefetchBatch / nctas;   // bytes per CTA and batch
+      // L2 prefetch of this CTA's weight tiles of projection gj in the order it
+      // will load them, after its first `skip` units, up to `budget` bytes
+      auto prefetch_weights = [&](int gj, int skip) {
+        const GemmParams& q = P.g[gj];
+        GemmIter it;
+        it.init(q, true);
+        GemmItem item;
+        int n = 0;
+        long long bytes = 0;
+        while (it.next(item)) {
+          for (int kb = item.kb0; kb < item.kb1; ++kb) {
+            if (n++ < skip) continue;
+            if (bytes >= budget) return;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+              const int x = (kb * KS + i) * 64;
+              if (gj == DL_GU) {
+                tma_prefetch_l2_2d(&P.w[gj][0], x, item.tile * 64);
+                tma_prefetch_l2_2d(&P.w[gj][1], x, item.tile * 64);
+              } else {
+                const int seg = seg_of_tile(q, item.tile);
+                tma_prefetch_l2_2d(&P.w[gj][seg], x, (item.tile - q.seg_tile0[seg]) * 128);
+              }
+            }
+            bytes += C::A_BYTES;
+          }
+        }
+      };
+      // L2 prefetch of the cached keys and values [0, T-1) of this CTA's
+      // attention units (the new token's row is appended during the step)
+      auto prefetch_kv = [&]() {
+        const AttnDecodeParams& a = P.attn;
+        const long long row_bytes = (long long)HD * 2;
+        const long long n_bytes = (long long)(a.T - 1) * row_bytes;
+        const int units = P.B * a.nkv;
+        long long bytes = 0;
+        // the units of this CTA's two worker groups, round by round
+        for (int u0 = (int)blockIdx.x * 2; u0 < units && bytes < budget; u0 += 2 * (int)nctas) {
+          for (int u = u0; u < u0 + 2 && u < units; ++u) {
+            const int b = u / a.nkv, g = u - b * a.nkv;
+            const size_t off = ((size_t)b * a.nkv + g) * (size_t)a.cap * HD;
+            for (long long o = 0; o < n_bytes; o += 32768) {
+              const uint32_t len = (uint32_t)min(32768ll, n_bytes - o);
+              bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(a.kc + off) + o, len);
+              bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(a.vc + off) + o, len);
+            }
+            bytes += 2 * n_bytes;
+          }
+        }
+      };
 #pragma unroll 1
       for (int gi = 0; gi < 4 && ok; ++gi) {
         const GemmParams& p = P.g[gi];
@@ -211,8 +285,21 @@ __global__ void __maxnreg__(200)
           }
         }
         if (!ok) break;
+        // keep HBM busy through the phases that stream no weights: the next
+        // bytes this CTA will want go to L2 now (one projection ahead, and the
+        // attention's keys and values during the QKV projection)
+        if (!P.l2_prefetch) {
+        } else if (gi == DL_QKV) {
+          prefetch_weights(DL_QKV, STAGES);
+          prefetch_kv();
+          prefetch_weights(DL_O, STAGES);
+        } else if (gi == DL_O) {
+          prefetch_weights(DL_GU, STAGES);
+        } else if (gi == DL_GU) {
+          prefetch_weights(DL_DOWN, STAGES);
+        }
         // 2. the activation of this projection is complete in every CTA
-        if (!dl_grid_wait(P.bar, kBarrierBefore[gi] * nctas, &abort_sh, P.status, P.limit_ns, gi)) break;
+        if (!dl_grid_wait(P.bar + kBarrierBefore[gi], nctas, &abort_sh, P.status, P.limit_ns, gi)) break;
         fence_proxy_async_global();
         for (int i = 0; i < pre; ++i)
           load_act(smem_u32(smem + pre_stage[i] * C::STAGE_BYTES) + C::A_BYTES, full_bar(pre_stage[i]), pre_kb[i]);
@@ -318,17 +405,17 @@ __global__ void __maxnreg__(200)
       mbar_wait(epi_bar, epi_phase, wc, 7);
       epi_phase ^= 1u;
     };
-    // this CTA's writes of the phase are done: count it at the grid barrier
-    auto arrive = [&]() {
+    // this CTA's writes of the phase are done: count it at grid barrier k
+    auto arrive = [&](int k) {
       fence_proxy_async_global();   // readers of these writes include TMA loads
       epi_sync();
       if (leader) {
         __threadfence();
-        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(P.bar), "r"(1u) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(P.bar + k), "r"(1u) : "memory");
       }
     };
-    auto grid_wait = [&](unsigned k) {
-      if (leader) dl_grid_wait(P.bar, k * nctas, &abort_sh, P.status, P.limit_ns, 10 + (int)k);
+    auto grid_wait = [&](int k) {
+      if (leader) dl_grid_wait(P.bar + k, nctas, &abort_sh, P.status, P.limit_ns, 10 + k);
       epi_sync();
       return *reinterpret_cast<volatile int*>(&abort_sh) == 0;
     };
@@ -368,24 +455,37 @@ __global__ void __maxnreg__(200)
     // the new token's RoPE angles, the same for every unit of the attention
     // phase (one position per step), once per group
     dec_attn_angles<HD, G>(P.attn, 0, wid & 127, ash[wid >> 7]);
-    // P0: RMSNorm-1 -- every CTA forms rstd of every row, then writes its columns
-    for (int j = ww; j < B; j += GEMM_EPI_WARPS) {
-      const float4* xr = reinterpret_cast<const float4*>(P.x_in + (size_t)j * dim);
-      float ss[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int i = lane; i < (dim >> 2); i += 32) {
-        const float4 v = __ldcg(xr + i);
-        ss[(i >> 5) & 3] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-      }
-      const float t = warp_sum((ss[0] + ss[1]) + (ss[2] + ss[3]));
-      if (lane == 0) rstd_sh[j] = rsqrtf(t / (float)dim + P.eps);
+    // P0: RMSNorm-1.  Each CTA sums the squares of its own columns of every
+    // row (16 threads a row), the shares meet at barrier 0, and every CTA adds
+    // the shares in CTA order (the same rstd everywhere) for its column slice.
+    {
+      const int j = wid >> 4, r = wid & 15;
+      float q = 0.f;
+      if (j < B)
+        for (int n = n0 + r; n < n1; n += 16) {
+          const float v = __ldcg(P.x_in + (size_t)j * dim + n);
+          q = fmaf(v, v, q);
+        }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      if (j < B && r == 0) P.slots[blockIdx.x * 16 + j] = q;
+    }
+    arrive(0);
+    if (grid_wait(0)) {
+      const int j = wid >> 4, r = wid & 15;
+      float q = 0.f;
+      if (j < B)
+        for (int c = r; c < (int)nctas; c += 16) q += __ldcg(P.slots + c * 16 + j);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      if (j < B && r == 0) rstd_sh[j] = rsqrtf(q / (float)dim + P.eps);
     }
     epi_sync();
     norm_slice(P.x_in, P.attn_norm);
-    arrive();   // -> 1
+    arrive(1);
     // P1: QKV projection (raw q, k, v)
     epilogues(std::integral_constant<int, EPI_BF16>{}, DL_QKV);
-    arrive();   // -> 2
+    arrive(2);
     // P2: RoPE + KV append + attention, one (sequence, KV head) per group of four warps
     if (grid_wait(2)) {
       const int grp = wid >> 7, tid = wid & 127;
@@ -398,10 +498,10 @@ __global__ void __maxnreg__(200)
         group_sync();   // the group's shared state is free for its next unit
       }
     }
-    arrive();   // -> 3
+    arrive(3);
     // P3: o_proj + residual -> x_mid, with each tile's sums of squares
     epilogues(std::integral_constant<int, EPI_RESID_F32>{}, DL_O);
-    arrive();   // -> 4
+    arrive(4);
     // P4: RMSNorm-2 from the tiles' sums of squares
     if (grid_wait(4)) {
       for (int j = ww; j < B; j += GEMM_EPI_WARPS) {
@@ -413,10 +513,10 @@ __global__ void __maxnreg__(200)
       epi_sync();
       norm_slice(P.x_out, P.ffn_norm);
     }
-    arrive();   // -> 5
+    arrive(5);
     // P5: gate/up + SiLU·mul -> m
     epilogues(std::integral_constant<int, EPI_SWIGLU_BF16>{}, DL_GU);
-    arrive();   // -> 6
+    arrive(6);
     // P6: down + residual -> block output
     epilogues(std::integral_constant<int, EPI_RESID_F32>{}, DL_DOWN);
   }
@@ -429,9 +529,8 @@ __global__ void __maxnreg__(200)
     // the last CTA to finish re-arms the barrier words for the next launch
     // (every CTA has passed all its waits by the time it counts itself here)
     __threadfence();
-    if (atomicAdd(P.bar + 1, 1u) == nctas - 1) {
-      atomicExch(P.bar, 0u);
-      atomicExch(P.bar + 1, 0u);
+    if (atomicAdd(P.bar + 7, 1u) == nctas - 1) {
+      for (int k = 0; k < 8; ++k) atomicExch(P.bar + k, 0u);
     }
   }
 }

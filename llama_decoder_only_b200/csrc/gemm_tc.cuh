@@ -224,12 +224,15 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
     // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count)
     const int n_contrib = (int)blockIdx.x - c_first;
     if (n_contrib > 0) {
-      if (leader) {
-        for (int c = c_first; c < (int)blockIdx.x; ++c) {
-          const uint64_t t0 = globaltimer_ns();
+      // the first epilogue warp waits for the contributors' flags, one lane
+      // each, so the waits overlap (one L2 round trip instead of one per piece)
+      if ((threadIdx.x >> 5) == 2) {
+        const int lane = (int)(threadIdx.x & 31);
+        const uint64_t t0 = globaltimer_ns();
+        for (int c = c_first + lane; c < (int)blockIdx.x; c += 32) {
           while (true) {
             unsigned f;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.flags + c) : "memory");
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(p.flags + c) : "memory");
             if (f == 1u || *reinterpret_cast<volatile int*>(abort_sh)) break;
             if (globaltimer_ns() - t0 > p.limit_ns) {
               *abort_sh = 1;
@@ -241,6 +244,8 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
           // this CTA is the only reader of c's piece: re-arm the flag for the next launch
           asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p.flags + c), "r"(0u) : "memory");
         }
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");   // the pieces are read after the flags were seen
+        __syncwarp();
       }
       epi_sync();
     }

@@ -6,9 +6,9 @@ choice is read once per process, so each kernel runs the decode parity tests
 of ``test_gpu_layer.py`` (head_dim 64 / 96 / 128, groups 1 / 4 / 8, against
 the fp64 oracle) in a child process, together with the full-size 13B-shaped
 decode check.  The same child runs cover the other decode forms: RoPE + KV
-append kept apart from the CUDA-core attention (LLAMA_FUSE_ROPE=0), a kernel
-per step instead of the persistent decode-block kernel at batch <= 16
-(LLAMA_DECODE_LAYER=0), and the RMSNorms taken into the ends of the residual
+append kept apart from the CUDA-core attention (LLAMA_FUSE_ROPE=0), the
+persistent decode-block kernel at batch <= 16 instead of a kernel per step
+(LLAMA_DECODE_LAYER=1), and the RMSNorms taken into the ends of the residual
 GEMMs (LLAMA_FUSE_NORM=1).
 """
 
@@ -25,9 +25,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.mark.parametrize("kernel,extra", [("mma", {}), ("simt", {}), ("simt", {"LLAMA_FUSE_ROPE": "0"}),
-                                          ("simt", {"LLAMA_DECODE_LAYER": "0"}),
+                                          ("simt", {"LLAMA_DECODE_LAYER": "1"}),
                                           ("mma", {"LLAMA_FUSE_NORM": "1"}), ("simt", {"LLAMA_FUSE_NORM": "1"})],
-                         ids=["mma", "simt", "simt-rope-apart", "simt-kernel-per-step", "mma-norm-fused",
+                         ids=["mma", "simt", "simt-rope-apart", "simt-decode-block", "mma-norm-fused",
                               "simt-norm-fused"])
 def test_decode_parity_with_each_attention_kernel(kernel, extra):
     env = dict(os.environ, LLAMA_DECODE_ATTN=kernel, **extra)
@@ -100,7 +100,7 @@ def test_decode_block_kernel_matches_kernel_per_step(tmp_path, rope):
     same way; RMSNorm-1 sums its squares in another order and the attention
     runs one key split instead of several, so values agree to within bf16
     rounding of the tensors the block stores."""
-    res = _child_runs(tmp_path, rope, 8, {"block": {}, "steps": {"LLAMA_DECODE_LAYER": "0"}})
+    res = _child_runs(tmp_path, rope, 8, {"block": {"LLAMA_DECODE_LAYER": "1"}, "steps": {}})
     a, b = res["block"], res["steps"]
     for t in range(2):
         for n in ("q", "k", "v", "y"):

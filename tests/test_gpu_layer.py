@@ -174,8 +174,9 @@ DECODE = [
     ("mha_hd96_b40_onesplit", 384, 4, 4, 96, 1024, 40, 700, "half"),
     ("gqa2_hd64_b40_onesplit", 512, 8, 4, 64, 1376, 40, 200, "interleaved"),
     ("mha_short_cache", 640, 5, 5, 128, 1728, 3, 40, "interleaved"),
-    # batch <= 16 with GQA group 1 or 2 runs the block as one persistent kernel
-    # (mha_b3, mha_hd96_b8 and mha_short_cache above too)
+    # batch <= 16 with GQA group 1 or 2: shapes the persistent decode-block
+    # kernel takes (with LLAMA_DECODE_LAYER=1; mha_b3, mha_hd96_b8 and
+    # mha_short_cache above too)
     ("gqa2_hd128_b16", 1024, 16, 8, 128, 2816, 16, 300, "half"),
     ("mha_hd64_b1", 512, 8, 8, 64, 1376, 1, 77, "interleaved"),
 ]
