@@ -271,17 +271,24 @@ int forced_decode_splits() {
 }
 
 // Which decode-attention kernel serves (head_dim, GQA group): the TMA-fed
-// tensor-core kernel for groups >= 4 (its 16-row tile fills), the CUDA-core one
-// below that.  LLAMA_DECODE_ATTN=mma | simt forces one of them.
-bool use_decode_mma(int hd, int grp) {
+// tensor-core kernel for groups >= 4 (its 16-row tile fills) and for head_dim
+// 96 (where the CUDA-core kernel's 24 elements a lane hold two CTAs per SM:
+// Phi-3-mini-shaped block, batch 8, cache 512: 16.8 vs 21.5 us), the CUDA-core
+// one otherwise.  LLAMA_DECODE_ATTN=mma | simt forces one of them.
+// LLAMA_DECODE_ATTN: 1 = mma, 2 = simt, 0 = not set.
+int decode_attn_forced() {
   static const int forced = [] {
     const char* e = std::getenv("LLAMA_DECODE_ATTN");
     if (e == nullptr) return 0;
     return std::strcmp(e, "mma") == 0 ? 1 : (std::strcmp(e, "simt") == 0 ? 2 : 0);
   }();
-  if (forced == 1) return true;
-  if (forced == 2) return false;
-  return grp >= 4 && (hd == 64 || hd == 128);
+  return forced;
+}
+
+bool use_decode_mma(int hd, int grp) {
+  if (decode_attn_forced() == 1) return true;
+  if (decode_attn_forced() == 2) return false;
+  return (grp >= 4 && (hd == 64 || hd == 128)) || hd == 96;
 }
 
 // LLAMA_EARLY_TRIGGER=1: the decode GEMMs, RMSNorm and the split combine signal
@@ -891,27 +898,49 @@ int decode_mma_stages() {
   return n;
 }
 
-template <int HD, int G, int ST>
+template <int HD, int G, int ST, bool ROPE>
 llama_status launch_attn_decode_mma_st(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
                                        dim3 grid, cudaStream_t st) {
   using C = DecMmaCfg<HD, ST>;
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_mma_kernel<HD, G, ST>), C::SMEM));
-  CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G, ST>, grid, 32 * (ST + 1), C::SMEM, st, tk, tv, p));
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_mma_kernel<HD, G, ST, ROPE>), C::SMEM));
+  CUDA_TRY(launch_k(attn_decode_mma_kernel<HD, G, ST, ROPE>, grid, 32 * (ST + 1), C::SMEM, st, tk, tv, p));
   return LLAMA_OK;
 }
 
 template <int HD, int G>
 llama_status launch_attn_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const AttnDecodeMmaParams& p,
-                                    dim3 grid, cudaStream_t st) {
-  if (decode_mma_stages() == 3) return launch_attn_decode_mma_st<HD, G, 3>(tk, tv, p, grid, st);
-  return launch_attn_decode_mma_st<HD, G, 4>(tk, tv, p, grid, st);
+                                    dim3 grid, cudaStream_t st, bool rope) {
+  if (decode_mma_stages() == 3)
+    return rope ? launch_attn_decode_mma_st<HD, G, 3, true>(tk, tv, p, grid, st)
+                : launch_attn_decode_mma_st<HD, G, 3, false>(tk, tv, p, grid, st);
+  return rope ? launch_attn_decode_mma_st<HD, G, 4, true>(tk, tv, p, grid, st)
+              : launch_attn_decode_mma_st<HD, G, 4, false>(tk, tv, p, grid, st);
 }
 
 // Decode attention for GQA groups of 4 or 8 on the tensor cores.
+// Key splits of the tensor-core decode attention (and keys per split, whole
+// 64-key chunks): one when the (sequence, KV head) grid covers every SM (two
+// CTAs fit on one), else about two CTAs per SM.  Clamped to [min_splits, max_splits].
+int mma_decode_splits(const llama_dims& d, int B, int T, int min_splits, int max_splits, int* kps_out) {
+  const int base = B * d.n_kv_heads;
+  int splits = base >= num_sms() ? 1 : cdiv(2 * num_sms(), base);
+  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 256))));
+  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, DEC_CHUNK)));
+  splits = std::max(std::min(min_splits, cdiv(T, DEC_CHUNK)), std::min(splits, max_splits));
+  const int kps = cdiv(cdiv(T, splits), DEC_CHUNK) * DEC_CHUNK;
+  if (kps_out != nullptr) *kps_out = kps;
+  return cdiv(T, kps);
+}
+
+struct RopeFuse {
+  float theta;
+  int style;
+};
+
 llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* kc, const void* vc, int capacity,
                              int B, int T, const __nv_bfloat16* qkv, int ld_qkv, __nv_bfloat16* out,
                              float* part_ml, float* part_o, DevStatus* status, int min_splits, int max_splits,
-                             const SeqTab* tab) {
+                             const SeqTab* tab, const RopeFuse* rope = nullptr) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   CUtensorMap tk, tv;
   // a head_dim of 96 runs as 128: the second 64-dim box reads dims 64..95 and
@@ -935,13 +964,14 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
   p.tab = tab;
-  const int base = B * d.n_kv_heads;
-  int splits = cdiv(2 * num_sms(), base);
-  splits = std::max(1, std::min(splits, std::min(kMaxAttnSplits, cdiv(T, 256))));
-  if (forced_decode_splits() > 0) splits = std::min(forced_decode_splits(), std::min(kMaxAttnSplits, cdiv(T, DEC_CHUNK)));
-  splits = std::max(std::min(min_splits, cdiv(T, DEC_CHUNK)), std::min(splits, max_splits));
-  int kps = cdiv(cdiv(T, splits), DEC_CHUNK) * DEC_CHUNK;
-  splits = cdiv(T, kps);
+  int kps = 0;
+  const int splits = mma_decode_splits(d, B, T, min_splits, max_splits, &kps);
+  if (rope != nullptr && splits != 1) return LLAMA_ERR_UNSUPPORTED;
+  p.kc = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(kc));
+  p.vc = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(vc));
+  p.cap = capacity;
+  p.theta = rope != nullptr ? rope->theta : 0.f;
+  p.rope_style = rope != nullptr ? rope->style : 0;
   p.splits = splits;
   p.keys_per_split = kps;
   dim3 grid(splits, d.n_kv_heads, B);
@@ -949,7 +979,8 @@ llama_status attn_decode_mma(cudaStream_t st, const llama_dims& d, const void* k
   {
     TRACE(K_ATTN_DECODE, st);
 #define DEC_MMA_CASE(HD_, G_) \
-    if ((hd == HD_ || (HD_ == 128 && hd == 96)) && grp == G_) r = launch_attn_decode_mma<HD_, G_>(tk, tv, p, grid, st);
+    if ((hd == HD_ || (HD_ == 128 && hd == 96)) && grp == G_) \
+      r = launch_attn_decode_mma<HD_, G_>(tk, tv, p, grid, st, rope != nullptr);
     DEC_MMA_CASE(128, 8) else DEC_MMA_CASE(128, 4) else DEC_MMA_CASE(128, 2) else DEC_MMA_CASE(128, 1)
     else DEC_MMA_CASE(64, 8) else DEC_MMA_CASE(64, 4) else DEC_MMA_CASE(64, 2) else DEC_MMA_CASE(64, 1)
 #undef DEC_MMA_CASE
@@ -993,18 +1024,14 @@ bool rope_fuse_enabled() {
 }
 
 // Whether the decode attention over keys [0, T) does RoPE + KV append itself
-// (attn_decode_bf16 with `rope`): the CUDA-core kernel with one key split, so
-// that one CTA owns the new token's q heads and k/v row of its KV head.
+// (attn_decode_bf16 with `rope`): either kernel with one key split, so that
+// one CTA owns the new token's q heads and k/v row of its KV head.
 bool decode_rope_fusable(const llama_dims& d, int B, int T, int min_splits = 1, int max_splits = kMaxAttnSplits) {
   if (!rope_fuse_enabled() || d.dtype != LLAMA_BF16) return false;
-  if (use_decode_mma(d.head_dim, d.n_heads / d.n_kv_heads)) return false;
+  if (use_decode_mma(d.head_dim, d.n_heads / d.n_kv_heads))
+    return mma_decode_splits(d, B, T, min_splits, max_splits, nullptr) == 1;
   return simt_decode_splits(d, B, T, min_splits, max_splits, nullptr) == 1;
 }
-
-struct RopeFuse {
-  float theta;
-  int style;
-};
 
 // Decode attention of one new token per sequence over keys [0, T).  Splits of
 // the key range are chosen by a heuristic, clamped to [min_splits, max_splits].
@@ -1018,11 +1045,9 @@ llama_status attn_decode_bf16(cudaStream_t st, const llama_dims& d, const void* 
                               int max_splits = kMaxAttnSplits, const SeqTab* tab = nullptr,
                               const RopeFuse* rope = nullptr) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
-  if (use_decode_mma(hd, grp)) {
-    if (rope != nullptr) return LLAMA_ERR_UNSUPPORTED;
+  if (use_decode_mma(hd, grp))
     return attn_decode_mma(st, d, kc, vc, capacity, B, T, qkv, ld_qkv, out, part_ml, part_o, status, min_splits,
-                           max_splits, tab);
-  }
+                           max_splits, tab, rope);
   AttnDecodeParams p{};
   p.qkv = qkv;
   p.ld_qkv = ld_qkv;
@@ -1081,7 +1106,7 @@ bool decode_layer_fusable(const llama_dims& d, int B, int T) {
   const int hd = d.head_dim, grp = d.n_heads / d.n_kv_heads;
   if (!on || d.dtype != LLAMA_BF16 || B < 1 || B > DL_BN) return false;
   if (!(hd == 64 || hd == 96 || hd == 128) || !(grp == 1 || grp == 2)) return false;
-  if (use_decode_mma(hd, grp)) return false;   // forced tensor-core decode attention (LLAMA_DECODE_ATTN=mma)
+  if (decode_attn_forced() == 1) return false;   // forced tensor-core decode attention (LLAMA_DECODE_ATTN=mma)
   if (d.dim % 64 != 0 || cdiv(d.dim, 128) > kMaxNormTiles || num_sms() > kMaxSkGrid) return false;
   return B * d.n_kv_heads <= 2 * num_sms() || T <= 2048;
 }

@@ -816,11 +816,53 @@ struct AttnDecodeMmaParams {
   DevStatus* status;
   unsigned long long limit_ns;
   const SeqTab* tab;          // ragged: sequence b sees tab->p0[b] + 1 keys; nullptr: all see T
+  // RoPE + KV append fused in (one key split; see AttnDecodeParams)
+  __nv_bfloat16* kc;          // the caches, for the append of the new token's row
+  __nv_bfloat16* vc;
+  int cap;
+  float theta;
+  int rope_style;
 };
+
+// RoPE of the new token (position pos) for KV head g of sequence b, by one
+// warp: the G query heads are rotated in place in qkv, the rotated key and the
+// value go to cache row pos.  Rounds like the stand-alone RoPE kernel.
+// cs / sn: the position's angles (dec_rope_angles_warp, then __syncwarp).
+__device__ __forceinline__ void dec_rope_angles_warp(const AttnDecodeMmaParams& p, int pos, float* cs, float* sn) {
+  for (int i = (int)(threadIdx.x & 31); i < (p.hd >> 1); i += 32) rope_cos_sin(pos, i, p.hd, p.theta, cs[i], sn[i]);
+}
+
+template <int G>
+__device__ __forceinline__ void dec_rope_append_warp(const AttnDecodeMmaParams& p, int b, int g, int pos,
+                                                     const float* cs, const float* sn) {
+  const int lane = threadIdx.x & 31, hd = p.hd, half = hd >> 1;
+  __nv_bfloat16* row = const_cast<__nv_bfloat16*>(p.qkv) + (size_t)b * p.ld_qkv;
+  const size_t crow = (((size_t)b * p.nkv + g) * p.cap + pos) * hd;
+  for (int h = 0; h <= G; ++h) {   // the G query heads, then the key head
+    __nv_bfloat16* src = row + (size_t)(h < G ? g * G + h : p.nh + g) * hd;
+    __nv_bfloat16* dst = h < G ? src : p.kc + crow;
+    for (int i = lane; i < half; i += 32) {
+      // rotate-half pairs (i, i + hd/2), interleaved pairs (2i, 2i + 1)
+      const int i0 = p.rope_style == 0 ? i : 2 * i, i1 = p.rope_style == 0 ? i + half : 2 * i + 1, pi = i;
+      // each pair is read and written by one lane, so q can rotate in place
+      const float x0 = __bfloat162float(src[i0]), x1 = __bfloat162float(src[i1]);
+      const float c = cs[pi], s = sn[pi];
+      dst[i0] = __float2bfloat16_rn(rope_lo(x0, x1, c, s));
+      dst[i1] = __float2bfloat16_rn(rope_hi(x0, x1, c, s));
+    }
+  }
+  const __nv_bfloat16* v = row + (size_t)(p.nh + p.nkv + g) * hd;
+  for (int i = lane; i < hd; i += 32) p.vc[crow + i] = v[i];
+  __syncwarp();
+}
 
 // ST stages and ST consumer warps: warp w takes chunks w, w + ST, ... so each
 // stage has one consumer, and its full / empty phases alternate in chunk order.
-template <int HD, int G, int ST>
+// ROPE (one key split): qkv holds the raw projections.  The producer warp
+// computes the angles before the PDL wait, puts the chunks that do not hold
+// the new token's row in flight, rotates q and the new key and appends the new
+// k / v row, and only then loads the last chunk (which holds that row).
+template <int HD, int G, int ST, bool ROPE>
 __global__ void __launch_bounds__(32 * (ST + 1), 1)
     attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const AttnDecodeMmaParams p) {
@@ -838,8 +880,12 @@ __global__ void __launch_bounds__(32 * (ST + 1), 1)
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float rcs[ROPE ? HD / 2 : 1], rsn[ROPE ? HD / 2 : 1];
+  // the new token's angles overlap the previous kernel (position known up front)
+  if (ROPE && p.tab == nullptr && warp == 0) dec_rope_angles_warp(p, p.T - 1, rcs, rsn);
   if (p.tab != nullptr) pdl_wait();   // the ragged table is written by an earlier kernel
   const int T = p.tab != nullptr ? p.tab->p0[b] + 1 : p.T;
+  if (ROPE && p.tab != nullptr && warp == 0) dec_rope_angles_warp(p, T - 1, rcs, rsn);
   const int j0 = split * p.keys_per_split;
   const int j1 = min(T, j0 + p.keys_per_split);
   const int n_chunks = j1 > j0 ? (j1 - j0 + DEC_CHUNK - 1) / DEC_CHUNK : 0;
@@ -857,26 +903,48 @@ __global__ void __launch_bounds__(32 * (ST + 1), 1)
   __syncthreads();
   pdl_wait();
   WaitCtx wc{&abort_sh, p.status, p.limit_ns, 4};
+  const int zkv = b * p.nkv + g;
+  int last_fill[DEC_STAGES];
+  for (int s = 0; s < DEC_STAGES; ++s) last_fill[s] = -1;
+  int c_next = 0;   // producer: the next chunk to fill
+  auto fill = [&](int c) -> bool {
+    const int s = c % DEC_STAGES;
+    if (!mbar_wait(empty_bar(s), ((c / DEC_STAGES) & 1) ^ 1u, wc, 1)) return false;
+    uint8_t* st = smem + s * C::STAGE;
+    mbar_arrive_expect_tx(full_bar(s), C::STAGE);
+    const int key0 = j0 + c * DEC_CHUNK;
+    for (int r = 0; r < C::NREG; ++r) {
+      tma_load_3d(smem_u32(st + r * DEC_REGION), &tmK, full_bar(s), r * 64, key0, zkv);
+      tma_load_3d(smem_u32(st + (C::NREG + r) * DEC_REGION), &tmV, full_bar(s), r * 64, key0, zkv);
+    }
+    last_fill[s] = c;
+    return true;
+  };
+  if (ROPE) {
+    if (warp == 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        // the chunks before the one holding row T - 1 do not depend on this step
+        while (c_next < min(DEC_STAGES, n_chunks - 1) && fill(c_next)) ++c_next;
+      }
+      __syncwarp();
+      dec_rope_append_warp<G>(p, b, g, T - 1, rcs, rsn);
+    }
+    __syncthreads();   // the consumers read the rotated q; the new row is written
+  }
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      const int zkv = b * p.nkv + g;
-      int last_fill[DEC_STAGES];
-      for (int s = 0; s < DEC_STAGES; ++s) last_fill[s] = -1;
-      for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % DEC_STAGES;
-        if (!mbar_wait(empty_bar(s), ((c / DEC_STAGES) & 1) ^ 1u, wc, 1)) break;
-        uint8_t* st = smem + s * C::STAGE;
-        mbar_arrive_expect_tx(full_bar(s), C::STAGE);
-        const int key0 = j0 + c * DEC_CHUNK;
-        for (int r = 0; r < C::NREG; ++r) {
-          tma_load_3d(smem_u32(st + r * DEC_REGION), &tmK, full_bar(s), r * 64, key0, zkv);
-          tma_load_3d(smem_u32(st + (C::NREG + r) * DEC_REGION), &tmV, full_bar(s), r * 64, key0, zkv);
-        }
-        last_fill[s] = c;
+      if (ROPE) {
+        // the new row was written by the warp's lanes through the generic proxy
+        // (ordered before this thread by the barrier); the fills read it by TMA
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      } else {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
       }
+      while (c_next < n_chunks && fill(c_next)) ++c_next;
       for (int s = 0; s < DEC_STAGES; ++s)
         if (last_fill[s] >= 0) mbar_wait(full_bar(s), (last_fill[s] / DEC_STAGES) & 1, wc, 9, false);
     }
@@ -893,13 +961,14 @@ __global__ void __launch_bounds__(32 * (ST + 1), 1)
         const int k0 = ks * 16 + qd * 2;
         uint32_t lo = 0, hi = 0, lo8 = 0, hi8 = 0;
         // dims past head_dim stay zero (head_dim is a multiple of 16 here)
+        // through L2: with ROPE the row was just rewritten by this CTA's producer warp
         if (r0 < G && k0 < hdm) {
-          lo = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * hdm + k0);
-          lo8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)r0 * hdm + k0 + 8);
+          lo = __ldcg(reinterpret_cast<const unsigned int*>(qrow0 + (size_t)r0 * hdm + k0));
+          lo8 = __ldcg(reinterpret_cast<const unsigned int*>(qrow0 + (size_t)r0 * hdm + k0 + 8));
         }
         if (r0 + 8 < G && k0 < hdm) {
-          hi = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * hdm + k0);
-          hi8 = *reinterpret_cast<const uint32_t*>(qrow0 + (size_t)(r0 + 8) * hdm + k0 + 8);
+          hi = __ldcg(reinterpret_cast<const unsigned int*>(qrow0 + (size_t)(r0 + 8) * hdm + k0));
+          hi8 = __ldcg(reinterpret_cast<const unsigned int*>(qrow0 + (size_t)(r0 + 8) * hdm + k0 + 8));
         }
         qa[ks][0] = lo;
         qa[ks][1] = hi;

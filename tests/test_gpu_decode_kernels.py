@@ -75,15 +75,16 @@ def _child_runs(tmp_path, rope, batch, envs):
     return res
 
 
+@pytest.mark.parametrize("kernel", ["simt", "mma"])
 @pytest.mark.parametrize("rope", ["half", "interleaved"])
-def test_rope_inside_attention_is_bit_identical_to_the_rope_kernel(tmp_path, rope):
-    """RoPE + KV append inside the decode attention (batch 40: one key split per
-    (sequence, KV head)) rounds exactly like the stand-alone kernel: the same
-    rotated q and appended k / v bits; the block output differs only by the
-    order in which the new key joins the softmax."""
+def test_rope_inside_attention_is_bit_identical_to_the_rope_kernel(tmp_path, rope, kernel):
+    """RoPE + KV append inside either decode attention kernel (batch 40: one key
+    split per (sequence, KV head)) rounds exactly like the stand-alone kernel:
+    the same rotated q and appended k / v bits; the block output differs only
+    by the order in which the new key joins the softmax."""
     res = _child_runs(tmp_path, rope, 40, {
-        "fused": {"LLAMA_DECODE_ATTN": "simt", "LLAMA_FUSE_ROPE": "1"},
-        "apart": {"LLAMA_DECODE_ATTN": "simt", "LLAMA_FUSE_ROPE": "0"}})
+        "fused": {"LLAMA_DECODE_ATTN": kernel, "LLAMA_FUSE_ROPE": "1"},
+        "apart": {"LLAMA_DECODE_ATTN": kernel, "LLAMA_FUSE_ROPE": "0"}})
     a, b = res["fused"], res["apart"]
     for t in range(2):
         for n in ("q", "k", "v"):
