@@ -10,9 +10,11 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <new>
 #include <set>
+#include <tuple>
 #include <utility>
 #include <unordered_map>
 #include <vector>
@@ -339,6 +341,27 @@ cudaError_t launch_k_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same for a kernel whose CTAs run in clusters of `cl` CTAs along x; grid.x is a multiple of cl.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k_cluster(void (*kernel)(KArgs...), int cl, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // cudaFuncSetAttribute acts on the current device only, so a kernel's dynamic
 // shared-memory limit is raised once per (kernel, device) pair.
 llama_status ensure_smem_attr(const void* kernel, int bytes) {
@@ -506,9 +529,108 @@ struct NormFuse {
   float eps;
 };
 
+// Cluster-split form of a decode GEMM: one weight tile per cluster of p.cl_split CTAs.
+template <int BN, int EPI>
+llama_status launch_gemm_cl(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
+                            cudaStream_t st, int kind) {
+  using C = GemmCfg<BN, false, 2, true>;
+  auto* k = gemm_tc_kernel<BN, true, EPI, 2, true>;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(k), C::SMEM_BYTES));
+  {
+    TRACE(kind, st);
+    CUDA_TRY(launch_k_cluster(k, p.cl_split, grid, GEMM_THREADS, C::SMEM_BYTES, st, a, w[0], w[1], w[2], p));
+  }
+  LAUNCH_CHECK();
+  return LLAMA_OK;
+}
+
+// Largest cluster the CL kernel of this width can reduce in shared memory
+// (the form exists for up to 16 token rows).
+int cl_max_split(int BN) { return BN == 16 ? kMaxClusterSplit : 0; }
+
+// True when every cluster of `cl` CTAs of the CL kernel (BN, epi) fits on the
+// device at once (`clusters` of them).  Cached per (BN, epi, cl, device).
+bool clusters_fit(int BN, int epi, int cl, int clusters) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
+  std::lock_guard<std::mutex> g(mu);
+  const auto key = std::make_tuple(BN, epi, cl, dev);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    const void* k = nullptr;
+    int smem = 0;
+    auto pick = [&](auto kern, int bytes) {
+      k = reinterpret_cast<const void*>(kern);
+      smem = bytes;
+    };
+    using C = GemmCfg<16, false, 2, true>;
+    if (epi == EPI_BF16) pick(gemm_tc_kernel<16, true, EPI_BF16, 2, true>, C::SMEM_BYTES);
+    else if (epi == EPI_RESID_F32) pick(gemm_tc_kernel<16, true, EPI_RESID_F32, 2, true>, C::SMEM_BYTES);
+    else pick(gemm_tc_kernel<16, true, EPI_SWIGLU_BF16, 2, true>, C::SMEM_BYTES);
+    int n = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3((unsigned)(cl * clusters));
+      cfg.blockDim = dim3(GEMM_THREADS);
+      cfg.dynamicSmemBytes = (size_t)smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)cl;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    it = cache.emplace(key, n).first;
+  }
+  return it->second >= clusters;
+}
+
+// A decode GEMM of at most 16 token rows whose weight tiles number at most
+// the SM count runs as one cluster per tile, its k-blocks split over the
+// cluster's CTAs and their pieces added in the rank-0 CTA's shared memory
+// instead of through L2 and flags, when that keeps at least 3/4 of the SMs
+// busy.  LLAMA_DECODE_CLUSTER=0 keeps every decode GEMM stream-K; =2 takes
+// clusters whatever the SM share (tests of small shapes).  Returns the
+// cluster size, 0 for stream-K.
+int decode_cluster_split(int n_tiles, int num_kb, int BN, int KS, int epi) {
+  static const int mode = [] {
+    const char* e = std::getenv("LLAMA_DECODE_CLUSTER");
+    return e == nullptr ? 1 : e[0] == '0' ? 0 : e[0] == '2' ? 2 : 1;
+  }();
+  // LLAMA_DECODE_CLUSTER_MIN=s: use clusters of at least s CTAs only
+  static const int min_split = [] {
+    const char* e = std::getenv("LLAMA_DECODE_CLUSTER_MIN");
+    const int v = e != nullptr ? std::atoi(e) : 1;
+    return v < 1 ? 1 : v;
+  }();
+  if (mode == 0 || KS != 2 || epi == EPI_F32 || cl_max_split(BN) < 1 || n_tiles <= 0) return 0;
+  const int sms = num_sms();
+  auto busy = [&](int S) { return mode == 2 || 4 * n_tiles * S >= 3 * sms; };
+  int S = std::min({cl_max_split(BN), sms / n_tiles, num_kb});
+  if (S < min_split || !busy(S)) return 0;
+  while (S >= min_split && !clusters_fit(BN, epi, S, n_tiles)) --S;
+  if (S < min_split || !busy(S)) return 0;
+  return S;
+}
+
 template <int BN, int KS>
 llama_status launch_gemm_sk(int epi, const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
                             cudaStream_t st, int kind) {
+  if constexpr (KS == 2 && BN == 16) {
+    if (p.cl_split > 0) {
+      switch (epi) {
+        case EPI_BF16: return launch_gemm_cl<BN, EPI_BF16>(a, w, p, grid, st, kind);
+        case EPI_RESID_F32: return launch_gemm_cl<BN, EPI_RESID_F32>(a, w, p, grid, st, kind);
+        case EPI_SWIGLU_BF16: return launch_gemm_cl<BN, EPI_SWIGLU_BF16>(a, w, p, grid, st, kind);
+      }
+      return LLAMA_ERR_INVALID_ARG;
+    }
+  }
   switch (epi) {
     case EPI_BF16: return launch_gemm_tc<BN, true, EPI_BF16, KS>(a, w, p, grid, st, kind);
     case EPI_RESID_F32: return launch_gemm_tc<BN, true, EPI_RESID_F32, KS>(a, w, p, grid, st, kind);
@@ -674,6 +796,11 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
     p.norm_eps = norm->eps;
     p.ssq = sk.ssq;
     p.norm_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsNormCtrOffset);
+  }
+  if (const int cl = decode_cluster_split(p.n_tiles, p.num_kb, BN, KS, epi); cl > 0) {
+    p.cl_split = cl;
+    grid = p.n_tiles * cl;
+    p.sk_grid = grid;
   }
   if (KS == 2) {
     switch (BN) {

@@ -40,6 +40,12 @@
 //    order (deterministic) and applies the epilogue itself.  For gate_up a
 //    weight tile is 64 gate rows followed by the matching 64 up rows, so
 //    SiLU(gate)·up pairs TMEM lane r with lane r + 64 (through shared memory).
+//    Cluster form (CL, at most 16 token rows, weight tiles <= SMs): one
+//    thread-block cluster of S <= 8 CTAs per weight tile, each CTA taking
+//    1/S of its k-blocks; ranks 1..S-1 store their fp32 pieces straight into
+//    rank 0's shared memory (st.shared::cluster) and arrive on its mbarrier,
+//    rank 0 adds them in rank order and applies the epilogue -- no L2 round
+//    trip, flag word or wait on another cluster.
 //
 // The weight can be given as up to three row segments with their own tensor
 // maps (q, k, v when the three projections are not contiguous; gate and up).
@@ -92,6 +98,10 @@ struct GemmParams {
   float* ssq;          // [n_tiles][BN]: per tile, the sum of squares of each token row's columns
   unsigned* norm_ctr;  // [2]: tiles finished, CTAs finished normalising (nullptr: ssq only)
   int sk_grid;         // stream-K: CTAs 0 .. sk_grid-1 share the units (<= gridDim.x, <= units)
+  // cluster split (the CL kernel form): weight tile blockIdx.x / cl_split, its
+  // k-blocks split over the cl_split CTAs of one thread-block cluster; ranks
+  // 1.. store their fp32 pieces into rank 0's shared memory, which adds them
+  int cl_split;
 };
 
 constexpr int GEMM_EPI_WARPS = 8;
@@ -100,7 +110,14 @@ constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 // PAIR: tile mode on a CTA pair (M = 256 per MMA); this CTA holds 128 rows of
 // A and BN / 2 rows of B per stage.  KS: 64-wide k sub-blocks per unit (decode:
 // a stage then reads KS x 128 contiguous bytes of every weight row).
-template <int BN, bool PAIR, int KS = 1>
+// CL: the cluster-split decode form (BN = 16), whose rank 0 also holds up to
+// kMaxClusterSplit - 1 pieces of [128][BN] fp32.  Fewer stages make room, so
+// that its shared memory stays within the plain form's: both then leave the
+// SM the same L1 share for the kernel that follows under PDL (the CUDA-core
+// decode attention streams the cache through L1).
+constexpr int kMaxClusterSplit = 8;
+
+template <int BN, bool PAIR, int KS = 1, bool CL = false>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_SUB = BM * BK * 2;
@@ -108,12 +125,15 @@ struct GemmCfg {
   static constexpr int A_BYTES = KS * A_SUB;
   static constexpr int B_BYTES = KS * B_SUB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int CL_BYTES = CL ? (kMaxClusterSplit - 1) * 128 * BN * 4 : 0;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static constexpr int STAGES_PLAIN = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+  static constexpr int STAGES = (STAGES_PLAIN * STAGE_BYTES - CL_BYTES) / STAGE_BYTES;
+  static_assert(STAGES >= 2, "pipeline depth");
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                         : (2 * BN <= 256) ? 256 : 512;
   static constexpr int EXCH_BYTES = 2 * 64 * 16 * 4;   // gate/up pairing exchange (stream-K gate_up)
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + EXCH_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + EXCH_BYTES + CL_BYTES;
 };
 
 // Work item shared by the three roles: one output tile and a k-block range.
@@ -137,6 +157,11 @@ struct GemmIter {
       next_tile = blockIdx.x >> 1;
       tile_stride = gridDim.x >> 1;
       tile_count = p.m_tiles * p.n_tiles;
+    } else if (p.cl_split > 0) {
+      // one weight tile per cluster; this CTA's share of its k-blocks
+      const long long S = p.cl_split, r = blockIdx.x % S, t = blockIdx.x / S;
+      u0 = t * num_kb + num_kb * r / S;
+      u = t * num_kb + num_kb * (r + 1) / S;
     } else {
       const long long G = p.sk_grid;
       if ((long long)blockIdx.x >= G) {
@@ -186,6 +211,18 @@ __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
   return s;
 }
 
+// mbarrier wait whose acquire covers writes that other CTAs of the cluster
+// released into this CTA's shared memory before arriving.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Stream-K epilogue of one work item (decode form): the accumulator holds
 // TMEM lane `row` = weight row of the tile, column j = token j.  A piece that
 // does not end its tile is published for the tile's finisher; the CTA that
@@ -193,12 +230,34 @@ __device__ __forceinline__ int seg_of_tile(const GemmParams& p, int wtile) {
 // and applies the epilogue.  Called by every epilogue thread; `leader` is one
 // of them (it handles the flag words), `xch` this thread's half of the
 // gate/up exchange buffer in shared memory.
-template <int BN, int EPI, typename Sync>
+template <int BN, int EPI, typename Sync, bool CL = false>
 __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const GemmItem& item, uint32_t tbase, int row,
                                                  int half, float* xch, bool leader, int* abort_sh, Sync& epi_sync,
-                                                 float (*red)[16]) {
+                                                 float (*red)[16], float* cl_buf = nullptr, uint32_t red_bar = 0) {
   // accumulator: TMEM lane `row` = weight row of the tile, column j = token j
-  if (item.kb1 < p.num_kb) {
+  const uint32_t cl_rank = CL ? blockIdx.x % (unsigned)p.cl_split : 0u;
+  if (CL && cl_rank > 0) {
+    // a piece of the cluster's tile: into slot rank - 1 of rank 0's shared memory
+    const uint32_t dst = mapa_shared(smem_u32(cl_buf + ((size_t)(cl_rank - 1) * 128 + row) * BN), 0);
+#pragma unroll 1
+    for (int c = half * 16; c < BN; c += 32) {
+      float v[16];
+      tmem_ld16(tbase + c, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(c + 4 * q) * 4u),
+                     "f"(v[4 * q]), "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
+                     : "memory");
+    }
+    epi_sync();
+    if (leader) {
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      mbar_arrive_remote(mapa_shared(red_bar, 0));
+    }
+    return;
+  }
+  if (!CL && item.kb1 < p.num_kb) {
     // a piece that does not end its tile: publish it for the tile's finisher
     float* dst = p.partial + ((size_t)blockIdx.x * 128 + row) * BN;
 #pragma unroll 1
@@ -221,9 +280,23 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
     const unsigned x = (unsigned)item.tile * KB;
     int c_first = (int)(((x + 1) * G + U - 1) / U) - 1;
     c_first = c_first < 0 ? 0 : c_first;
-    // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count)
-    const int n_contrib = (int)blockIdx.x - c_first;
-    if (n_contrib > 0) {
+    // CTAs c_first .. blockIdx.x-1 (none has an empty range: the grid is at most the unit count);
+    // cluster split: ranks 1 .. cl_split - 1, from this CTA's shared memory
+    const int n_contrib = CL ? p.cl_split - 1 : (int)blockIdx.x - c_first;
+    if (CL && n_contrib > 0) {
+      if (leader) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_cluster(red_bar, 0)) {
+          if (*reinterpret_cast<volatile int*>(abort_sh)) break;
+          if (globaltimer_ns() - t0 > p.limit_ns) {
+            *abort_sh = 1;
+            record_error(p.status, LLAMA_ERR_DEVICE_TIMEOUT, 14, item.tile);
+            break;
+          }
+        }
+      }
+      epi_sync();
+    } else if (n_contrib > 0) {
       // the first epilogue warp waits for the contributors' flags, one lane
       // each, so the waits overlap (one L2 round trip instead of one per piece)
       if ((threadIdx.x >> 5) == 2) {
@@ -269,8 +342,9 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
       if (active) {
         tmem_ld16(tbase + c, v);
         tmem_ld_wait();
-        // the contributors' pieces, in CTA order, up to four per round trip to L2
-        const float4* src = reinterpret_cast<const float4*>(p.partial + ((size_t)c_first * 128 + row) * BN + c);
+        // the contributors' pieces, in CTA (rank) order, up to four per round trip
+        const float4* src = reinterpret_cast<const float4*>(
+            CL ? cl_buf + (size_t)row * BN + c : p.partial + ((size_t)c_first * 128 + row) * BN + c);
         constexpr size_t STRIDE4 = (size_t)128 * BN / 4;
 #pragma unroll 1
         for (int k = 0; k < n_contrib; k += 4) {
@@ -279,7 +353,8 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              a[i][q] = k + i < n_contrib ? __ldcg(src + (size_t)(k + i) * STRIDE4 + q)
+              a[i][q] = k + i < n_contrib ? (CL ? src[(size_t)(k + i) * STRIDE4 + q]
+                                                : __ldcg(src + (size_t)(k + i) * STRIDE4 + q))
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -420,20 +495,21 @@ __device__ __forceinline__ void fused_rmsnorm(const GemmParams& p, bool leader, 
   }
 }
 
-template <int BN, bool SWAP, int EPI, int KS = 1>
+template <int BN, bool SWAP, int EPI, int KS = 1, bool CL = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW0,
                    const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                    const GemmParams p) {
   constexpr bool PAIR = !SWAP;            // tile mode runs 256 x BN tiles on CTA pairs
   static_assert(KS == 1 || SWAP, "k sub-blocks are a decode (stream-K) form");
-  using C = GemmCfg<BN, PAIR, KS>;
+  static_assert(!CL || (SWAP && BN == 16), "the cluster split is a decode form of 16 token columns");
+  using C = GemmCfg<BN, PAIR, KS, CL>;
   constexpr int STAGES = C::STAGES;
   constexpr int WROWS = SWAP ? 128 : BN;  // weight rows per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, epilogue group
+  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, epilogue group, cluster pieces
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float red_sh[SWAP ? GEMM_EPI_WARPS : 1][16];   // fused RMSNorm: per-warp sums
@@ -449,6 +525,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
   const uint32_t epi_bar = bar0 + 8u * (2 * STAGES + 5);
+  const uint32_t red_bar = bar0 + 8u * (2 * STAGES + 6);
+  static_assert(8 * (2 * STAGES + 7) <= 256, "barrier block");
+  // cluster split: the other ranks' pieces, in rank 0's shared memory
+  float* cl_buf = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256 + C::EXCH_BYTES);
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -463,6 +543,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     mbar_init(drain_bar, 1);
     mbar_init(epi_bar, 32 * GEMM_EPI_WARPS);
+    if (CL) mbar_init(red_bar, p.cl_split > 1 ? p.cl_split - 1 : 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -482,8 +563,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
   tc_fence_before();
   // pair: the peer's TMA loads and the leader's commits target barriers of the
-  // other CTA, so both must be initialised before either proceeds
-  if constexpr (PAIR) cluster_sync(); else __syncthreads();
+  // other CTA, so both must be initialised before either proceeds (cluster
+  // split: the other ranks arrive on rank 0's red_bar)
+  if constexpr (PAIR || CL) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (p.early_trigger) pdl_trigger();
   // stream-K (decode): the producer starts the weight stream before its PDL wait
@@ -702,9 +784,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(abuf * BN);
       if constexpr (SWAP) {
-        streamk_epilogue<BN, EPI>(p, item, tbase, row, half,
-                                  reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16),
-                                  threadIdx.x == 64, &abort_sh, epi_sync, red_sh);
+        streamk_epilogue<BN, EPI, decltype(epi_sync), CL>(
+            p, item, tbase, row, half,
+            reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256) + half * (64 * 16), threadIdx.x == 64,
+            &abort_sh, epi_sync, red_sh, cl_buf, red_bar);
       } else {
         int mt, wtile;
         tile_coords(p, item.tile, mt, wtile);
@@ -905,8 +988,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   pdl_trigger();   // the next kernel may start its prologue while this CTA tears down
   tc_fence_before();
   // pair: neither CTA leaves while the other may still use its shared memory
-  // (rank 0's MMAs read rank 1's stages; rank 1's epilogue arrives on rank 0)
-  if constexpr (PAIR) cluster_sync(); else __syncthreads();
+  // (rank 0's MMAs read rank 1's stages; rank 1's epilogue arrives on rank 0);
+  // cluster split: rank 0 stays while the others may still store their pieces
+  if constexpr (PAIR || CL) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     if constexpr (PAIR) {

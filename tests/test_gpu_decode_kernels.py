@@ -8,8 +8,11 @@ the fp64 oracle) in a child process, together with the full-size 13B-shaped
 decode check.  The same child runs cover the other decode forms: RoPE + KV
 append kept apart from the CUDA-core attention (LLAMA_FUSE_ROPE=0), the
 persistent decode-block kernel at batch <= 16 instead of a kernel per step
-(LLAMA_DECODE_LAYER=1), and the RMSNorms taken into the ends of the residual
-GEMMs (LLAMA_FUSE_NORM=1).
+(LLAMA_DECODE_LAYER=1), the RMSNorms taken into the ends of the residual
+GEMMs (LLAMA_FUSE_NORM=1), the decode GEMMs split over thread-block
+clusters whatever the SM share (LLAMA_DECODE_CLUSTER=2, where by default only
+the full-size shapes take clusters), and every decode GEMM kept stream-K
+(LLAMA_DECODE_CLUSTER=0).
 """
 
 import os
@@ -26,15 +29,22 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.mark.parametrize("kernel,extra", [("mma", {}), ("simt", {}), ("simt", {"LLAMA_FUSE_ROPE": "0"}),
                                           ("simt", {"LLAMA_DECODE_LAYER": "1"}),
-                                          ("mma", {"LLAMA_FUSE_NORM": "1"}), ("simt", {"LLAMA_FUSE_NORM": "1"})],
+                                          ("mma", {"LLAMA_FUSE_NORM": "1"}), ("simt", {"LLAMA_FUSE_NORM": "1"}),
+                                          ("mma", {"LLAMA_DECODE_CLUSTER": "2"}),
+                                          ("mma", {"LLAMA_DECODE_CLUSTER": "2", "LLAMA_FUSE_NORM": "1"}),
+                                          ("simt", {"LLAMA_DECODE_CLUSTER": "0"})],
                          ids=["mma", "simt", "simt-rope-apart", "simt-decode-block", "mma-norm-fused",
-                              "simt-norm-fused"])
+                              "simt-norm-fused", "mma-cluster-split", "mma-cluster-split-norm-fused",
+                              "simt-stream-k-only"])
 def test_decode_parity_with_each_attention_kernel(kernel, extra):
     env = dict(os.environ, LLAMA_DECODE_ATTN=kernel, **extra)
     targets = ["tests/test_gpu_layer.py", "-k", "decode"]
-    if extra.get("LLAMA_FUSE_NORM") == "1":
+    if extra.get("LLAMA_FUSE_NORM") == "1" or extra.get("LLAMA_DECODE_CLUSTER"):
         # a whole model chains each down GEMM into the next block's first RMSNorm
         targets = ["tests/test_gpu_layer.py", "tests/test_gpu_fullsize.py", "-k", "decode or phi3_two_layer"]
+    if extra.get("LLAMA_DECODE_CLUSTER"):
+        # the ragged batches' decode rows take the same GEMM forms
+        targets = targets[:-2] + ["tests/test_gpu_ragged.py", "-k", "decode or phi3_two_layer or ragged"]
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", "-m", "gpu"] + targets,
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
     print(r.stdout[-3000:])
