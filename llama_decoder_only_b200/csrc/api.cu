@@ -957,10 +957,25 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
 // Ragged batch (tab != nullptr): L is the longest sequence's new tokens, Mtot
 // the packed rows in all and T the most keys any sequence sees; the per-
 // sequence values come from the device table.
+// Prefill attention's key step: 64 keys (attn_prefill_k64_kernel, two S
+// buffers per query tile) for head_dim below 128, 128 keys (attn_prefill_kernel)
+// at 128, where the 64-key S MMAs re-read Q from shared memory twice as often
+// and measured slower.  LLAMA_ATTN_KSTEP=64 or 128 takes one kernel for all.
+bool attn_prefill_k64(int hd) {
+  static const int forced = [] {
+    const char* e = std::getenv("LLAMA_ATTN_KSTEP");
+    if (e == nullptr) return 0;
+    return std::strcmp(e, "64") == 0 ? 64 : std::strcmp(e, "128") == 0 ? 128 : 0;
+  }();
+  if (forced != 0) return forced == 64;
+  return hd < 128;
+}
+
 llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int L, int p0,
                                const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status,
                                const SeqTab* tab = nullptr, int Mtot = 0, int Tmax = 0) {
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(attn_prefill_kernel), ATT_SMEM));
+  auto* kernel = attn_prefill_k64(d.head_dim) ? attn_prefill_k64_kernel : attn_prefill_kernel;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(kernel), ATT_SMEM));
   const int hd = d.head_dim;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
   const int T = tab != nullptr ? Tmax : p0 + L;
@@ -1002,7 +1017,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   // heaviest query blocks dispatched first (see the kernel)
   dim3 grid(p.head_pair ? d.n_heads / 2 : d.n_heads, B, p.n_qblocks);
   TRACE(K_ATTN_PREFILL, st);
-  CUDA_TRY(launch_k(attn_prefill_kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
+  CUDA_TRY(launch_k(kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
   LAUNCH_CHECK();
   return LLAMA_OK;
 }

@@ -13,6 +13,9 @@
 //    ping-pong so one tile's softmax overlaps the other tile's MMAs.  The running max is only moved (and
 //    O rescaled) when it grows by more than 2^8, which is exact because the
 //    final division uses the same stale maximum for numerator and sum.
+//  * attn_prefill_k64_kernel (head_dim below 128): the same with 64-key
+//    steps and two S buffers per query tile, so a tile's next S is computed
+//    while its softmax runs.
 //  * attn_decode_kernel (and attn_decode_mma_kernel for GQA groups >= 4):
 //    one new query per sequence; the cache of each (sequence, KV head) is
 //    split along the key axis over several CTAs; the query heads of a GQA
@@ -384,6 +387,333 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_arrive(p_full(t));
     }
     if (ok && my_kv > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done(t), (my_kv - 1) & 1, wc, 12))) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((size_t)row_base + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
+      for (int c = 0; c < hd_pad; c += 32) {
+        float v[32];
+        tmem_ld32(tO + c, v);
+        tmem_ld_wait();
+        if (tok < Ls) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (c + 8 * q < hd) {
+              uint4 w;
+              w.x = pack_bf16x2(v[8 * q + 0] * inv, v[8 * q + 1] * inv);
+              w.y = pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv);
+              w.z = pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv);
+              w.w = pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c + 8 * q) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// The same work split with the key axis advanced 64 keys per step.  Each query
+// tile then has two S buffers of 64 TMEM columns (S_t at t * 128 + 64 (s & 1),
+// O_t at 256 + 128 t, as before), so S_t(s + 1) is computed while the softmax
+// works on S_t(s), and the softmax of one tile runs step after step instead of
+// waiting for its own P·V and next S.  P_t(s) (bf16 pairs) goes over the first
+// 32 columns of its S buffer.  The MMA warp issues, per step and tile, P·V of
+// step s and then S of step s + 2 into the buffer P_t(s) came from: tcgen05
+// MMAs of one thread run in order, so the P·V has read P before S overwrites
+// it, and the softmax, having seen S_t(s) complete, knows that every P·V up
+// to s - 2 has completed (a commit covers all earlier MMAs of its thread).
+// The softmax waits for the previous P·V only to rescale O.  K / V arrive as
+// 128-key tiles in the same 4-slot ring; step s reads rows 64 (s & 1) .. of
+// tile s / 2.
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_prefill_k64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const AttnPrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                                   // tile t at t * ATT_TILE
+  uint8_t* sKV = sQ + 2 * ATT_TILE;                     // slot s at s * ATT_TILE
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + ATT_SLOTS * ATT_TILE);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // heaviest query blocks first (grid.z), as in attn_prefill_kernel
+  const int qb = p.n_qblocks - 1 - blockIdx.z;
+  const int b = blockIdx.y;
+  const bool hp = p.head_pair != 0;
+  const int h0 = hp ? 2 * blockIdx.x : blockIdx.x;
+  const int g = h0 / (p.nh / p.nkv);
+  const int hd = p.hd;
+  const int nreg = hd > 64 ? 2 : 1;
+  const int hd_pad = nreg * 64;
+  const int q_row0 = qb * (hp ? 128 : 256);
+  const int qoff1 = hp ? 0 : 128;
+  int Ls = p.L, p0s = p.p0, row_base = b * p.L;
+  if (p.tab != nullptr) {
+    pdl_wait();   // the table is written by an earlier kernel
+    Ls = p.tab->len[b];
+    p0s = p.tab->p0[b];
+    row_base = p.tab->start[b];
+  }
+  const bool q0_valid = q_row0 < Ls;
+  const bool q1_valid = q_row0 + qoff1 < Ls;
+  // 64-key steps with any key visible to tile t (0 for an empty tile)
+  const int n_st0 = q0_valid ? (p0s + min(Ls, q_row0 + 128) - 1) / 64 + 1 : 0;
+  const int n_st1 = q1_valid ? (p0s + min(Ls, q_row0 + qoff1 + 128) - 1) / 64 + 1 : 0;
+  const int n_st = max(n_st0, n_st1);
+  const int n_kv = (n_st + 1) / 2;   // 128-key tiles to load
+
+  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t q_full = bar0;
+  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ATT_SLOTS + s); };
+  // per tile t and S buffer u
+  auto s_full = [&](int t, int u) { return bar0 + 8u * (1 + 2 * ATT_SLOTS + 2 * t + u); };
+  auto p_full = [&](int t, int u) { return bar0 + 8u * (5 + 2 * ATT_SLOTS + 2 * t + u); };
+  auto pv_done = [&](int t, int u) { return bar0 + 8u * (9 + 2 * ATT_SLOTS + 2 * t + u); };
+  const uint32_t drain = bar0 + 8u * (13 + 2 * ATT_SLOTS);
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ATT_SLOTS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t)
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(s_full(t, u), 1);
+        mbar_init(p_full(t, u), 128);
+        mbar_init(pv_done(t, u), 1);
+      }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  const uint32_t tmem = tmem_base_sh;
+  WaitCtx wc{&abort_sh, p.status, p.limit_ns, 3};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_fill[ATT_SLOTS];
+      for (int s = 0; s < ATT_SLOTS; ++s) last_fill[s] = -1;
+      const int nq = q1_valid ? 2 : (q0_valid ? 1 : 0);
+      mbar_arrive_expect_tx(q_full, nq * nreg * ATT_REGION);
+      for (int t = 0; t < nq; ++t)
+        for (int r = 0; r < nreg; ++r) {
+          const int col = (h0 + (hp ? t : 0)) * hd + r * 64, row = q_row0 + (t ? qoff1 : 0);
+          if (p.tab != nullptr)
+            tma_load_2d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, col, row_base + row);
+          else
+            tma_load_3d(smem_u32(sQ + t * ATT_TILE + r * ATT_REGION), &tmQ, q_full, col, row, b);
+        }
+      const int zkv = b * p.nkv + g;
+      for (int f = 0; f < 2 * n_kv; ++f) {   // fill f: K_{f/2} (f even) or V_{f/2} (f odd)
+        const int s = f % ATT_SLOTS;
+        if (!mbar_wait(kv_empty(s), ((f / ATT_SLOTS) & 1) ^ 1u, wc, 1)) break;
+        const CUtensorMap* m = (f & 1) ? &tmV : &tmK;
+        mbar_arrive_expect_tx(kv_full(s), nreg * ATT_REGION);
+        for (int r = 0; r < nreg; ++r)
+          tma_load_3d(smem_u32(sKV + s * ATT_TILE + r * ATT_REGION), m, kv_full(s), r * 64, (f >> 1) * 128, zkv);
+        last_fill[s] = f;
+      }
+      mbar_wait(q_full, 0, wc, 9, false);
+      for (int s = 0; s < ATT_SLOTS; ++s)
+        if (last_fill[s] >= 0) mbar_wait(kv_full(s), (last_fill[s] / ATT_SLOTS) & 1, wc, 9, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(128, hd_pad, 0, 1);   // V is MN-major
+      const int ksteps = hd / 16;
+      const int nst[2] = {n_st0, n_st1};
+      bool ok = mbar_wait(q_full, 0, wc, 2);
+      bool issued = false;
+      auto fill_ready = [&](int f) -> bool {   // fill f of the ring has landed
+        return mbar_wait(kv_full(f % ATT_SLOTS), (f / ATT_SLOTS) & 1, wc, 3);
+      };
+      // S_t(s) = Q_t K^T over keys 64 s .. 64 s + 63, into buffer s & 1
+      auto issue_s = [&](int t, int s) -> bool {
+        if (!fill_ready(2 * (s >> 1))) return false;
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + t * ATT_TILE);
+        const uint32_t aK = smem_u32(sKV + ((2 * (s >> 1)) % ATT_SLOTS) * ATT_TILE) + (uint32_t)((s & 1) * 64 * 128);
+        const uint32_t d = tmem + (uint32_t)(t * 128 + (s & 1) * 64);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t off = (ks >> 2) * ATT_REGION + (ks & 3) * 32;
+          umma_bf16(d, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(aK + off, 16, 1024), idesc_s,
+                    ks > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full(t, s & 1));
+        issued = true;
+        return true;
+      };
+      // O_t += P_t(s) V over the same 64 keys, P_t(s) the A operand in TMEM
+      auto issue_pv = [&](int t, int s) -> bool {
+        if (!mbar_wait(p_full(t, s & 1), (s >> 1) & 1, wc, 5)) return false;
+        if (!fill_ready(2 * (s >> 1) + 1)) return false;
+        tc_fence_after();
+        const uint32_t aV =
+            smem_u32(sKV + ((2 * (s >> 1) + 1) % ATT_SLOTS) * ATT_TILE) + (uint32_t)((s & 1) * 64 * 128);
+        const uint32_t pa = tmem + (uint32_t)(t * 128 + (s & 1) * 64);
+        for (int ks = 0; ks < 4; ++ks)   // 16 keys per MMA (8 TMEM columns of bf16 pairs)
+          umma_bf16_ts(tmem + 256 + t * 128, pa + 8 * ks, smem_desc_sw128(aV + ks * 16 * 128, ATT_REGION, 1024),
+                       idesc_o, (s > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(pv_done(t, s & 1));
+        return true;
+      };
+      for (int s = 0; s < 2 && ok; ++s)
+        for (int t = 0; t < 2 && ok; ++t)
+          if (s < nst[t]) ok = issue_s(t, s);
+      if (ok && n_st > 0) umma_commit(kv_empty(0));   // K_0: steps 0 and 1 issued
+      for (int s = 0; ok && s < n_st; ++s) {
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (s >= nst[t]) continue;
+          ok = issue_pv(t, s);
+          if (ok && s + 2 < nst[t]) ok = issue_s(t, s + 2);
+        }
+        if (!ok) break;
+        if (s & 1) {
+          // after step s (odd): V_{s/2} read by its last P·V, K_{(s+1)/2} by its last S
+          umma_commit(kv_empty((2 * (s >> 1) + 1) % ATT_SLOTS));
+          const int jk = (s + 1) >> 1;
+          if (jk < n_kv) umma_commit(kv_empty((2 * jk) % ATT_SLOTS));
+        }
+      }
+      if (issued) {
+        umma_commit(drain);
+        mbar_wait(drain, 0, wc, 8, false);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / correction / epilogue
+    const int t = (warp - 2) >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int tok = q_row0 + (t ? qoff1 : 0) + row;
+    const int pos = p0s + tok;
+    const int pos_min = p0s + q_row0 + (t ? qoff1 : 0);
+    const int h = h0 + (hp ? t : 0);
+    const int my_st = t == 0 ? n_st0 : n_st1;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int s = 0; s < my_st && ok; ++s) {
+      const int u = s & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full(t, u), (s >> 1) & 1, wc, 10))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[2][32];
+      tmem_ld32(tS + u * 64, sv[0]);
+      tmem_ld32(tS + u * 64 + 32, sv[1]);
+      tmem_ld_wait();
+      if (s * 64 + 63 > pos_min) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (s * 64 + i > pos) sv[i >> 5][i & 31] = -INFINITY;
+      }
+      float mr[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mr[k] = sv[0][k];
+#pragma unroll
+      for (int i = 4; i < 64; ++i) mr[i & 3] = fmaxf(mr[i & 3], sv[i >> 5][i & 31]);
+      const float mx = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3])) * p.scale_log2;
+      // the reference maximum moves only when it grew by more than 2^8
+      float alpha = 1.f;
+      const bool need = mx > m_used + 8.0f;
+      if (need) {
+        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mx);
+        m_used = mx;
+      }
+      const bool rescale = __any_sync(0xffffffffu, need && s > 0);
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      const float sc = p.scale_log2;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pw[2][16];
+#pragma unroll
+      for (int g2 = 0; g2 < 2; ++g2)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = ex2_approx(fmaf(sv[g2][2 * e], sc, -mref));
+          const float bb = ex2_approx(fmaf(sv[g2][2 * e + 1], sc, -mref));
+          ps[e & 3] += a + bb;
+          pw[g2][e] = pack_bf16x2(a, bb);
+        }
+      tmem_st16u(tS + u * 64, pw[0]);
+      tmem_st16u(tS + u * 64 + 16, pw[1]);
+      if (rescale) {
+        // O must hold every earlier step: wait for P·V of step s - 1 (those up
+        // to s - 2 completed before S_t(s), which the wait above saw)
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done(t, u ^ 1), ((s - 1) >> 1) & 1, wc, 11))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        l *= alpha;
+        if (hd_pad == 128) {
+          float v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(tO + 0, v0);
+          tmem_ld32(tO + 32, v1);
+          tmem_ld32(tO + 64, v2);
+          tmem_ld32(tO + 96, v3);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v0[i] *= alpha;
+            v1[i] *= alpha;
+            v2[i] *= alpha;
+            v3[i] *= alpha;
+          }
+          tmem_st32(tO + 0, v0);
+          tmem_st32(tO + 32, v1);
+          tmem_st32(tO + 64, v2);
+          tmem_st32(tO + 96, v3);
+        } else {
+          float v0[32], v1[32];
+          tmem_ld32(tO + 0, v0);
+          tmem_ld32(tO + 32, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v0[i] *= alpha;
+            v1[i] *= alpha;
+          }
+          tmem_st32(tO + 0, v0);
+          tmem_st32(tO + 32, v1);
+        }
+      }
+      tmem_st_wait();   // P (and a rescaled O) in TMEM before the MMA warp is told
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      tc_fence_before();
+      mbar_arrive(p_full(t, u));
+    }
+    // the last P·V (those before it completed before the last S)
+    const int sl = my_st - 1;
+    if (ok && my_st > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done(t, sl & 1), (sl >> 1) & 1, wc, 12))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       __nv_bfloat16* orow = p.out + ((size_t)row_base + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
