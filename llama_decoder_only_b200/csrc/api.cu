@@ -957,25 +957,29 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
 // Ragged batch (tab != nullptr): L is the longest sequence's new tokens, Mtot
 // the packed rows in all and T the most keys any sequence sees; the per-
 // sequence values come from the device table.
-// Prefill attention's key step: 64 keys (attn_prefill_k64_kernel, two S
-// buffers per query tile) for head_dim below 128, 128 keys (attn_prefill_kernel)
-// at 128, where the 64-key S MMAs re-read Q from shared memory twice as often
-// and measured slower.  LLAMA_ATTN_KSTEP=64 or 128 takes one kernel for all.
-bool attn_prefill_k64(int hd) {
+// Which prefill-attention kernel runs: 1 = attn_prefill_kernel (two query
+// tiles share each K/V tile, 128-key steps, one S buffer per tile), 2 =
+// attn_prefill_k64_kernel (the same with 64-key steps and two S buffers per
+// tile), 3 = attn_prefill_1t_kernel (one query tile, 128-key steps, two S
+// buffers).  Default: 2 for head_dim below 128, 1 at 128.
+// LLAMA_ATTN_FORM=pair | k64 | one takes one kernel for every shape.
+int attn_prefill_form(int hd) {
   static const int forced = [] {
-    const char* e = std::getenv("LLAMA_ATTN_KSTEP");
+    const char* e = std::getenv("LLAMA_ATTN_FORM");
     if (e == nullptr) return 0;
-    return std::strcmp(e, "64") == 0 ? 64 : std::strcmp(e, "128") == 0 ? 128 : 0;
+    return std::strcmp(e, "pair") == 0 ? 1 : std::strcmp(e, "k64") == 0 ? 2 : std::strcmp(e, "one") == 0 ? 3 : 0;
   }();
-  if (forced != 0) return forced == 64;
-  return hd < 128;
+  if (forced != 0) return forced;
+  return hd < 128 ? 2 : 1;
 }
 
 llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_cache* kv, int B, int L, int p0,
                                const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status,
                                const SeqTab* tab = nullptr, int Mtot = 0, int Tmax = 0) {
-  auto* kernel = attn_prefill_k64(d.head_dim) ? attn_prefill_k64_kernel : attn_prefill_kernel;
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(kernel), ATT_SMEM));
+  const int form = attn_prefill_form(d.head_dim);
+  auto* kernel = form == 3 ? attn_prefill_1t_kernel : form == 2 ? attn_prefill_k64_kernel : attn_prefill_kernel;
+  const int smem = form == 3 ? ATT1_SMEM : ATT_SMEM;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem));
   const int hd = d.head_dim;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
   const int T = tab != nullptr ? Tmax : p0 + L;
@@ -1007,8 +1011,8 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.hd = hd;
   // GQA (group >= 2): a CTA takes two query heads of one KV group over 128
   // query rows, sharing every K/V tile; MHA: one head over 256 query rows
-  p.head_pair = (d.n_heads / d.n_kv_heads) >= 2 ? 1 : 0;
-  p.n_qblocks = cdiv(L, p.head_pair ? 128 : 256);
+  p.head_pair = (form != 3 && (d.n_heads / d.n_kv_heads) >= 2) ? 1 : 0;
+  p.n_qblocks = cdiv(L, (form == 3 || p.head_pair) ? 128 : 256);
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
@@ -1017,7 +1021,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   // heaviest query blocks dispatched first (see the kernel)
   dim3 grid(p.head_pair ? d.n_heads / 2 : d.n_heads, B, p.n_qblocks);
   TRACE(K_ATTN_PREFILL, st);
-  CUDA_TRY(launch_k(kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
+  CUDA_TRY(launch_k(kernel, grid, form == 3 ? ATT1_THREADS : ATT_THREADS, smem, st, tq, tk, tv, p));
   LAUNCH_CHECK();
   return LLAMA_OK;
 }
