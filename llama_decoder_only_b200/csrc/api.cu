@@ -960,14 +960,13 @@ llama_status gemm_decode_q4(cudaStream_t st, const void* act, int M, int K, cons
 // Which prefill-attention kernel runs: 1 = attn_prefill_kernel (two query
 // tiles share each K/V tile, 128-key steps, one S buffer per tile), 2 =
 // attn_prefill_k64_kernel (the same with 64-key steps and two S buffers per
-// tile), 3 = attn_prefill_1t_kernel (one query tile, 128-key steps, two S
-// buffers).  Default: 2 for head_dim below 128, 1 at 128.
-// LLAMA_ATTN_FORM=pair | k64 | one takes one kernel for every shape.
+// tile).  Default: 2 for head_dim below 128, 1 at 128.
+// LLAMA_ATTN_FORM=pair | k64 takes one kernel for every shape.
 int attn_prefill_form(int hd) {
   static const int forced = [] {
     const char* e = std::getenv("LLAMA_ATTN_FORM");
     if (e == nullptr) return 0;
-    return std::strcmp(e, "pair") == 0 ? 1 : std::strcmp(e, "k64") == 0 ? 2 : std::strcmp(e, "one") == 0 ? 3 : 0;
+    return std::strcmp(e, "pair") == 0 ? 1 : std::strcmp(e, "k64") == 0 ? 2 : 0;
   }();
   if (forced != 0) return forced;
   return hd < 128 ? 2 : 1;
@@ -977,9 +976,8 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
                                const __nv_bfloat16* qkv, __nv_bfloat16* out, DevStatus* status,
                                const SeqTab* tab = nullptr, int Mtot = 0, int Tmax = 0) {
   const int form = attn_prefill_form(d.head_dim);
-  auto* kernel = form == 3 ? attn_prefill_1t_kernel : form == 2 ? attn_prefill_k64_kernel : attn_prefill_kernel;
-  const int smem = form == 3 ? ATT1_SMEM : ATT_SMEM;
-  TRY(ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem));
+  auto* kernel = form == 2 ? attn_prefill_k64_kernel : attn_prefill_kernel;
+  TRY(ensure_smem_attr(reinterpret_cast<const void*>(kernel), ATT_SMEM));
   const int hd = d.head_dim;
   const int qkvn = (d.n_heads + 2 * d.n_kv_heads) * hd;
   const int T = tab != nullptr ? Tmax : p0 + L;
@@ -1011,8 +1009,8 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   p.hd = hd;
   // GQA (group >= 2): a CTA takes two query heads of one KV group over 128
   // query rows, sharing every K/V tile; MHA: one head over 256 query rows
-  p.head_pair = (form != 3 && (d.n_heads / d.n_kv_heads) >= 2) ? 1 : 0;
-  p.n_qblocks = cdiv(L, (form == 3 || p.head_pair) ? 128 : 256);
+  p.head_pair = (d.n_heads / d.n_kv_heads) >= 2 ? 1 : 0;
+  p.n_qblocks = cdiv(L, p.head_pair ? 128 : 256);
   p.scale_log2 = kLog2e / sqrtf((float)hd);
   p.out = out;
   p.status = status;
@@ -1021,7 +1019,7 @@ llama_status attn_prefill_bf16(cudaStream_t st, const llama_dims& d, llama_kv_ca
   // heaviest query blocks dispatched first (see the kernel)
   dim3 grid(p.head_pair ? d.n_heads / 2 : d.n_heads, B, p.n_qblocks);
   TRACE(K_ATTN_PREFILL, st);
-  CUDA_TRY(launch_k(kernel, grid, form == 3 ? ATT1_THREADS : ATT_THREADS, smem, st, tq, tk, tv, p));
+  CUDA_TRY(launch_k(kernel, grid, ATT_THREADS, ATT_SMEM, st, tq, tk, tv, p));
   LAUNCH_CHECK();
   return LLAMA_OK;
 }

@@ -745,311 +745,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// One 128-row query tile per CTA with 128-key steps and two S buffers of 128
-// TMEM columns (S at 128 (s & 1), O at 256): the MMA warp computes S(s + 1)
-// while the softmax works on S(s), and issues P·V of step s and then S of
-// step s + 2 into the buffer P came from (in-order MMAs; the softmax, having
-// seen S(s) complete, knows every P·V up to s - 2 has completed).  The K / V
-// tiles serve one query tile only (twice the L2 -> shared-memory traffic of
-// the two-tile kernels), in exchange for a softmax that never waits on its
-// own MMAs.  192 threads: TMA producer, MMA issuer, one softmax warpgroup.
-constexpr int ATT1_THREADS = 192;
-constexpr int ATT1_SMEM = 1024 + ATT_TILE + ATT_SLOTS * ATT_TILE + 256;
-
-__global__ void __launch_bounds__(ATT1_THREADS, 1)
-    attn_prefill_1t_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, const AttnPrefillParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + ATT_TILE;                         // slot s at s * ATT_TILE
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + ATT_SLOTS * ATT_TILE);
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // heaviest query blocks first (grid.z), as in attn_prefill_kernel
-  const int qb = p.n_qblocks - 1 - blockIdx.z;
-  const int b = blockIdx.y;
-  const int h = blockIdx.x;
-  const int g = h / (p.nh / p.nkv);
-  const int hd = p.hd;
-  const int nreg = hd > 64 ? 2 : 1;
-  const int hd_pad = nreg * 64;
-  const int q_row0 = qb * 128;
-  int Ls = p.L, p0s = p.p0, row_base = b * p.L;
-  if (p.tab != nullptr) {
-    pdl_wait();   // the table is written by an earlier kernel
-    Ls = p.tab->len[b];
-    p0s = p.tab->p0[b];
-    row_base = p.tab->start[b];
-  }
-  const bool q_valid = q_row0 < Ls;
-  // 128-key steps with any key visible to the tile (0 for an empty tile)
-  const int n_st = q_valid ? (p0s + min(Ls, q_row0 + 128) - 1) / 128 + 1 : 0;
-
-  const uint32_t bar0 = smem_u32(bars);
-  const uint32_t q_full = bar0;
-  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ATT_SLOTS + s); };
-  auto s_full = [&](int u) { return bar0 + 8u * (1 + 2 * ATT_SLOTS + u); };
-  auto p_full = [&](int u) { return bar0 + 8u * (3 + 2 * ATT_SLOTS + u); };
-  auto pv_done = [&](int u) { return bar0 + 8u * (5 + 2 * ATT_SLOTS + u); };
-  const uint32_t drain = bar0 + 8u * (7 + 2 * ATT_SLOTS);
-
-  if (threadIdx.x == 0) {
-    abort_sh = 0;
-    mbar_init(q_full, 1);
-    for (int s = 0; s < ATT_SLOTS; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
-    }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(s_full(u), 1);
-      mbar_init(p_full(u), 128);
-      mbar_init(pv_done(u), 1);
-    }
-    mbar_init(drain, 1);
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_base_sh), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  pdl_wait();
-  const uint32_t tmem = tmem_base_sh;
-  WaitCtx wc{&abort_sh, p.status, p.limit_ns, 3};
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int last_fill[ATT_SLOTS];
-      for (int s = 0; s < ATT_SLOTS; ++s) last_fill[s] = -1;
-      if (q_valid) {
-        mbar_arrive_expect_tx(q_full, nreg * ATT_REGION);
-        for (int r = 0; r < nreg; ++r) {
-          if (p.tab != nullptr)
-            tma_load_2d(smem_u32(sQ + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64, row_base + q_row0);
-          else
-            tma_load_3d(smem_u32(sQ + r * ATT_REGION), &tmQ, q_full, h * hd + r * 64, q_row0, b);
-        }
-      } else {
-        mbar_arrive(q_full);
-      }
-      const int zkv = b * p.nkv + g;
-      for (int f = 0; f < 2 * n_st; ++f) {   // fill f: K_{f/2} (f even) or V_{f/2} (f odd)
-        const int s = f % ATT_SLOTS;
-        if (!mbar_wait(kv_empty(s), ((f / ATT_SLOTS) & 1) ^ 1u, wc, 1)) break;
-        const CUtensorMap* m = (f & 1) ? &tmV : &tmK;
-        mbar_arrive_expect_tx(kv_full(s), nreg * ATT_REGION);
-        for (int r = 0; r < nreg; ++r)
-          tma_load_3d(smem_u32(sKV + s * ATT_TILE + r * ATT_REGION), m, kv_full(s), r * 64, (f >> 1) * 128, zkv);
-        last_fill[s] = f;
-      }
-      mbar_wait(q_full, 0, wc, 9, false);
-      for (int s = 0; s < ATT_SLOTS; ++s)
-        if (last_fill[s] >= 0) mbar_wait(kv_full(s), (last_fill[s] / ATT_SLOTS) & 1, wc, 9, false);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t idesc_o = idesc_bf16_f32(128, hd_pad, 0, 1);   // V is MN-major
-      const int ksteps = hd / 16;
-      bool ok = mbar_wait(q_full, 0, wc, 2);
-      bool issued = false;
-      auto fill_ready = [&](int f) -> bool {
-        return mbar_wait(kv_full(f % ATT_SLOTS), (f / ATT_SLOTS) & 1, wc, 3);
-      };
-      // S(s) = Q K_s^T into buffer s & 1; K_s is then free once it completes
-      auto issue_s = [&](int s) -> bool {
-        if (!fill_ready(2 * s)) return false;
-        tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ);
-        const uint32_t aK = smem_u32(sKV + ((2 * s) % ATT_SLOTS) * ATT_TILE);
-        const uint32_t d = tmem + (uint32_t)((s & 1) * 128);
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * ATT_REGION + (ks & 3) * 32;
-          umma_bf16(d, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(aK + off, 16, 1024), idesc_s,
-                    ks > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full(s & 1));
-        umma_commit(kv_empty((2 * s) % ATT_SLOTS));
-        issued = true;
-        return true;
-      };
-      // O += P(s) V_s with P(s) the A operand in TMEM; V_s is then free
-      auto issue_pv = [&](int s) -> bool {
-        if (!mbar_wait(p_full(s & 1), (s >> 1) & 1, wc, 5)) return false;
-        if (!fill_ready(2 * s + 1)) return false;
-        tc_fence_after();
-        const uint32_t aV = smem_u32(sKV + ((2 * s + 1) % ATT_SLOTS) * ATT_TILE);
-        const uint32_t pa = tmem + (uint32_t)((s & 1) * 128);
-        for (int ks = 0; ks < 8; ++ks)   // 128 keys, 16 per MMA (8 TMEM columns of bf16 pairs)
-          umma_bf16_ts(tmem + 256, pa + 8 * ks, smem_desc_sw128(aV + ks * 16 * 128, ATT_REGION, 1024), idesc_o,
-                       (s > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(pv_done(s & 1));
-        umma_commit(kv_empty((2 * s + 1) % ATT_SLOTS));
-        return true;
-      };
-      for (int s = 0; s < 2 && s < n_st && ok; ++s) ok = issue_s(s);
-      for (int s = 0; ok && s < n_st; ++s) {
-        ok = issue_pv(s);
-        if (ok && s + 2 < n_st) ok = issue_s(s + 2);
-      }
-      if (issued) {
-        umma_commit(drain);
-        mbar_wait(drain, 0, wc, 8, false);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ softmax / correction / epilogue
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int tok = q_row0 + row;
-    const int pos = p0s + tok;
-    const int pos_min = p0s + q_row0;
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off;
-    const uint32_t tO = tmem + lane_off + 256;
-    float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int s = 0; s < n_st && ok; ++s) {
-      const int u = s & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full(u), (s >> 1) & 1, wc, 10))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t tSu = tS + (uint32_t)(u * 128);
-      float sv[4][32];
-      tmem_ld32(tSu + 0, sv[0]);
-      tmem_ld32(tSu + 32, sv[1]);
-      tmem_ld32(tSu + 64, sv[2]);
-      tmem_ld32(tSu + 96, sv[3]);
-      tmem_ld_wait();
-      if (s * 128 + 127 > pos_min) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (s * 128 + i > pos) sv[i >> 5][i & 31] = -INFINITY;
-      }
-      float mr[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) mr[k] = sv[0][k];
-#pragma unroll
-      for (int i = 4; i < 128; ++i) mr[i & 3] = fmaxf(mr[i & 3], sv[i >> 5][i & 31]);
-      const float mx = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3])) * p.scale_log2;
-      // the reference maximum moves only when it grew by more than 2^8
-      float alpha = 1.f;
-      const bool need = mx > m_used + 8.0f;
-      if (need) {
-        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mx);
-        m_used = mx;
-      }
-      const bool rescale = __any_sync(0xffffffffu, need && s > 0);
-      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-      const float sc = p.scale_log2;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
-      // P(s) over the first 64 columns of its S buffer (whose P·V of step
-      // s - 2 completed before S(s) did)
-#pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
-        uint32_t pw[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = ex2_approx(fmaf(sv[g4][2 * e], sc, -mref));
-          const float bb = ex2_approx(fmaf(sv[g4][2 * e + 1], sc, -mref));
-          ps[e & 3] += a + bb;
-          pw[e] = pack_bf16x2(a, bb);
-        }
-        tmem_st16u(tSu + 16 * g4, pw);
-      }
-      if (rescale) {
-        // O must hold every earlier step: wait for P·V of step s - 1
-        if (!__all_sync(0xffffffffu, mbar_wait(pv_done(u ^ 1), ((s - 1) >> 1) & 1, wc, 11))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        l *= alpha;
-        if (hd_pad == 128) {
-          float v0[32], v1[32], v2[32], v3[32];
-          tmem_ld32(tO + 0, v0);
-          tmem_ld32(tO + 32, v1);
-          tmem_ld32(tO + 64, v2);
-          tmem_ld32(tO + 96, v3);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            v0[i] *= alpha;
-            v1[i] *= alpha;
-            v2[i] *= alpha;
-            v3[i] *= alpha;
-          }
-          tmem_st32(tO + 0, v0);
-          tmem_st32(tO + 32, v1);
-          tmem_st32(tO + 64, v2);
-          tmem_st32(tO + 96, v3);
-        } else {
-          float v0[32], v1[32];
-          tmem_ld32(tO + 0, v0);
-          tmem_ld32(tO + 32, v1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            v0[i] *= alpha;
-            v1[i] *= alpha;
-          }
-          tmem_st32(tO + 0, v0);
-          tmem_st32(tO + 32, v1);
-        }
-      }
-      tmem_st_wait();
-      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      tc_fence_before();
-      mbar_arrive(p_full(u));
-    }
-    const int sl = n_st - 1;
-    if (ok && n_st > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done(sl & 1), (sl >> 1) & 1, wc, 12))) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((size_t)row_base + tok) * (size_t)(p.nh * hd) + (size_t)h * hd;
-      for (int c = 0; c < hd_pad; c += 32) {
-        float v[32];
-        tmem_ld32(tO + c, v);
-        tmem_ld_wait();
-        if (tok < Ls) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (c + 8 * q < hd) {
-              uint4 w;
-              w.x = pack_bf16x2(v[8 * q + 0] * inv, v[8 * q + 1] * inv);
-              w.y = pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv);
-              w.z = pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv);
-              w.w = pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv);
-              *reinterpret_cast<uint4*>(orow + c + 8 * q) = w;
-            }
-          }
-        }
-      }
-    }
-  }
-
-  pdl_trigger();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
 // ====================================================================== decode
 
 struct AttnDecodeParams {
