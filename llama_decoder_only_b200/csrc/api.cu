@@ -529,6 +529,20 @@ struct NormFuse {
   float eps;
 };
 
+// An RMSNorm computed by the decode GEMM that consumes it (cluster form): its
+// B operand is bf16(g * x * rstd(x row)), rstd from the sums of squares that
+// the residual GEMM which wrote x left in `ssq` ([tiles][BN]).
+struct NormB {
+  const float* x;
+  int ldx;
+  const float* g;
+  const float* ssq;
+  int tiles;
+  int dim;
+  float eps;
+  void* h;   // bf16 [rows][dim]: the normalised rows are also stored here (nullptr: not)
+};
+
 // Cluster-split form of a decode GEMM: one weight tile per cluster of p.cl_split CTAs.
 template <int BN, int EPI>
 llama_status launch_gemm_cl(const CUtensorMap& a, const CUtensorMap* w, const GemmParams& p, int grid,
@@ -782,7 +796,8 @@ llama_status prep_decode_gemm(const void* act, int M, int K, const WSeg* segs, i
 // it (published in `sk.partial` under `sk.flags`) and applies the epilogue.
 llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const WSeg* segs, int nseg, int epi,
                          void* out, int ldo, const float* resid, int ldr, SkScratch sk, DevStatus* status,
-                         int kind, const NormFuse* norm = nullptr) {
+                         int kind, const NormFuse* norm = nullptr, const NormB* nb = nullptr,
+                         bool ssq_out = false) {
   const int BN = swap_bn(M);
   const int KS = decode_ksub();
   GemmParams p;
@@ -797,10 +812,31 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
     p.ssq = sk.ssq;
     p.norm_ctr = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(sk.flags) - kWsFlagsOffset + kWsNormCtrOffset);
   }
+  if (ssq_out) {
+    // the sums of squares of the rows this GEMM finishes, for the next GEMM's RMSNorm
+    if (epi != EPI_RESID_F32 || norm != nullptr || p.n_tiles > kMaxNormTiles) return LLAMA_ERR_INVALID_ARG;
+    p.ssq = sk.ssq;
+    p.write_ssq = 1;
+  }
   if (const int cl = decode_cluster_split(p.n_tiles, p.num_kb, BN, KS, epi); cl > 0) {
     p.cl_split = cl;
     grid = p.n_tiles * cl;
     p.sk_grid = grid;
+  }
+  if (nb != nullptr) {
+    // the B operand from RMSNorm(x): the cluster form only, 16-byte aligned rows
+    if (p.cl_split == 0 || BN != 16 || (nb->ldx & 3) != 0 || !aligned16(nb->x) || !aligned16(nb->g) ||
+        nb->dim != K)
+      return LLAMA_ERR_INVALID_ARG;
+    p.nb_x = nb->x;
+    p.nb_ldx = nb->ldx;
+    p.nb_g = nb->g;
+    p.nb_ssq = nb->ssq;
+    p.nb_tiles = nb->tiles;
+    p.nb_dim = nb->dim;
+    p.nb_eps = nb->eps;
+    if (nb->h != nullptr && !aligned16(nb->h)) return LLAMA_ERR_INVALID_ARG;
+    p.nb_h = nb->h;
   }
   if (KS == 2) {
     switch (BN) {
@@ -821,9 +857,11 @@ llama_status gemm_decode(cudaStream_t st, const void* act, int M, int K, const W
 // Prefill-or-decode dispatch of one projection.
 llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int K, const WSeg* segs, int nseg,
                        int epi, void* out, int ldo, const float* resid, int ldr, SkScratch sk,
-                       DevStatus* status, int kind, const NormFuse* norm = nullptr) {
+                       DevStatus* status, int kind, const NormFuse* norm = nullptr, const NormB* nb = nullptr,
+                       bool ssq_out = false) {
   if (decode && M <= kSwapMaxTokens)
-    return gemm_decode(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, kind, norm);
+    return gemm_decode(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, sk, status, kind, norm, nb, ssq_out);
+  if (nb != nullptr || ssq_out) return LLAMA_ERR_INVALID_ARG;
   return gemm_prefill(st, act, M, K, segs, nseg, epi, out, ldo, resid, ldr, status, kind);
 }
 
@@ -833,6 +871,31 @@ llama_status gemm_bf16(cudaStream_t st, bool decode, const void* act, int M, int
 // RMSNorm kernel behind a programmatic-dependent launch (13B-shaped layer at
 // batch 16: 0.346 vs 0.344 ms per step; Phi-3-mini-shaped model at batch 8:
 // 3.38 vs 3.29 ms).
+// True when the decode GEMM over these weight segments takes the cluster form
+// (the same choice gemm_decode makes).
+bool decode_gemm_clustered(int M, int K, const WSeg* segs, int nseg, int epi) {
+  if (M > kSwapMaxTokens) return false;
+  const int KS = decode_ksub();
+  int tiles = 0;
+  if (epi == EPI_SWIGLU_BF16) {
+    tiles = cdiv(segs[0].rows, 64);
+  } else {
+    for (int s = 0; s < nseg; ++s) tiles += cdiv(segs[s].rows, 128);
+  }
+  return decode_cluster_split(tiles, cdiv(K, 64 * KS), swap_bn(M), KS, epi) > 0;
+}
+
+// The decode RMSNorms inside the GEMMs that consume them (cluster form; the
+// residual GEMM before leaves each row's sums of squares per column tile).
+// LLAMA_NORM_IN_GEMM=0 keeps them as kernels of their own.
+bool norm_in_gemm_enabled(const llama_dims& d, int M) {
+  static const bool on = [] {
+    const char* e = std::getenv("LLAMA_NORM_IN_GEMM");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on && d.dtype == LLAMA_BF16 && M <= 16 && d.dim % 8 == 0 && cdiv(d.dim, 128) <= kMaxNormTiles;
+}
+
 bool norm_fusable(const llama_dims& d, int M) {
   static const bool on = [] {
     const char* e = std::getenv("LLAMA_FUSE_NORM");
@@ -1381,9 +1444,13 @@ llama_status check_layer_call(const llama_dims* dims, const llama_layer_weights*
 // the next block's first one, or the model's final one -- run at the end of
 // the down GEMM into `next_out`; `h_ready`: this block's RMSNorm-1 output is
 // already in the workspace (the previous block's down GEMM wrote it).
+// x_ssq_ready: the workspace's sums of squares hold x_in's rows (written by
+// the previous block's down GEMM); ssq_next: this block's down GEMM writes
+// them for the next block.
 llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_kv_cache* kv, int B, int L,
                        const float* x_in, float* x_out, uint8_t* ws, const WsLayout& lay, cudaStream_t st,
-                       const float* next_norm = nullptr, void* next_out = nullptr, bool h_ready = false) {
+                       const float* next_norm = nullptr, void* next_out = nullptr, bool h_ready = false,
+                       bool x_ssq_ready = false, bool ssq_next = false) {
   DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   const int M = B * L;
   const int nh = d.n_heads, nkv = d.n_kv_heads, hd = d.head_dim;
@@ -1422,8 +1489,17 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       kv->length = p0 + L;
       return LLAMA_OK;
     }
+    // RMSNorms inside the consuming GEMMs (cluster form): RMSNorm-1 when the
+    // previous block left x_in's sums of squares, RMSNorm-2 from o_proj's
+    const bool nig = decode && !fuse_norm && norm_in_gemm_enabled(d, M);
+    const bool nig1 = nig && x_ssq_ready && decode_gemm_clustered(M, d.dim, segs, nseg, EPI_BF16);
+    WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
+    const bool nig2 = nig && decode_gemm_clustered(M, d.dim, sg, 2, EPI_SWIGLU_BF16);
+    const int ssq_tiles = cdiv(d.dim, 128);
+    const NormB nb1{x_in, d.dim, w.attn_norm, part.ssq, ssq_tiles, d.dim, d.eps, h};
+    const NormB nb2{x_out, d.dim, w.ffn_norm, part.ssq, ssq_tiles, d.dim, d.eps, h};
     // a2: RMSNorm-1 -> h (bf16)
-    if (!(fuse_norm && h_ready)) {
+    if (!(fuse_norm && h_ready) && !nig1) {
       TRACE(K_RMSNORM, st);
       // with RoPE fused into the QKV GEMM, it also writes each token's cos/sin row
       const RopeTab rt{fuse_rope ? rtab : nullptr, hd, L, p0, d.rope_theta, early_trigger()};
@@ -1440,7 +1516,8 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
       TRY(gemm_prefill(st, h, M, d.dim, segs, nseg, EPI_QKV_ROPE_BF16, qkv, qkvn, nullptr, 0, status, K_GEMM_QKV,
                        &ra));
     } else {
-      TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV));
+      TRY(gemm_bf16(st, decode, h, M, d.dim, segs, nseg, EPI_BF16, qkv, qkvn, nullptr, 0, part, status, K_GEMM_QKV,
+                    nullptr, nig1 ? &nb1 : nullptr));
       // a4: RoPE + KV append (decode with one key split: inside the attention kernel)
       if (!rope_in_attn) {
         TRACE(K_ROPE_APPEND, st);
@@ -1462,22 +1539,21 @@ llama_status run_layer(const llama_dims& d, const llama_layer_weights& w, llama_
     WSeg so{w.wo, d.dim, 0};
     const NormFuse n2{w.ffn_norm, h, d.eps};
     TRY(gemm_bf16(st, decode, att, M, nh * hd, &so, 1, EPI_RESID_F32, x_out, d.dim, x_in, d.dim, part, status,
-                  K_GEMM_O, fuse_norm ? &n2 : nullptr));
+                  K_GEMM_O, fuse_norm ? &n2 : nullptr, nullptr, nig2));
     // a8: RMSNorm-2 + gate_up + SiLU·mul
-    if (!fuse_norm) {
+    if (!fuse_norm && !nig2) {
       TRACE(K_RMSNORM, st);
       CUDA_TRY(launch_k(rmsnorm_kernel<bf>, M, rmsnorm_threads(d.dim), 0, st, x_out, d.dim, w.ffn_norm, h, M, d.dim,
                         d.eps, RopeTab{nullptr, 0, 0, 0, 0.f, early_trigger()}));
       LAUNCH_CHECK();
     }
-    WSeg sg[2] = {{w.w1, d.ffn_dim, 0}, {w.w3, d.ffn_dim, 0}};
     TRY(gemm_bf16(st, decode, h, M, d.dim, sg, 2, EPI_SWIGLU_BF16, mb, d.ffn_dim, nullptr, 0, part, status,
-                  K_GEMM_GATE_UP));
+                  K_GEMM_GATE_UP, nullptr, nig2 ? &nb2 : nullptr));
     // a9: down + residual (in place on x_out); decode: the next RMSNorm at its end
     WSeg sd{w.w2, d.dim, 0};
     const NormFuse nn{next_norm, next_out, d.eps};
     TRY(gemm_bf16(st, decode, mb, M, d.ffn_dim, &sd, 1, EPI_RESID_F32, x_out, d.dim, x_out, d.dim, part, status,
-                  K_GEMM_DOWN, (fuse_norm && next_norm != nullptr) ? &nn : nullptr));
+                  K_GEMM_DOWN, (fuse_norm && next_norm != nullptr) ? &nn : nullptr, nullptr, nig && ssq_next));
   } else {
     float* qkv = reinterpret_cast<float*>(ws + lay.qkv);
     float* h = reinterpret_cast<float*>(ws + lay.h);
@@ -2058,8 +2134,10 @@ llama_status model_forward(const llama_model* m, llama_kv_cache* const* caches, 
   for (int l = 0; l < m->n_layers; ++l) {
     const bool last = l + 1 == m->n_layers;
     const float* nn = chain ? (last ? m->final_norm : m->layers[l + 1].attn_norm) : nullptr;
+    // without the chained norms: each down GEMM leaves its rows' sums of
+    // squares for the next block's QKV GEMM, which then does RMSNorm-1 itself
     TRY(run_layer(d, m->layers[l], caches[l], batch, seq_len, xa, xb, ws, lay, st, nn, last ? hl_buf : hbuf,
-                  chain && l > 0));
+                  chain && l > 0, !chain && l > 0, !chain && !last));
     std::swap(xa, xb);
   }
   // a10: final norm + lm_head on the last row of each sequence + argmax

@@ -102,6 +102,18 @@ struct GemmParams {
   // k-blocks split over the cl_split CTAs of one thread-block cluster; ranks
   // 1.. store their fp32 pieces into rank 0's shared memory, which adds them
   int cl_split;
+  // decode residual GEMM: write ssq (as with norm_g) for an RMSNorm done by the next GEMM
+  int write_ssq;
+  // cluster form only: the B operand (token rows) is RMSNorm(x) computed here
+  // instead of loaded: bf16(nb_g * (x * rstd(x row))), rstd from the sums of
+  // squares nb_ssq[tile][BN] of nb_tiles column tiles written by the GEMM
+  // that produced x (nb_x == nullptr: B by TMA from the activation map)
+  const float* nb_x;
+  const float* nb_g;
+  const float* nb_ssq;
+  int nb_ldx, nb_tiles, nb_dim;
+  float nb_eps;
+  void* nb_h;          // bf16 [rows][nb_dim]: the normalised rows also stored here (by tile 0's cluster)
 };
 
 constexpr int GEMM_EPI_WARPS = 8;
@@ -409,7 +421,7 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
               reinterpret_cast<float*>(p.out)[o_idx] = v[j];
           }
         }
-        if (EPI == EPI_RESID_F32 && p.norm_g != nullptr) {
+        if (EPI == EPI_RESID_F32 && (p.norm_g != nullptr || p.write_ssq)) {
           // this tile's share of each token row's sum of squares: over the warp's
           // 32 rows by shuffles, then over the four warps of the same column half
           const int ew = (int)(threadIdx.x >> 5) - 2, lane = (int)(threadIdx.x & 31);
@@ -502,7 +514,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                    const GemmParams p) {
   constexpr bool PAIR = !SWAP;            // tile mode runs 256 x BN tiles on CTA pairs
   static_assert(KS == 1 || SWAP, "k sub-blocks are a decode (stream-K) form");
-  static_assert(!CL || (SWAP && BN == 16), "the cluster split is a decode form of 16 token columns");
+  static_assert(!CL || (SWAP && BN == 16 && KS == 2), "the cluster split is a decode form of 16 token columns");
   using C = GemmCfg<BN, PAIR, KS, CL>;
   constexpr int STAGES = C::STAGES;
   constexpr int WROWS = SWAP ? 128 : BN;  // weight rows per tile
@@ -526,6 +538,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
   const uint32_t epi_bar = bar0 + 8u * (2 * STAGES + 5);
   const uint32_t red_bar = bar0 + 8u * (2 * STAGES + 6);
+  // cluster form with the RMSNorm in the prologue: the epilogue threads write B
+  const bool norm_b = CL && p.nb_x != nullptr;
   static_assert(8 * (2 * STAGES + 7) <= 256, "barrier block");
   // cluster split: the other ranks' pieces, in rank 0's shared memory
   float* cl_buf = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256 + C::EXCH_BYTES);
@@ -533,7 +547,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_sh = 0;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      // (+ one arrival per epilogue thread when they write the B operand)
+      mbar_init(full_bar(s), norm_b ? 1 + 32 * GEMM_EPI_WARPS : 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -547,7 +562,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmAct);
+    if (!norm_b) tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmW0);
     if (p.nseg > 1) tma_prefetch_desc(&tmW1);
     if (p.nseg > 2) tma_prefetch_desc(&tmW2);
@@ -613,14 +628,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         GemmItem item;
         while (skip < STAGES && it.next(item)) {
           for (int kb = item.kb0; kb < item.kb1 && skip < STAGES; ++kb) {
-            mbar_arrive_expect_tx(full_bar(skip), C::STAGE_BYTES);
+            mbar_arrive_expect_tx(full_bar(skip), norm_b ? C::A_BYTES : C::STAGE_BYTES);
             load_weight_swap(smem_u32(smem + skip * C::STAGE_BYTES), full_bar(skip), item.tile, kb);
             pre_kb[skip++] = kb;
           }
         }
         pdl_wait();
         for (int s = 0; s < skip; ++s) {
-          load_act_swap(smem_u32(smem + s * C::STAGE_BYTES) + C::A_BYTES, full_bar(s), pre_kb[s]);
+          if (!norm_b) load_act_swap(smem_u32(smem + s * C::STAGE_BYTES) + C::A_BYTES, full_bar(s), pre_kb[s]);
           filled_parity[s] = 0;
         }
         stage = skip % STAGES;
@@ -654,9 +669,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
           if (SWAP) {
-            mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+            mbar_arrive_expect_tx(full_bar(stage), norm_b ? C::A_BYTES : C::STAGE_BYTES);
             load_weight_swap(sa, full_bar(stage), wtile, kb);
-            load_act_swap(sb, full_bar(stage), kb);
+            if (!norm_b) load_act_swap(sb, full_bar(stage), kb);
           } else {
             // both CTAs' bytes land on rank 0's full barrier, which rank 0 arms
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
@@ -758,6 +773,84 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_wait(epi_bar, epi_phase, wc, 7);
       epi_phase ^= 1u;
     };
+    if constexpr (CL) {
+      if (norm_b) {
+        // B operand = RMSNorm of the token rows ([MLX-13B] 4. RMSNorm;
+        // [DeepDive] LLaMARMSNorm), written into each stage as TMA would lay
+        // it out (128-byte rows, 16-byte chunk c of row r at c ^ (r & 7)):
+        // thread e takes token row e / 16 and 8 consecutive k of each k-block.
+        const int e = (int)threadIdx.x - 64;
+        static_assert(BN * 16 == 32 * GEMM_EPI_WARPS, "one 16-byte chunk per thread and k-block");
+        const int brow = e >> 4, sub = (e >> 3) & 1, chunk = e & 7;
+        const bool brow_ok = brow < p.act_rows;
+        const uint32_t boff = (uint32_t)(C::A_BYTES + sub * C::B_SUB + brow * 128 + ((chunk ^ (brow & 7)) << 4));
+        // the first weight tile's cluster covers every k once: it also stores the rows
+        const bool store_h = p.nb_h != nullptr && (int)blockIdx.x < p.cl_split;
+        GemmIter bit;
+        bit.init(p, true);
+        GemmItem bitem;
+        const bool have = bit.next(bitem);   // the cluster form gives a CTA one item
+        const int kbeg = have ? bitem.kb0 : 0, kend = have ? bitem.kb1 : 0;
+        // this thread's x and g for a k-block, three k-blocks ahead of the stores
+        constexpr int AHEAD = 3;
+        float4 xq[AHEAD][2], gq[AHEAD][2];
+        auto fetch = [&](int kb, float4 (&xs)[2], float4 (&gs)[2]) {
+          const int k0 = (kb * KS + sub) * 64 + chunk * 8;
+          if (kb < kend && brow_ok && k0 < p.K) {
+            const float4* xr = reinterpret_cast<const float4*>(p.nb_x + (size_t)brow * p.nb_ldx + k0);
+            const float4* gr = reinterpret_cast<const float4*>(p.nb_g + k0);
+            xs[0] = __ldcg(xr);
+            xs[1] = __ldcg(xr + 1);
+            gs[0] = __ldg(gr);
+            gs[1] = __ldg(gr + 1);
+          } else {
+            xs[0] = xs[1] = gs[0] = gs[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        };
+#pragma unroll
+        for (int a = 0; a < AHEAD; ++a) fetch(kbeg + a, xq[a], gq[a]);
+        // rstd of each token row from the producing GEMM's per-tile sums of
+        // squares: 16 threads per row (lanes of one half-warp) split the tiles
+        {
+          const int r = e >> 4, part = e & 15;
+          float ss = 0.f;
+          for (int t = part; t < p.nb_tiles; t += 16) ss += __ldcg(p.nb_ssq + (size_t)t * BN + r);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (part == 0) rstd_sh[r] = rsqrtf(ss / (float)p.nb_dim + p.nb_eps);
+        }
+        epi_sync();
+        const float rs = rstd_sh[brow];
+        for (int n = 0; n < kend - kbeg; ++n) {
+          const int kb = kbeg + n, stage = n % STAGES;
+          if (!mbar_wait(empty_bar(stage), ((uint32_t)(n / STAGES) & 1u) ^ 1u, wc, 13)) break;
+          const int k0 = (kb * KS + sub) * 64 + chunk * 8;
+          uint4 o;
+          o.x = pack_bf16x2(gq[0][0].x * (xq[0][0].x * rs), gq[0][0].y * (xq[0][0].y * rs));
+          o.y = pack_bf16x2(gq[0][0].z * (xq[0][0].z * rs), gq[0][0].w * (xq[0][0].w * rs));
+          o.z = pack_bf16x2(gq[0][1].x * (xq[0][1].x * rs), gq[0][1].y * (xq[0][1].y * rs));
+          o.w = pack_bf16x2(gq[0][1].z * (xq[0][1].z * rs), gq[0][1].w * (xq[0][1].w * rs));
+          if (store_h && brow_ok && k0 < p.K)
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.nb_h) + (size_t)brow * p.nb_dim + k0) = o;
+          const uint32_t dst = smem_u32(smem + stage * C::STAGE_BYTES) + boff;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+                       : "memory");
+          // generic-proxy writes, read by the tensor core through the async proxy
+          // (one arrival per thread: measured faster than a warp sync and one
+          // arrival per warp)
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(full_bar(stage));
+#pragma unroll
+          for (int a = 0; a + 1 < AHEAD; ++a) {
+            xq[a][0] = xq[a + 1][0];
+            xq[a][1] = xq[a + 1][1];
+            gq[a][0] = gq[a + 1][0];
+            gq[a][1] = gq[a + 1][1];
+          }
+          fetch(kb + AHEAD, xq[AHEAD - 1], gq[AHEAD - 1]);
+        }
+      }
+    }
     int abuf = 0;
     uint32_t aphase = 0;
     GemmIter it;
