@@ -423,13 +423,27 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
         }
         if (EPI == EPI_RESID_F32 && (p.norm_g != nullptr || p.write_ssq)) {
           // this tile's share of each token row's sum of squares: over the warp's
-          // 32 rows by shuffles, then over the four warps of the same column half
+          // 32 rows by a halving butterfly (each step a lane keeps half of its
+          // 16 sums and adds its partner's copy of them: 16 shuffles, after
+          // which lanes 2j and 2j + 1 hold token j's sum), then over the four
+          // warps of the same column half
           const int ew = (int)(threadIdx.x >> 5) - 2, lane = (int)(threadIdx.x & 31);
+          float sq[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float q = warp_sum(xo[j] * xo[j]);
-            if (lane == j) red[ew][j] = q;
+          for (int j = 0; j < 16; ++j) sq[j] = xo[j] * xo[j];
+#pragma unroll
+          for (int st = 0; st < 4; ++st) {
+            const int W = 8 >> st, bit = 16 >> st;
+            const bool upper = (lane & bit) != 0;
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+              const float send = upper ? sq[i] : sq[i + W];
+              const float keep = upper ? sq[i + W] : sq[i];
+              sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+            }
           }
+          sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], 1);
+          if ((lane & 1) == 0) red[ew][lane >> 1] = sq[0];
           epi_sync();
           const int e = (int)threadIdx.x - 64;
           if (e < 32) {
@@ -441,7 +455,10 @@ __device__ __forceinline__ void streamk_epilogue(const GemmParams& p, const Gemm
               p.ssq[(size_t)item.tile * BN + c2] = q;
             }
           }
-          epi_sync();
+          // red is reused by the next column block or work item, and the fused
+          // RMSNorm counts the tile after this barrier; a cluster-form CTA's
+          // last block with the sums only has neither
+          if (!(CL && p.norm_g == nullptr && c0 + 32 >= BN)) epi_sync();
         }
       }
     }
